@@ -1,0 +1,189 @@
+"""Pins of the oracle's MoE steps: brute-force loops on tiny inputs, closed
+forms and invariants.  CPU only."""
+
+import itertools
+
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import moe as M
+
+from test_oracle_formats import grid_weights
+
+
+def _bf16(rng, shape, std=1.0):
+    return F.bf16_encode_rne(rng.normal(0, std, shape))
+
+
+# --------------------------------------------------------------------------- GEMV / GEMM
+
+
+@pytest.mark.parametrize("rows,K,n", [(16, 256, 1), (16, 512, 3), (32, 256, 2)])
+def test_stq_gemv_brute_force_from_structure(rows, K, n):
+    # y[t, r] = sum over groups, over non-zero lanes, of sign * d * x, built
+    # directly from (zero lane, sign, d) without the byte layout.
+    rng = np.random.default_rng(rows + K + n)
+    w, z, s, d = grid_weights(rng, rows, K)
+    xb = _bf16(rng, (n, K))
+    x = F.bf16_decode(xb)
+    y, S = M.stq1_gemv(F.stq1_pack(w), rows, K, xb)
+    for t in range(n):
+        for r in range(rows):
+            acc = 0.0
+            sabs = 0.0
+            for j in range(K // 4):
+                for l in range(4):
+                    if l == z[r, j]:
+                        continue
+                    term = s[r, j, l] * d[r, (4 * j) // 256] * x[t, 4 * j + l]
+                    acc += term
+                    sabs += abs(term)
+            assert abs(y[t, r] - acc) <= 1e-12 * (sabs + 1)
+            assert abs(S[t, r] - sabs) <= 1e-12 * (sabs + 1)
+
+
+def test_stq_gemv_one_hot_and_all_positive():
+    rows, K = 16, 512
+    # d = 1, all-positive rows with zero lane 3: y = sum of x over lanes 0..2 of every group
+    code = np.full((rows, K // 256, 64), 8 * 3, dtype=np.int64)
+    dbits = np.full((rows, K // 256), F.fp16_encode_rne(1.0), np.uint16)
+    packed = F.stq1_layout(code, dbits)
+    rng = np.random.default_rng(11)
+    xb = _bf16(rng, (1, K))
+    x = F.bf16_decode(xb)[0]
+    y, _ = M.stq1_gemv(packed, rows, K, xb)
+    ref = sum(x[k] for k in range(K) if k % 4 != 3)
+    assert np.allclose(y[0], ref, rtol=0, atol=1e-12)
+    # one-hot x picks one weight column exactly
+    w, *_ = grid_weights(rng, rows, K)
+    b = F.stq1_pack(w)
+    for k in [0, 1, 255, 256, 511]:
+        e = np.zeros((1, K))
+        e[0, k] = 1.0
+        yk, _ = M.stq1_gemv(b, rows, K, F.bf16_encode_rne(e))
+        assert np.array_equal(yk[0], w[:, k].astype(np.float64))
+
+
+def test_w4a8_gemm_brute_force():
+    rng = np.random.default_rng(12)
+    N, K, Mt = 4, 64, 3
+    wc = rng.integers(0, 256, (N, K // 2)).astype(np.uint8)
+    ws = rng.integers(118, 128, (N, K // 32)).astype(np.uint8)
+    ac, asc = F.mxfp8_quantize(F.bf16_decode(_bf16(rng, (Mt, K))))
+    Y, S = M.w4a8_gemm(wc, ws, ac, asc, N, K)
+    for m in range(Mt):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                byte = wc[n, k // 2]
+                nib = (byte >> (4 * (k % 2))) & 15
+                wv = F.e2m1_decode(np.uint8(nib)) * 2.0 ** (int(ws[n, k // 32]) - 127)
+                av = F.e4m3_decode(ac[m, k]) * 2.0 ** (int(asc[m, k // 32]) - 127)
+                acc += wv * av
+            assert abs(Y[m, n] - acc) <= 1e-12 * (abs(acc) + 1)
+
+
+# --------------------------------------------------------------------------- router
+
+
+def test_router_softmax_topk_properties():
+    rng = np.random.default_rng(13)
+    T, H, E, k = 5, 64, 32, 8
+    xb = _bf16(rng, (T, H))
+    wr = _bf16(rng, (E, H), 0.5)
+    ids, w, p = M.router_topk(xb, wr, k)
+    assert np.allclose(p.sum(axis=1), 1.0, atol=1e-12)
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-12)
+    for t in range(T):
+        # brute force: sort (prob desc, id asc)
+        order = sorted(range(E), key=lambda e: (-p[t, e], e))[:k]
+        assert list(ids[t]) == order
+        logits = F.bf16_decode(xb[t]) @ F.bf16_decode(wr).T
+        q = np.exp(logits - logits.max())
+        assert np.allclose(p[t], q / q.sum(), rtol=1e-12)
+    # relabelling the experts relabels the choice
+    perm = rng.permutation(E)
+    ids2, w2, _ = M.router_topk(xb, wr[perm], k)
+    assert np.array_equal(perm[ids2], ids) and np.allclose(w2, w)
+
+
+def test_router_ties_go_to_lower_id():
+    T, H, E = 1, 32, 16
+    xb = F.bf16_encode_rne(np.ones((T, H)))
+    wr = F.bf16_encode_rne(np.zeros((E, H)))
+    ids, w, _ = M.router_topk(xb, wr, 8)
+    assert list(ids[0]) == list(range(8)) and np.allclose(w, 1 / 8)
+
+
+# --------------------------------------------------------------------------- permute
+
+
+def test_permute_matches_stable_sort_by_loops():
+    rng = np.random.default_rng(14)
+    for T, E, k in [(1, 4, 2), (7, 16, 8), (33, 256, 8)]:
+        ids = rng.integers(0, E, (T, k))
+        counts, offsets, perm, inv = M.permute(ids, E)
+        flat = ids.reshape(-1)
+        ref = sorted(range(T * k), key=lambda p: (flat[p], p))
+        assert list(perm) == ref
+        assert counts.sum() == T * k and offsets[0] == 0 and offsets[-1] == T * k
+        assert np.all(np.diff(offsets) == counts)
+        for e in range(E):
+            assert counts[e] == sum(1 for v in flat if v == e)
+            assert all(flat[perm[i]] == e for i in range(offsets[e], offsets[e + 1]))
+        assert np.array_equal(perm[inv], np.arange(T * k))
+
+
+def test_permute_rejects_bad_ids():
+    with pytest.raises(ValueError):
+        M.permute(np.array([[0, 256]]), 256)
+
+
+# --------------------------------------------------------------------------- SwiGLU and combine
+
+
+def test_silu_closed_forms():
+    v = np.linspace(-30, 30, 601)
+    # silu(v) - silu(-v) = v(sigmoid(v) + sigmoid(-v)) = v
+    assert np.allclose(M.silu(v) - M.silu(-v), v, atol=1e-12)
+    assert M.silu(0.0) == 0.0
+    assert abs(M.silu(1.0) - 1.0 / (1.0 + np.exp(-1.0))) < 1e-15
+    assert abs(M.silu(40.0) - 40.0) < 1e-12 and abs(M.silu(-800.0)) == 0.0
+
+
+def test_swiglu_rounds_inputs_to_f32():
+    g = np.array([1.0 + 2.0 ** -30])
+    u = np.array([2.0])
+    assert M.swiglu(g, u)[0] == M.silu(1.0) * 2.0
+
+
+def test_combine_brute_force():
+    rng = np.random.default_rng(15)
+    T, k, H = 3, 4, 5
+    Y = rng.normal(size=(T * k, H))
+    S = np.abs(Y)
+    w = rng.random((T, k))
+    sh = rng.normal(size=(T, H))
+    res = rng.normal(size=(T, H))
+    y, s = M.combine(Y, S, w, sh, None, res)
+    for t, h in itertools.product(range(T), range(H)):
+        ref = sum(w[t, j] * Y[t * k + j, h] for j in range(k)) + sh[t, h] + res[t, h]
+        assert abs(y[t, h] - ref) < 1e-12
+        assert s[t, h] >= abs(y[t, h]) - 1e-12
+
+
+def test_expert_ffn_stage_consistency():
+    rng = np.random.default_rng(16)
+    I, H, n = 16, 256, 2
+    wg, *_ = grid_weights(rng, I, H)
+    wu, *_ = grid_weights(rng, I, H)
+    wd, *_ = grid_weights(rng, H, I * 16)
+    wd = wd[:, :I]
+    X = F.bf16_decode(_bf16(rng, (n, H)))
+    out = M.expert_ffn_bf16h(wg, wu, wd, X)
+    g = X @ wg.astype(np.float64).T
+    u = X @ wu.astype(np.float64).T
+    h = F.bf16_decode(F.bf16_encode_rne(M.silu(g.astype(np.float32).astype(np.float64)) * u.astype(np.float32)))
+    assert np.array_equal(out["h"], h)
+    assert np.allclose(out["y"], h @ wd.astype(np.float64).T, rtol=1e-13, atol=1e-15)

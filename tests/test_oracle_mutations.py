@@ -1,0 +1,87 @@
+"""Plant plausible mistakes in the oracle (on the CPU, via monkeypatch) and check
+that the pins catch each one.  This shows the pins constrain the oracle rather
+than restate it."""
+
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import moe as M
+
+import test_oracle_formats as TF
+import test_oracle_moe as TM
+
+
+def _fails(fn, *args):
+    with pytest.raises(AssertionError):
+        fn(*args)
+
+
+def test_reversed_sign_order_is_caught(monkeypatch):
+    monkeypatch.setattr(F, "_NZ_LANES", F._NZ_LANES[:, ::-1].copy())
+    _fails(TF.test_codebook_is_zero_lane_and_ordered_signs)
+    _fails(TF.test_stq_layout_second_reading)
+
+
+def test_wrong_scale_boundary_is_caught(monkeypatch):
+    orig = F.mxfp8_scale_exponent
+
+    def off_by_one(amax):
+        fm, E = np.frexp(np.asarray(amax, np.float64))
+        m, e = 2.0 * fm, E - 1
+        k = np.where(m < 1.75, e - 8, e - 7)          # '<' instead of '<='
+        return np.where(np.asarray(amax) == 0, 127, np.clip(k + 127, 0, 254)).astype(np.int64)
+
+    monkeypatch.setattr(F, "mxfp8_scale_exponent", off_by_one)
+    _fails(TF.test_mxfp8_quant_exhaustive_bf16_own_amax)
+    monkeypatch.setattr(F, "mxfp8_scale_exponent", orig)
+
+
+def test_round_half_away_is_caught(monkeypatch):
+    def rta(v, frac_bits, emin):
+        v = np.asarray(v, np.float64)
+        a = np.abs(v)
+        _, E = np.frexp(a)
+        q = np.ldexp(1.0, np.maximum(E - 1, emin) - frac_bits)
+        return np.copysign(np.floor(a / q + 0.5) * q, v)
+
+    monkeypatch.setattr(F, "round_to_binary", rta)
+    _fails(TF.test_e2m1_rounding_brute_force)
+    _fails(TF.test_bf16_rne_matches_library_cast)
+
+
+def test_transposed_gemv_is_caught(monkeypatch):
+    def transposed(W, X):
+        W = np.asarray(W, np.float64)
+        X = np.asarray(X, np.float64)
+        Wt = W.reshape(W.shape[1], W.shape[0]) if W.shape[0] != W.shape[1] else W.T
+        return X @ Wt.T.reshape(W.shape).T, np.abs(X) @ np.abs(W).T
+
+    monkeypatch.setattr(M, "matvec_with_scale", transposed)
+    _fails(TM.test_stq_gemv_brute_force_from_structure, 16, 256, 1)
+
+
+def test_dropped_slot_in_combine_is_caught(monkeypatch):
+    orig = M.combine
+
+    def drop_last(Y, S, w, shared=None, shared_S=None, residual=None):
+        w = np.array(w, np.float64)
+        w[:, -1] = 0.0
+        return orig(Y, S, w, shared, shared_S, residual)
+
+    monkeypatch.setattr(M, "combine", drop_last)
+    _fails(TM.test_combine_brute_force)
+
+
+def test_unstable_permute_is_caught(monkeypatch):
+    def unstable(ids, E):
+        flat = np.asarray(ids, np.int64).reshape(-1)
+        counts = np.bincount(flat, minlength=E)
+        offsets = np.concatenate([[0], np.cumsum(counts)])
+        perm = np.argsort(-np.arange(flat.size))[np.argsort(flat[::-1], kind="stable")]
+        inv = np.empty_like(perm)
+        inv[perm] = np.arange(perm.size)
+        return counts, offsets, perm, inv
+
+    monkeypatch.setattr(M, "permute", unstable)
+    _fails(TM.test_permute_matches_stable_sort_by_loops)
