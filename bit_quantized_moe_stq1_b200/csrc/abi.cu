@@ -1,0 +1,59 @@
+// Status strings, version and error-word access of the C ABI.
+#include "moe_internal.cuh"
+
+extern "C" const char* stq_status_string(stq_status s) {
+  switch (s) {
+    case STQ_OK: return "STQ_OK";
+    case STQ_ERR_INVALID_ARG: return "STQ_ERR_INVALID_ARG";
+    case STQ_ERR_SHAPE: return "STQ_ERR_SHAPE";
+    case STQ_ERR_ALIGN: return "STQ_ERR_ALIGN";
+    case STQ_ERR_NONFINITE: return "STQ_ERR_NONFINITE";
+    case STQ_ERR_CUDA: return "STQ_ERR_CUDA";
+    case STQ_ERR_DEVICE: return "STQ_ERR_DEVICE";
+    case STQ_ERR_WORKSPACE: return "STQ_ERR_WORKSPACE";
+    case STQ_ERR_TIMEOUT: return "STQ_ERR_TIMEOUT";
+    case STQ_ERR_UNSUPPORTED: return "STQ_ERR_UNSUPPORTED";
+    default: return "STQ_ERR_UNKNOWN";
+  }
+}
+
+extern "C" int32_t stq_abi_version(void) { return STQMOE_ABI_VERSION; }
+
+extern "C" stq_status stq_read_error(int32_t* err, stq_stream_t stream) {
+  if (err == nullptr) return STQ_ERR_INVALID_ARG;
+  cudaStream_t s = stq_cuda_stream(stream);
+  int32_t host = 0;
+  if (cudaMemcpyAsync(&host, err, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess) return STQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return STQ_ERR_CUDA;
+  if (host != 0) {
+    if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return STQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return STQ_ERR_CUDA;
+  }
+  return host;
+}
+
+extern "C" stq_status moe_get_device_error(void* workspace, stq_stream_t stream) {
+  if (workspace == nullptr) return STQ_ERR_INVALID_ARG;
+  return stq_read_error(static_cast<int32_t*>(workspace), stream);
+}
+
+static stq_timing* g_timing = nullptr;
+
+extern "C" stq_status stq_set_timing(stq_timing* t) {
+  g_timing = t;
+  return STQ_OK;
+}
+
+StqTimed::StqTimed(int kind, cudaStream_t st) : s(st), slot(-1) {
+  stq_timing* t = g_timing;
+  if (t == nullptr || t->count >= t->capacity) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+  slot = t->count++;
+  t->kinds[slot] = kind;
+  cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * slot]), st);
+}
+
+StqTimed::~StqTimed() {
+  if (slot >= 0 && g_timing != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(g_timing->events[2 * slot + 1]), s);
+}

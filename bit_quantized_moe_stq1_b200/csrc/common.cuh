@@ -1,0 +1,70 @@
+// Shared device/host helpers for the stqmoe kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/stqmoe.h"
+
+#define STQ_HOST_CHECK(cond, code) \
+  do {                             \
+    if (!(cond)) return (code);    \
+  } while (0)
+
+static inline bool stq_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static inline stq_status stq_launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
+}
+
+static inline cudaStream_t stq_cuda_stream(stq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// First error wins: only replace a 0 word.
+__device__ __forceinline__ void stq_set_error(int32_t* err, int32_t code) {
+  if (err != nullptr) atomicCAS(err, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// float -> bf16 bits, round to nearest even (the library conversion intrinsic).
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// D = A * B + D for one m16n8k16 bf16 tile with FP32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+
+// Round an FP32 value to the bf16 grid and back (for intermediates stored as bf16).
+__device__ __forceinline__ float round_bf16(float f) { return __bfloat162float(__float2bfloat16_rn(f)); }
+
+// Timing hook (abi.cu): bracket one kernel launch with events when installed.
+struct StqTimed {
+  StqTimed(int kind, cudaStream_t s);
+  ~StqTimed();
+  cudaStream_t s;
+  int slot;
+};
+
+template <typename T>
+__host__ __device__ constexpr T ceil_div(T a, T b) { return (a + b - 1) / b; }
+
+static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

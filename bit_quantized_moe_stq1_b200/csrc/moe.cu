@@ -1,0 +1,610 @@
+// MoE layer: router, token-to-expert grouping, expert GEMVs with fused SwiGLU,
+// shared expert, and the top-k combine.
+//
+// Shapes: "Hy4-preview-FlashMoE-STQ1_0", "Package details" (hidden 6144, MoE
+// intermediate 2048, 256 routed experts, top-8, one shared expert).  The router
+// (softmax, top-k, renormalise), the shared BF16 expert and the SwiGLU between
+// gate/up and down are this library's reading of "run the experts"; the pages give
+// the shapes and formats only.
+//
+// Data flow of moe_expert_forward (one stream, launches in this order):
+//   permute   ids [T,k] -> counts, offsets, perm (pair at each sorted position),
+//             inv (sorted position of each pair), list of touched experts
+//   [MXFP4]   x -> MXFP8 (see gemm_mx.cu)
+//   gate/up   per touched expert and 128-feature tile: g, u (FP32) -> h = silu(g)u
+//             -> h[pos, I] (bf16 for STQ1_0; MXFP8 for MXFP4); the shared expert is
+//             a second set of CTAs (bf16 weights) writing h[P + t, I]
+//   down      per touched expert and 256-row tile: Y[pos, H] (FP32); shared -> Y[P+t]
+//   combine   y[t] = sum_s w[t,s] Y[inv[t,s]] (+ Y[P+t]) (+ x[t]) in slot order
+
+#include "gemv.cuh"
+#include "moe_internal.cuh"
+
+namespace {
+
+using namespace stq;
+
+// ----------------------------------------------------------------------------- block scan
+
+// Exclusive scan of one value per thread over a 1024-thread block; returns the
+// exclusive prefix and writes the total to *total (shared).
+__device__ __forceinline__ int block_excl_scan_1024(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int s = wsum[lane];
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, si, o);
+      if (lane >= o) si += n;
+    }
+    wsum[lane] = si - s;
+    if (lane == 31) *total = si;
+  }
+  __syncthreads();
+  const int r = incl - v + wsum[warp];
+  __syncthreads();
+  return r;
+}
+
+// ----------------------------------------------------------------------------- permute
+
+__global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                           MoeWs ws) {
+  extern __shared__ int32_t sm[];
+  int32_t* cnt = sm;             // [E]
+  int32_t* cursor = sm + E;      // [E]
+  int32_t* whist = sm + 2 * E;   // [32][E]
+  __shared__ int wsum[32];
+  __shared__ int total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += 1024) cnt[e] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int p = tid; p < P; p += 1024) {
+    const int e = ids[p];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1); else bad = true;
+  }
+  if (__syncthreads_or(bad) && tid == 0) stq_set_error(ws.err, STQ_ERR_DEVICE);
+  // offsets (exclusive scan of counts) and the touched-expert list; E <= 1024
+  const int v = tid < E ? cnt[tid] : 0;
+  const int ex = block_excl_scan_1024(v, wsum, &total);
+  if (tid < E) {
+    cursor[tid] = ex;
+    ws.offsets[tid] = ex;
+    ws.counts[tid] = v;
+  }
+  if (tid == 0) ws.offsets[E] = total;
+  const int flag = (tid < E && v > 0) ? 1 : 0;
+  const int fx = block_excl_scan_1024(flag, wsum, &total);
+  if (flag) ws.tlist[fx] = tid;
+  if (tid == 0) *ws.ntouched = total;
+  __syncthreads();
+  // stable placement: chunks of 1024 pairs in pair order
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0; base < P; base += 1024) {
+    const int p = base + tid;
+    const bool valid = p < P;
+    const int e = valid ? ids[p] : -1;
+    const bool ok = valid && e >= 0 && e < E;
+    for (int i = tid; i < 32 * E; i += 1024) whist[i] = 0;
+    __syncthreads();
+    const int key = ok ? e : -1 - lane;
+    const unsigned peers = __match_any_sync(kFull, key);
+    const int rank = __popc(peers & lt);
+    if (ok && rank == 0) whist[warp * E + e] = __popc(peers);
+    __syncthreads();
+    for (int e2 = tid; e2 < E; e2 += 1024) {
+      int run = cursor[e2];
+#pragma unroll 4
+      for (int w = 0; w < 32; ++w) {
+        const int c = whist[w * E + e2];
+        whist[w * E + e2] = run;
+        run += c;
+      }
+      cursor[e2] = run;
+    }
+    __syncthreads();
+    if (ok) {
+      const int pos = whist[warp * E + e] + rank;
+      ws.perm[pos] = p;
+      ws.inv[p] = pos;
+    } else if (valid) {
+      ws.inv[p] = -1;
+    }
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------- router
+
+__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc = fmaf(bf16_bits_to_float(aw[i] & 0xFFFFu), bf16_bits_to_float(bw[i] & 0xFFFFu), acc);
+    acc = fmaf(bf16_bits_to_float(aw[i] >> 16), bf16_bits_to_float(bw[i] >> 16), acc);
+  }
+  return acc;
+}
+
+// logits[t, e] = sum_h x[t, h] wr[e, h] (FP32).  CTA = 8 warps over 4 experts; warp
+// w takes expert 4*blockIdx + (w & 3) and half (w >> 2) of H.
+__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                            const uint16_t* __restrict__ wr, int T, int H, int E,
+                                                            float* __restrict__ logits) {
+  __shared__ float red[2][4][8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 4 + (warp & 3), half = warp >> 2;
+  const int hh = H / 2;
+  const int k0 = half * hh, k1 = k0 + hh;
+  for (int t0 = 0; t0 < T; t0 += 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (e < E) {
+      for (int k = k0 + lane * 8; k < k1; k += 256) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wr + size_t(e) * H + k);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (t0 + j < T) acc[j] = dot8_bf16(wv, *reinterpret_cast<const uint4*>(x + size_t(t0 + j) * H + k), acc[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(kFull, acc[j], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) red[half][warp & 3][j] = acc[j];
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int ei = threadIdx.x >> 3, j = threadIdx.x & 7;
+      const int ee = blockIdx.x * 4 + ei;
+      if (ee < E && t0 + j < T) logits[size_t(t0 + j) * E + ee] = red[0][ei][j] + red[1][ei][j];
+    }
+    __syncthreads();
+  }
+}
+
+// One warp per token: softmax over E (max-shifted exp), top-k by probability with
+// ties to the lower id, weights renormalised over the chosen k.
+__global__ void router_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ ids,
+                                   float* __restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  constexpr int kMaxPer = 32;  // E <= 1024
+  float p[kMaxPer];
+  const int per = (E + 31) / 32;
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < kMaxPer; ++j) {
+    const int e = lane + 32 * j;
+    p[j] = (j < per && e < E) ? logits[size_t(t) * E + e] : -INFINITY;
+    m = fmaxf(m, p[j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+#pragma unroll
+  for (int j = 0; j < kMaxPer; ++j) p[j] = (p[j] == -INFINITY) ? -1.f : expf(p[j] - m);
+  float sel_sum = 0.f;
+  for (int r = 0; r < k; ++r) {
+    float bp = -1.f;
+    int bid = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+      const int e = lane + 32 * j;
+      if (p[j] > bp) { bp = p[j]; bid = e; }   // ascending e within a lane: ties keep the lower id
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float op = __shfl_xor_sync(kFull, bp, o);
+      const int oid = __shfl_xor_sync(kFull, bid, o);
+      if (op > bp || (op == bp && oid < bid)) { bp = op; bid = oid; }
+    }
+    if ((bid & 31) == lane) p[bid >> 5] = -1.f;  // remove the chosen expert
+    sel_sum += bp;
+    if (lane == 0) {
+      ids[size_t(t) * k + r] = bid;
+      w[size_t(t) * k + r] = bp;
+    }
+  }
+  __syncwarp();
+  if (lane < k) w[size_t(t) * k + lane] = w[size_t(t) * k + lane] / sel_sum;
+}
+
+// ----------------------------------------------------------------------------- expert GEMVs
+
+// Shared expert, gate/up: CTA = 16 features; the CTA's four warps split H.
+__device__ __forceinline__ void shared_gateup(const MoeArgs& a, int bid, float (*red)[2][4][4][32]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int f0 = bid * 16;
+  const int kq = a.H / 4, k0 = warp * kq, k1 = k0 + kq;
+  const uint16_t* rowg[2] = {a.sg + size_t(f0 + g) * a.H, a.su + size_t(f0 + g) * a.H};
+  for (int t0 = 0; t0 < a.T; t0 += 32) {
+    const uint16_t* xr[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int tok = t0 + 8 * c + g;
+      xr[c] = tok < a.T ? a.x + size_t(tok) * a.H : nullptr;
+    }
+    float acc[2][4][4] = {};
+    bf16_warp_gemv<2, 4>(rowg, a.H, k0, k1, xr, acc);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[warp][i][c][j][lane] = acc[i][c][j];
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float gs = ((red[0][0][c][j][lane] + red[1][0][c][j][lane]) + red[2][0][c][j][lane]) + red[3][0][c][j][lane];
+          const float us = ((red[0][1][c][j][lane] + red[1][1][c][j][lane]) + red[2][1][c][j][lane]) + red[3][1][c][j][lane];
+          const int tok = t0 + 8 * c + 2 * t + (j & 1);
+          const int f = f0 + g + 8 * (j >> 1);
+          if (tok < a.T) a.h[size_t(a.P + tok) * a.I + f] = float_to_bf16_bits(silu_f32(gs) * us);
+        }
+    }
+    __syncthreads();
+  }
+}
+
+// Shared expert, down: CTA = 16 rows of H; the four warps split I.
+__device__ __forceinline__ void shared_down(const MoeArgs& a, int bid, float (*red)[2][4][4][32]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int r0 = bid * 16;
+  const int kq = a.I / 4, k0 = warp * kq, k1 = k0 + kq;
+  const uint16_t* rowg[1] = {a.sd + size_t(r0 + g) * a.I};
+  for (int t0 = 0; t0 < a.T; t0 += 32) {
+    const uint16_t* xr[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int tok = t0 + 8 * c + g;
+      xr[c] = tok < a.T ? a.h + size_t(a.P + tok) * a.I : nullptr;
+    }
+    float acc[1][4][4] = {};
+    bf16_warp_gemv<1, 4>(rowg, a.I, k0, k1, xr, acc);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) red[warp][0][c][j][lane] = acc[0][c][j];
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float ys = ((red[0][0][c][j][lane] + red[1][0][c][j][lane]) + red[2][0][c][j][lane]) + red[3][0][c][j][lane];
+          const int tok = t0 + 8 * c + 2 * t + (j & 1);
+          const int r = r0 + g + 8 * (j >> 1);
+          if (tok < a.T) a.Y[size_t(a.P + tok) * a.H + r] = ys;
+        }
+    }
+    __syncthreads();
+  }
+}
+
+// Routed STQ1_0 gate/up + SwiGLU.  CTA = 128 features of one touched expert; warp =
+// 32 features = 2 gate tiles + 2 up tiles over all of H.
+__global__ void __launch_bounds__(128) moe_gateup_stq_kernel(MoeArgs a) {
+  __shared__ float red[4][2][4][4][32];
+  int bid = blockIdx.x;
+  if (bid < a.n_shared_cta) {
+    shared_gateup(a, bid, red);
+    return;
+  }
+  bid -= a.n_shared_cta;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int per_expert = a.I / 128;
+  const int slot = bid / per_expert, ct = bid % per_expert;
+  if (slot >= *a.ntouched) return;
+  const int e = a.tlist[slot];
+  const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+  const int nb = a.H / 256;
+  const size_t mat = size_t(a.I) * nb * 42;
+  const int f0 = ct * 128 + warp * 32;
+  const uint8_t* gb = a.wg + size_t(e) * mat;
+  const uint8_t* ub = a.wu + size_t(e) * mat;
+  const size_t tstride = size_t(nb) * kTileBlockBytes;
+  const uint8_t* tb[4] = {gb + size_t(f0 / 16) * tstride, gb + size_t(f0 / 16 + 1) * tstride,
+                          ub + size_t(f0 / 16) * tstride, ub + size_t(f0 / 16 + 1) * tstride};
+  const uint32_t lut = lut_entry(lane);
+  for (int c0 = 0; c0 < cnt; c0 += 8) {
+    const int j = c0 + g;
+    const uint16_t* xrow = j < cnt ? a.x + size_t(a.perm[pos0 + j] / a.k) * a.H : nullptr;
+    float acc[4][4] = {};
+    stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
+#pragma unroll
+    for (int tp = 0; tp < 2; ++tp)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = c0 + 2 * t + (q & 1);
+        const int f = f0 + 16 * tp + g + 8 * (q >> 1);
+        if (col < cnt) a.h[size_t(pos0 + col) * a.I + f] = float_to_bf16_bits(silu_f32(acc[tp][q]) * acc[tp + 2][q]);
+      }
+  }
+}
+
+// Routed STQ1_0 down.  CTA = 256 rows of H of one touched expert; warp = 4 tiles.
+__global__ void __launch_bounds__(128) moe_down_stq_kernel(MoeArgs a) {
+  __shared__ float red[4][2][4][4][32];
+  int bid = blockIdx.x;
+  if (bid < a.n_shared_cta) {
+    shared_down(a, bid, red);
+    return;
+  }
+  bid -= a.n_shared_cta;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int per_expert = a.H / 256;
+  const int slot = bid / per_expert, ct = bid % per_expert;
+  if (slot >= *a.ntouched) return;
+  const int e = a.tlist[slot];
+  const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+  const int nb = a.I / 256;
+  const size_t mat = size_t(a.H) * nb * 42;
+  const int r0 = ct * 256 + warp * 64;
+  const uint8_t* db = a.wd + size_t(e) * mat;
+  const size_t tstride = size_t(nb) * kTileBlockBytes;
+  const uint8_t* tb[4] = {db + size_t(r0 / 16) * tstride, db + size_t(r0 / 16 + 1) * tstride,
+                          db + size_t(r0 / 16 + 2) * tstride, db + size_t(r0 / 16 + 3) * tstride};
+  const uint32_t lut = lut_entry(lane);
+  for (int c0 = 0; c0 < cnt; c0 += 8) {
+    const int j = c0 + g;
+    const uint16_t* xrow = j < cnt ? a.h + size_t(pos0 + j) * a.I : nullptr;
+    float acc[4][4] = {};
+    stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = c0 + 2 * t + (q & 1);
+        const int r = r0 + 16 * i + g + 8 * (q >> 1);
+        if (col < cnt) a.Y[size_t(pos0 + col) * a.H + r] = acc[i][q];
+      }
+  }
+}
+
+// ----------------------------------------------------------------------------- combine
+
+__global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __restrict__ Y,
+                                   const int32_t* __restrict__ inv, const float* __restrict__ topk_w, int has_shared,
+                                   const uint16_t* __restrict__ resid, void* __restrict__ y, int out_fp32) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int h4 = H / 4;
+  if (idx >= int64_t(T) * h4) return;
+  const int t = int(idx / h4), c = int(idx % h4);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < k; ++s) {
+    const int pos = inv[size_t(t) * k + s];
+    if (pos < 0) continue;
+    const float w = topk_w[size_t(t) * k + s];
+    const float4 v = reinterpret_cast<const float4*>(Y + size_t(pos) * H)[c];
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
+  }
+  if (has_shared) {
+    const float4 v = reinterpret_cast<const float4*>(Y + size_t(P + t) * H)[c];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  if (resid != nullptr) {
+    const uint2 r = reinterpret_cast<const uint2*>(resid + size_t(t) * H)[c];
+    acc.x += bf16_bits_to_float(r.x & 0xFFFFu);
+    acc.y += bf16_bits_to_float(r.x >> 16);
+    acc.z += bf16_bits_to_float(r.y & 0xFFFFu);
+    acc.w += bf16_bits_to_float(r.y >> 16);
+  }
+  if (out_fp32) {
+    reinterpret_cast<float4*>(static_cast<float*>(y) + size_t(t) * H)[c] = acc;
+  } else {
+    const uint32_t lo = uint32_t(float_to_bf16_bits(acc.x)) | (uint32_t(float_to_bf16_bits(acc.y)) << 16);
+    const uint32_t hi = uint32_t(float_to_bf16_bits(acc.z)) | (uint32_t(float_to_bf16_bits(acc.w)) << 16);
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + size_t(t) * H)[c] = make_uint2(lo, hi);
+  }
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------------------- host side
+
+MoeWsLayout moe_ws_layout(const moe_desc& d) {
+  MoeWsLayout L{};
+  const size_t T = size_t(d.T), H = size_t(d.H), I = size_t(d.I), E = size_t(d.E), P = T * size_t(d.k);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
+  L.err = take(sizeof(int32_t));
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.tlist = take(E * 4);
+  L.ntouched = take(4);
+  L.perm = take(P * 4);
+  L.inv = take(P * 4);
+  L.h = take((P + T) * I * 2);
+  L.Y = take((P + T) * H * 4);
+  L.xq = take(T * H);
+  L.xs = take(T * (H / 32));
+  L.hq = take(P * I);
+  L.hs = take(P * (I / 32));
+  L.total = o;
+  return L;
+}
+
+MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
+  uint8_t* b = static_cast<uint8_t*>(workspace);
+  MoeWs w;
+  w.err = reinterpret_cast<int32_t*>(b + L.err);
+  w.counts = reinterpret_cast<int32_t*>(b + L.counts);
+  w.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+  w.tlist = reinterpret_cast<int32_t*>(b + L.tlist);
+  w.ntouched = reinterpret_cast<int32_t*>(b + L.ntouched);
+  w.perm = reinterpret_cast<int32_t*>(b + L.perm);
+  w.inv = reinterpret_cast<int32_t*>(b + L.inv);
+  w.h = reinterpret_cast<uint16_t*>(b + L.h);
+  w.Y = reinterpret_cast<float*>(b + L.Y);
+  w.xq = b + L.xq;
+  w.xs = b + L.xs;
+  w.hq = b + L.hq;
+  w.hs = b + L.hs;
+  return w;
+}
+
+static bool desc_ok(const moe_desc* d) {
+  return d && d->T >= 0 && d->H > 0 && d->I > 0 && d->E > 0 && d->E <= 1024 && d->k > 0 && d->k <= 32 &&
+         d->k <= d->E;
+}
+
+extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
+  if (!desc_ok(d)) return 0;
+  return moe_ws_layout(*d).total;
+}
+
+extern "C" size_t moe_workspace_offset(const moe_desc* d, int32_t region) {
+  if (!desc_ok(d)) return ~size_t(0);
+  const MoeWsLayout L = moe_ws_layout(*d);
+  switch (region) {
+    case STQ_WS_COUNTS: return L.counts;
+    case STQ_WS_OFFSETS: return L.offsets;
+    case STQ_WS_PERM: return L.perm;
+    case STQ_WS_INV: return L.inv;
+    case STQ_WS_TLIST: return L.tlist;
+    case STQ_WS_NTOUCHED: return L.ntouched;
+    case STQ_WS_H: return L.h;
+    case STQ_WS_Y: return L.Y;
+    case STQ_WS_XQ: return L.xq;
+    case STQ_WS_XS: return L.xs;
+    case STQ_WS_HQ: return L.hq;
+    case STQ_WS_HS: return L.hs;
+    default: return ~size_t(0);
+  }
+}
+
+stq_status moe_launch_permute(const int32_t* ids, int P, int E, const MoeWs& ws, cudaStream_t s) {
+  const size_t smem = size_t(34) * E * sizeof(int32_t);
+  static int configured_smem = 0;  // dynamic shared memory opt-in (process-wide, set once per size growth)
+  if (int(smem) > configured_smem) {
+    if (cudaFuncSetAttribute(moe_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return STQ_ERR_CUDA;
+    configured_smem = int(smem);
+  }
+  StqTimed tm(STQ_K_PERMUTE, s);
+  moe_permute_kernel<<<1, 1024, smem, s>>>(ids, P, E, ws);
+  return stq_launch_status();
+}
+
+stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const float* topk_w, bool has_shared,
+                              const uint16_t* x, void* y, cudaStream_t s) {
+  const int64_t n = int64_t(d.T) * (d.H / 4);
+  if (n == 0) return STQ_OK;
+  StqTimed tm(STQ_K_COMBINE, s);
+  moe_combine_kernel<<<unsigned(ceil_div<int64_t>(n, 256)), 256, 0, s>>>(
+      d.T, d.H, d.k, P, ws.Y, ws.inv, topk_w, has_shared ? 1 : 0, d.add_residual ? x : nullptr, y, d.out_fp32);
+  return stq_launch_status();
+}
+
+extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, const int32_t* topk_ids,
+                                         const float* topk_w, const moe_weights* w, void* y, void* workspace,
+                                         size_t ws_bytes, stq_stream_t stream) {
+  STQ_HOST_CHECK(desc_ok(d) && w && x && topk_ids && topk_w && y && workspace, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(w->fmt == STQ_FMT_STQ1_0 || w->fmt == STQ_FMT_MXFP4, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(w->gate && w->up && w->down, STQ_ERR_INVALID_ARG);
+  const bool has_shared = w->sh_gate != nullptr;
+  STQ_HOST_CHECK(!has_shared || (w->sh_up && w->sh_down), STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(d->H % 256 == 0 && d->I % 256 == 0, STQ_ERR_SHAPE);
+  if (w->fmt == STQ_FMT_MXFP4) STQ_HOST_CHECK(w->gate_sc && w->up_sc && w->down_sc, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(y) && stq_aligned16(w->gate) && stq_aligned16(w->up) &&
+                     stq_aligned16(w->down) && stq_aligned16(topk_ids) && stq_aligned16(topk_w),
+                 STQ_ERR_ALIGN);
+  STQ_HOST_CHECK((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, STQ_ERR_ALIGN);
+  if (has_shared)
+    STQ_HOST_CHECK(stq_aligned16(w->sh_gate) && stq_aligned16(w->sh_up) && stq_aligned16(w->sh_down), STQ_ERR_ALIGN);
+  const MoeWsLayout L = moe_ws_layout(*d);
+  STQ_HOST_CHECK(ws_bytes >= L.total, STQ_ERR_WORKSPACE);
+  if (d->T == 0) return STQ_OK;
+  cudaStream_t s = stq_cuda_stream(stream);
+  const MoeWs ws = moe_ws_pointers(workspace, L);
+  const int P = d->T * d->k;
+  stq_status st = moe_launch_permute(topk_ids, P, d->E, ws, s);
+  if (st != STQ_OK) return st;
+
+  MoeArgs a{};
+  a.T = d->T; a.H = d->H; a.I = d->I; a.E = d->E; a.k = d->k; a.P = P;
+  a.x = x;
+  a.wg = w->gate; a.wu = w->up; a.wd = w->down;
+  a.gsc = w->gate_sc; a.usc = w->up_sc; a.dsc = w->down_sc;
+  a.sg = w->sh_gate; a.su = w->sh_up; a.sd = w->sh_down;
+  a.offsets = ws.offsets; a.perm = ws.perm; a.tlist = ws.tlist; a.ntouched = ws.ntouched;
+  a.h = ws.h; a.Y = ws.Y;
+  a.xq = ws.xq; a.xs = ws.xs; a.hq = ws.hq; a.hs = ws.hs;
+  a.err = ws.err;
+  const int slots = d->E < P ? d->E : P;
+
+  if (w->fmt == STQ_FMT_STQ1_0) {
+    a.n_shared_cta = has_shared ? d->I / 16 : 0;
+    {
+      StqTimed tm(STQ_K_GATE_UP, s);
+      moe_gateup_stq_kernel<<<unsigned(a.n_shared_cta + slots * (d->I / 128)), 128, 0, s>>>(a);
+    }
+    if ((st = stq_launch_status()) != STQ_OK) return st;
+    a.n_shared_cta = has_shared ? d->H / 16 : 0;
+    {
+      StqTimed tm(STQ_K_DOWN, s);
+      moe_down_stq_kernel<<<unsigned(a.n_shared_cta + slots * (d->H / 256)), 128, 0, s>>>(a);
+    }
+    if ((st = stq_launch_status()) != STQ_OK) return st;
+  } else {
+    st = moe_mx_experts(a, slots, has_shared, s);
+    if (st != STQ_OK) return st;
+  }
+  return moe_launch_combine(*d, P, ws, topk_w, has_shared, x, y, s);
+}
+
+extern "C" stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T, int32_t H, int32_t E,
+                                      int32_t k, float* logits, int32_t* topk_ids, float* topk_w,
+                                      stq_stream_t stream) {
+  STQ_HOST_CHECK(x && w_router && logits && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(H % 16 == 0, STQ_ERR_SHAPE);
+  STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
+  if (T == 0) return STQ_OK;
+  cudaStream_t s = stq_cuda_stream(stream);
+  {
+    StqTimed tm(STQ_K_ROUTER_LOGITS, s);
+    router_logits_kernel<<<unsigned(ceil_div(E, 4)), 256, 0, s>>>(x, w_router, T, H, E, logits);
+  }
+  stq_status st = stq_launch_status();
+  if (st != STQ_OK) return st;
+  {
+    StqTimed tm(STQ_K_ROUTER_TOPK, s);
+    router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+  }
+  return stq_launch_status();
+}
+
+extern "C" stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E, int32_t* counts,
+                                  int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tlist, int32_t* ntouched,
+                                  int32_t* err, stq_stream_t stream) {
+  STQ_HOST_CHECK(counts && offsets && tlist && ntouched, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(T >= 0 && k > 0 && E > 0 && E <= 1024, STQ_ERR_INVALID_ARG);
+  const int64_t P64 = int64_t(T) * k;
+  STQ_HOST_CHECK(P64 < (int64_t(1) << 30), STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(P64 == 0 || (topk_ids && perm && inv), STQ_ERR_INVALID_ARG);
+  MoeWs ws{};
+  ws.err = err; ws.counts = counts; ws.offsets = offsets; ws.perm = perm; ws.inv = inv;
+  ws.tlist = tlist; ws.ntouched = ntouched;
+  return moe_launch_permute(topk_ids, int(P64), E, ws, stq_cuda_stream(stream));
+}

@@ -1,0 +1,50 @@
+// Internal structures shared by the MoE translation units (not part of the ABI).
+#pragma once
+
+#include "common.cuh"
+
+struct MoeWsLayout {
+  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, total;
+};
+
+// Device pointers into the caller's workspace.
+struct MoeWs {
+  int32_t* err;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* tlist;
+  int32_t* ntouched;
+  int32_t* perm;
+  int32_t* inv;
+  uint16_t* h;   // [(P+T), I] bf16: routed pairs (sorted order) then shared-expert tokens
+  float* Y;      // [(P+T), H] fp32
+  uint8_t* xq;   // [T, H]     MXFP8 codes of x
+  uint8_t* xs;   // [T, H/32]
+  uint8_t* hq;   // [P, I]     MXFP8 codes of h (MXFP4 experts)
+  uint8_t* hs;   // [P, I/32]
+};
+
+// Kernel arguments (by value).
+struct MoeArgs {
+  int T, H, I, E, k, P;
+  const uint16_t* x;
+  const uint8_t *wg, *wu, *wd;     // routed experts (STQ1_0 bytes or MXFP4 codes)
+  const uint8_t *gsc, *usc, *dsc;  // MXFP4 scales
+  const uint16_t *sg, *su, *sd;    // shared expert, bf16
+  const int32_t *offsets, *perm, *tlist, *ntouched;
+  uint16_t* h;
+  float* Y;
+  uint8_t *xq, *xs, *hq, *hs;
+  int32_t* err;
+  int n_shared_cta;
+};
+
+MoeWsLayout moe_ws_layout(const moe_desc& d);
+MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L);
+
+// Routed MXFP4 experts (+ the shared BF16 expert): gate/up, SwiGLU, down.
+stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStream_t s);
+
+// BF16 -> MXFP8 quantisation launch (pack.cu).
+stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales,
+                                     cudaStream_t s);

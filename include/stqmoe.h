@@ -1,0 +1,250 @@
+/*
+ * stqmoe.h - C ABI of libstqmoe.so: the routed-expert FFN of one MoE layer over
+ * packed low-bit expert weights, on one NVIDIA B200 (sm_100a).
+ *
+ * Two weight formats (the problem as the pages state it):
+ *
+ *  STQ1_0  3:4 sparse ternary.  "Hy4-preview-GGUF", section 3 "STQ1_0 and the
+ *          mixed-precision strategy": weights {-d, 0, +d}, exactly one zero per
+ *          four lanes, one FP16 scale per 256 weights, 42 bytes per 256 weights
+ *          (1.3125 bpw).  "Hy4-preview-FlashMoE-STQ1_0", "How the STQ1_0 packing
+ *          works": 64 four-weight groups per block, 4 x 2^3 = 32 patterns, five
+ *          bits each.  The byte layout is this library's own (GGML type 43's
+ *          literal codebook is not given on the pages; no byte compatibility is
+ *          claimed):
+ *            pattern c = 8*z + s: z = zero lane, bit n of s = sign of the n-th
+ *            non-zero lane counted upward (1 = negative); weight = d * (0 | +-1);
+ *            group j of 256-block b covers k = 256*b + 4*j + lane.
+ *            Matrix [rows, K] (rows % 16 == 0, K % 256 == 0) = tiles of 16 rows,
+ *            each tile = K/256 tile-blocks of 672 bytes (16 rows x 42 bytes):
+ *              [0,32)    word g (g=0..7) = fp16 d(row g) | fp16 d(row g+8) << 16
+ *              [32,544)  lane L: words 0..3 of its 160-bit code stream at 32+16L
+ *              [544,672) lane L: word 4 at 544+4L
+ *            lane L = 4g+t holds rows g, g+8 and groups j = 16t+s (s = 0..15);
+ *            code i = 2s+h (row g+8h) sits at stream bits [5i, 5i+5).
+ *  MXFP4 x MXFP8 ("W4A8").  "Hy4-preview-SF-WFP4AFP8", "Quant Diff": routed
+ *          experts are FP4 E2M1 weights with FP8 E4M3 activations, group 32,
+ *          UE8M0 scales.  Weights [rows, K]: codes [rows][K/2] (element 2i in the
+ *          low nibble) + scales [rows][K/32]; activations: codes [rows][K] +
+ *          scales [rows][K/32].  Element encodings follow the OCP MX spec.
+ *
+ * Conventions (every entry point):
+ *  - Pointers named in the argument lists are DEVICE pointers owned by the
+ *    caller, unless the name ends in _host.  The library allocates nothing and
+ *    frees nothing.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream) and return
+ *    after enqueueing.  Argument errors are detected on the host before any
+ *    launch; on error nothing is launched and outputs are untouched.
+ *  - Device-side data errors (non-finite weights in a pack, an expert id out of
+ *    range, a bounded wait that ran out) are recorded in a caller-owned device
+ *    int32 "error word" (first error wins); read it with stq_read_error().
+ *  - Device pointers must be 16-byte aligned; sizes are element counts.
+ *  - Not thread-safe per workspace / error word.
+ */
+#ifndef STQMOE_H
+#define STQMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* stq_stream_t; /* same type as cudaStream_t */
+typedef int32_t stq_status;
+
+enum {
+  STQ_OK = 0,
+  STQ_ERR_INVALID_ARG = -1, /* null pointer, bad enum, negative size */
+  STQ_ERR_SHAPE = -2,       /* K % 256 (STQ1_0), K % 32 (MX), rows % 16, H/I mismatch */
+  STQ_ERR_ALIGN = -3,       /* a device pointer is not 16-byte aligned */
+  STQ_ERR_NONFINITE = -4,   /* pack: NaN/Inf weight, or an STQ block amax above 65504 */
+  STQ_ERR_CUDA = -5,        /* a CUDA runtime call failed (launch, attribute) */
+  STQ_ERR_DEVICE = -6,      /* device-detected: expert id out of range */
+  STQ_ERR_WORKSPACE = -7,   /* workspace smaller than moe_workspace_bytes() */
+  STQ_ERR_TIMEOUT = -8,     /* device-detected: a bounded wait ran out */
+  STQ_ERR_UNSUPPORTED = -9  /* valid request this build does not implement */
+};
+
+/* Human-readable name of a status code (static string). */
+const char* stq_status_string(stq_status s);
+
+/* ABI version of this header (bumped on any signature or layout change). */
+#define STQMOE_ABI_VERSION 1
+int32_t stq_abi_version(void);
+
+/* Synchronise `stream`, return the error word's value and reset it to 0.
+ * `err` is a device int32.  Returns STQ_ERR_CUDA if the synchronisation fails. */
+stq_status stq_read_error(int32_t* err, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Packing.  Sources: "Hy4-preview-GGUF" section 3 (upstream quantiser: d = amax, */
+/* zero the lane of smallest |w|) for STQ1_0; "Hy4-preview-SF-WFP4AFP8", "Quant   */
+/* Diff" for MXFP4 (E2M1 g32, UE8M0).                                             */
+/* ------------------------------------------------------------------------- */
+
+/* w: float32 [rows, K] row-major -> out: rows*K/256*42 bytes in the STQ1_0 layout
+ * above.  Per 256-block d = fp16_rne(max |w|); per group the zero goes to the
+ * first lane of smallest |w|, the other lanes keep sign(w).  d == 0 gives all
+ * codes 0.  Exact (pack(unpack(b)) == b) on canonical bytes.  A NaN/Inf weight or
+ * a block amax > 65504 sets STQ_ERR_NONFINITE in *err (err may be NULL).
+ * rows % 16 == 0, K % 256 == 0. */
+stq_status stq1_pack(const float* w, int64_t rows, int64_t K, uint8_t* out,
+                     int32_t* err, stq_stream_t stream);
+
+/* STQ1_0 bytes -> float32 [rows, K]: +-d on non-zero lanes (sign applied to d),
+ * +0 on the zero lane.  Bit-exact. */
+stq_status stq1_unpack(const uint8_t* in, int64_t rows, int64_t K, float* w,
+                       stq_stream_t stream);
+
+/* w: float32 [rows, K] -> codes [rows, K/2], scales [rows, K/32].  Per 32 along
+ * K: e = clamp(k + 127, 0, 254) with k the smallest integer such that
+ * max|w| <= 6 * 2^k (e = 127 for an all-zero group); codes = E2M1 round to
+ * nearest even of w * 2^-k, sign of w kept (-0 -> code 8).  NaN/Inf weights set
+ * STQ_ERR_NONFINITE in *err.  K % 32 == 0. */
+stq_status mxfp4_pack(const float* w, int64_t rows, int64_t K, uint8_t* codes,
+                      uint8_t* scales, int32_t* err, stq_stream_t stream);
+
+/* codes/scales -> float32 [rows, K] = e2m1(code) * 2^(e-127) rounded to binary32
+ * (overflow -> +-inf; e = 255 -> NaN).  Bit-exact. */
+stq_status mxfp4_unpack(const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                        int64_t K, float* w, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Activation quantisation BF16 -> MXFP8 (E4M3 g32, UE8M0).  Source: the       */
+/* "Hy4-preview-SF-WFP4AFP8" recipe (weight_fp4_activation_fp8, group 32,      */
+/* ue8m0 / e4m3); scale rule: smallest power of two putting the group amax     */
+/* <= 448.                                                                      */
+/* ------------------------------------------------------------------------- */
+
+/* x: bf16 bits [rows, K] -> codes [rows, K], scales [rows, K/32].  e as for MXFP4
+ * with 448 in place of 6; codes = E4M3 RNE of x * 2^-k including subnormals, sign
+ * kept (negative values that round to zero give 0x80).  A group holding NaN/Inf
+ * gets e = 255 and codes 0x7F.  Bit-exact.  K % 32 == 0. */
+stq_status mxfp8_quantize_bf16(const uint16_t* x, int64_t rows, int64_t K,
+                               uint8_t* codes, uint8_t* scales, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Single-matrix products (the two single-matrix workloads).                  */
+/* ------------------------------------------------------------------------- */
+
+/* y[n, r] = sum_k W[r, k] x[n, k] (FP32 accumulate) for an STQ1_0 matrix W
+ * [rows, K] and bf16 activations x [n, K]; y float32 [n, rows].  Tolerance
+ * |y - y_ref| <= 1e-3 * sum_k |W x| + 1e-5.  rows % 16 == 0, K % 256 == 0. */
+stq_status stq1_gemv(const uint8_t* W, int64_t rows, int64_t K, const uint16_t* x,
+                     int64_t n, float* y, stq_stream_t stream);
+
+/* y[m, n] = sum_k a[m, k] w[n, k] for MXFP4 weights w [N, K] and MXFP8
+ * activations a [M, K] (tcgen05 block-scaled MMA, FP32 accumulate); y float32
+ * [M, N].  `err` (device int32, may be NULL) records STQ_ERR_TIMEOUT if a
+ * pipeline wait ran out.  N % 128 == 0, K % 128 == 0. */
+stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales, int64_t N,
+                     int64_t K, const uint8_t* a_codes, const uint8_t* a_scales,
+                     int64_t M, float* y, int32_t* err, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* MoE layer.  Shapes: "Hy4-preview-FlashMoE-STQ1_0", "Package details"        */
+/* (hidden 6144, MoE intermediate 2048, 256 routed experts, top-8, 1 shared).  */
+/* ------------------------------------------------------------------------- */
+
+enum { STQ_FMT_STQ1_0 = 0, STQ_FMT_MXFP4 = 1 };
+
+/* Router: logits = x Wr^T (FP32 accumulate), softmax over E, top-k by
+ * probability (ties -> lower id), weights renormalised over the k chosen.
+ * x bf16 [T, H], w_router bf16 [E, H] -> logits f32 [T, E] (caller-owned; also
+ * the scratch of the top-k step), topk_ids int32 [T, k], topk_w f32 [T, k].
+ * E <= 1024, k <= 32, k <= E, H % 16 == 0. */
+stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T,
+                           int32_t H, int32_t E, int32_t k, float* logits,
+                           int32_t* topk_ids, float* topk_w, stq_stream_t stream);
+
+/* Token-to-expert grouping (the step every expert launch reads).  Pairs are
+ * p = t*k + slot.  counts [E]; offsets [E+1] = exclusive scan of counts;
+ * perm [P] = pair at each sorted position, sorted by expert and stably by p;
+ * inv [P] = sorted position of each pair (-1 for an id outside [0, E), which
+ * also sets STQ_ERR_DEVICE in *err); tlist [E] = touched experts in ascending
+ * order, ntouched [1] their number.  Integer, exact.  E <= 1024. */
+stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                       int32_t* tlist, int32_t* ntouched, int32_t* err,
+                       stq_stream_t stream);
+
+typedef struct {
+  int32_t fmt;              /* STQ_FMT_STQ1_0 or STQ_FMT_MXFP4 (routed experts) */
+  const uint8_t* gate;      /* E matrices [I, H], expert-major, contiguous      */
+  const uint8_t* up;        /* E matrices [I, H]                                 */
+  const uint8_t* down;      /* E matrices [H, I]                                 */
+  const uint8_t* gate_sc;   /* MXFP4 scales, E x [I, H/32]; NULL for STQ1_0      */
+  const uint8_t* up_sc;     /* E x [I, H/32]                                     */
+  const uint8_t* down_sc;   /* E x [H, I/32]                                     */
+  const uint16_t* sh_gate;  /* shared expert, bf16 [I, H]; NULL = no shared      */
+  const uint16_t* sh_up;    /* bf16 [I, H]                                       */
+  const uint16_t* sh_down;  /* bf16 [H, I]                                       */
+} moe_weights;
+
+typedef struct {
+  int32_t T, H, I, E, k;    /* tokens, hidden, intermediate, experts, top-k     */
+  int32_t out_fp32;         /* 1: y is float32 [T, H]; 0: y is bf16 [T, H]      */
+  int32_t add_residual;     /* 1: y += x                                         */
+} moe_desc;
+
+/* Bytes of device workspace moe_expert_forward needs for `d` (256-byte aligned
+ * regions; the first int32 is the error word). 0 on an invalid descriptor. */
+size_t moe_workspace_bytes(const moe_desc* d);
+
+/* y[t] = sum_s topk_w[t,s] * FFN_{topk_ids[t,s]}(x[t]) + FFN_shared(x[t]) (+ x[t])
+ * with FFN_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x)).  The intermediate h is
+ * rounded to bf16 (STQ1_0 and shared expert) or re-quantised to MXFP8 (MXFP4
+ * experts, whose input x is quantised to MXFP8 first).  Slots are summed in order
+ * s = 0..k-1, without atomics.  Duplicate ids in a token are separate slots; an
+ * id outside [0, E) sets STQ_ERR_DEVICE in the workspace error word and its slot
+ * contributes 0.  workspace: >= moe_workspace_bytes(d) bytes, 256-B aligned. */
+stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x,
+                              const int32_t* topk_ids, const float* topk_w,
+                              const moe_weights* w, void* y, void* workspace,
+                              size_t ws_bytes, stq_stream_t stream);
+
+/* Byte offset, inside the workspace of `d`, of one intermediate region, so that
+ * callers (and the parity tests) can inspect each stage:
+ *   STQ_WS_COUNTS, _OFFSETS, _PERM, _INV, _TLIST, _NTOUCHED: as moe_permute;
+ *   STQ_WS_H   bf16 [(P+T), I]: h of routed pairs (sorted order), then shared tokens;
+ *   STQ_WS_Y   f32  [(P+T), H]: expert outputs, same row order (unweighted);
+ *   STQ_WS_XQ/_XS  MXFP8 of x [T, H] / [T, H/32] (MXFP4 layers);
+ *   STQ_WS_HQ/_HS  MXFP8 of h [P, I] / [P, I/32] (MXFP4 layers).
+ * P = T*k.  Returns (size_t)-1 for an invalid descriptor or region. */
+enum { STQ_WS_COUNTS = 0, STQ_WS_OFFSETS, STQ_WS_PERM, STQ_WS_INV, STQ_WS_TLIST,
+       STQ_WS_NTOUCHED, STQ_WS_H, STQ_WS_Y, STQ_WS_XQ, STQ_WS_XS, STQ_WS_HQ, STQ_WS_HS };
+size_t moe_workspace_offset(const moe_desc* d, int32_t region);
+
+/* Synchronise `stream`, return the workspace's error word (0 = none) and clear it. */
+stq_status moe_get_device_error(void* workspace, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Instrumentation (no counterpart on the pages).                             */
+/* ------------------------------------------------------------------------- */
+
+/* Kernel kinds reported by the timing hook. */
+enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
+       STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM, STQ_K_COUNT };
+
+/* Caller-owned host struct.  While installed, every kernel launched by
+ * moe_router_topk, moe_expert_forward, stq1_gemv and w4a8_gemm outside stream
+ * capture is bracketed by cudaEventRecord(events[2n]) / (events[2n+1]) on the
+ * call's stream, kinds[n] is set to its STQ_K_* kind and n = count++ (until
+ * capacity pairs are used).  events: cudaEvent_t[2*capacity] created with timing.
+ * Process-wide, not thread-safe; NULL uninstalls.  Used by the benchmark to time
+ * each kernel on its own stream. */
+typedef struct {
+  void* const* events;
+  int32_t capacity;
+  int32_t* kinds;
+  int32_t count;
+} stq_timing;
+stq_status stq_set_timing(stq_timing* t);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STQMOE_H */

@@ -256,10 +256,11 @@ def mxfp4_unpack_f32(codes, scales, rows, K):
 #   [0, 32)     8 little-endian words; word g = d(row g) | d(row g+8) << 16
 #   [32, 544)   lane L (0..31) owns 16 bytes at 32 + 16*L: words 0..3 of its stream
 #   [544, 672)  lane L's word 4 at 544 + 4*L
-# Lane L = 4*g + t owns the 32 codes of rows g and g+8 whose group index j is
-# congruent to t mod 4; code number i = 2*s + h belongs to row g + 8*h and group
-# j = 4*s + t, and occupies bits [5*i, 5*i + 5) of the lane's 160-bit stream
-# (words 0..4, little-endian).  Tile rows are relative to the tile.
+# Lane L = 4*g + t owns the 32 codes of rows g and g+8 whose group index j lies
+# in [16*t, 16*t + 16) (k in [64*t, 64*t + 64) of the block); code number
+# i = 2*s + h belongs to row g + 8*h and group j = 16*t + s, and occupies bits
+# [5*i, 5*i + 5) of the lane's 160-bit stream (words 0..4, little-endian).  Tile
+# rows are relative to the tile.
 
 STQ_BLOCK = 256
 STQ_TILE_ROWS = 16
@@ -293,7 +294,7 @@ def _lane_maps():
     i = np.arange(32)[None, :]
     g, t = L // 4, L % 4
     s, h = i // 2, i % 2
-    return g + 8 * h, 4 * s + t
+    return g + 8 * h, 16 * t + s
 
 
 def stq1_codes_from_float(w):

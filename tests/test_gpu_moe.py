@@ -1,0 +1,219 @@
+"""GPU parity of the MoE layer steps against the oracle, stage by stage:
+grouping (exact), router (top-k set exact away from near-ties), gate/up + SwiGLU
+(propagated bound), down and shared expert (1e-3 * S + 1e-5 on the GPU's own h),
+combine (FP32 sum of the GPU's own expert outputs)."""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import formats as F
+from oracle import moe as M
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def S():
+    import bit_quantized_moe_stq1_b200 as S
+    return S
+
+
+def np_bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+# --------------------------------------------------------------------------- grouping
+
+
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (8, 8, 256), (32, 8, 256), (4096, 8, 256), (5, 3, 7), (300, 8, 1024)])
+def test_permute_exact(S, T, k, E):
+    if T * k >= 4096 * 8:
+        ids, _ = W.zipf_routing(T, E, k, DEV, 0, "pz")
+    else:
+        g = W.generator(DEV, 0, "pu", T, k, E)
+        ids = torch.randint(0, E, (T, k), generator=g, device=DEV, dtype=torch.int32)
+    out = S.moe_permute(ids, E)
+    counts, offsets, perm, inv = M.permute(ids.cpu().numpy(), E)
+    assert np.array_equal(out["counts"].cpu().numpy(), counts)
+    assert np.array_equal(out["offsets"].cpu().numpy(), offsets)
+    assert np.array_equal(out["perm"].cpu().numpy(), perm)
+    assert np.array_equal(out["inv"].cpu().numpy(), inv)
+    touched = np.flatnonzero(counts)
+    assert int(out["ntouched"].item()) == touched.size
+    assert np.array_equal(out["tlist"].cpu().numpy()[:touched.size], touched)
+
+
+def test_permute_bad_ids_and_empty(S):
+    ids = torch.tensor([[0, 300], [-1, 2]], dtype=torch.int32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = S.moe_permute(ids, 256, err=err)
+    assert S.read_error(err) == -6
+    assert out["inv"].cpu().tolist() == [0, -1, -1, 1]
+    assert out["counts"].sum().item() == 2
+    out = S.moe_permute(torch.zeros((0, 8), dtype=torch.int32, device=DEV), 256)
+    assert int(out["ntouched"].item()) == 0 and int(out["offsets"][-1].item()) == 0
+
+
+# --------------------------------------------------------------------------- router
+
+
+@pytest.mark.parametrize("T,H,E,k", [(8, 6144, 256, 8), (32, 6144, 256, 8), (3, 512, 20, 4)])
+def test_router_topk(S, T, H, E, k):
+    x = W.bf16_normal((T, H), 1.0, DEV, 0, "rx", T)
+    wr = W.bf16_normal((E, H), 0.02, DEV, 0, "rw", E)
+    ids, w, logits = S.moe_router_topk(x, wr, k)
+    ri, rw, p = M.router_topk(np_bits(x), np_bits(wr), k)
+    _, lr = M.router_probs(np_bits(x), np_bits(wr))
+    sl = np.abs(F.bf16_decode(np_bits(x))) @ np.abs(F.bf16_decode(np_bits(wr))).T
+    assert np.all(np.abs(logits.cpu().double().numpy() - lr) <= 1e-3 * sl + 1e-5)
+    ids, w = ids.cpu().numpy(), w.cpu().double().numpy()
+    for t in range(T):
+        ps = np.sort(p[t])[::-1]
+        if ps[k - 1] - ps[k] < 1e-6 * ps[0]:
+            continue                      # near-tie at the k-th place: any valid choice
+        assert set(ids[t]) == set(ri[t])
+        for j, e in enumerate(ids[t]):
+            assert abs(w[t, j] - rw[t, list(ri[t]).index(e)]) <= 1e-5
+        assert abs(w[t].sum() - 1.0) < 1e-5
+
+
+# --------------------------------------------------------------------------- STQ1_0 MoE layer
+
+
+def _make_layer(S, T, H, I, E, k, shared, tag):
+    gw = [W.stq_grid_weights(E * I, H, DEV, 0, tag, "g"), W.stq_grid_weights(E * I, H, DEV, 0, tag, "u"),
+          W.stq_grid_weights(E * H, I, DEV, 0, tag, "d")]
+    packs = [S.stq1_pack(m) for m in gw]
+    sh = None
+    if shared:
+        sh = [W.bf16_normal((I, H), 0.02, DEV, 0, tag, "sg"), W.bf16_normal((I, H), 0.02, DEV, 0, tag, "su"),
+              W.bf16_normal((H, I), 0.02, DEV, 0, tag, "sd")]
+    wr = W.bf16_normal((E, H), 0.02, DEV, 0, tag, "r")
+    x = W.bf16_normal((T, H), 1.0, DEV, 0, tag, "x")
+    return gw, packs, sh, wr, x
+
+
+def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None):
+    gw, packs, sh, wr, x = _make_layer(S, T, H, I, E, k, shared, tag)
+    if ids is None:
+        ids, tw, _ = S.moe_router_topk(x, wr, k)
+    desc = S.make_desc(T, H, I, E, k, out_fp32=True, add_residual=residual)
+    ws = torch.zeros(S.moe_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    y = torch.empty((T, H), dtype=torch.float32, device=DEV)
+    ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, *(None, None, None),
+                         *(sh if sh else (None, None, None)))
+    S.moe_expert_forward(desc, x, ids, tw, ew, y, ws)
+    assert S.moe_get_device_error(ws) == 0
+    P = T * k
+    st = dict(
+        h=S.moe_workspace_view(desc, ws, "h", torch.bfloat16, (P + T, I)).float().cpu().double().numpy(),
+        Y=S.moe_workspace_view(desc, ws, "Y", torch.float32, (P + T, H)).cpu().double().numpy(),
+        perm=S.moe_workspace_view(desc, ws, "perm", torch.int32, (P,)).cpu().numpy(),
+        inv=S.moe_workspace_view(desc, ws, "inv", torch.int32, (P,)).cpu().numpy(),
+        offsets=S.moe_workspace_view(desc, ws, "offsets", torch.int32, (E + 1,)).cpu().numpy(),
+    )
+    return dict(gw=gw, sh=sh, x=x, ids=ids.cpu().numpy(), tw=tw.cpu().double().numpy(), y=y.cpu().double().numpy(),
+                **st)
+
+
+SILU_DMAX = 1.1  # max |silu'(g)| (about 1.0998)
+
+
+def _check_gate_up(Wg, Wu, X, h_gpu):
+    """h = bf16(silu(g) u): bound from the GEMV tolerance of g and u, plus one bf16 ulp."""
+    g, sg = M.matvec_with_scale(Wg, X)
+    u, su = M.matvec_with_scale(Wu, X)
+    tg, tu = 1e-3 * sg + 1e-5, 1e-3 * su + 1e-5
+    h = M.silu(g) * u
+    bound = SILU_DMAX * tg * (np.abs(u) + tu) + np.abs(M.silu(g)) * tu + 2.0 ** -7 * (np.abs(h) + SILU_DMAX * tg * (np.abs(u) + tu) + np.abs(M.silu(g)) * tu) + 1e-6
+    err = np.abs(h_gpu - h)
+    assert np.all(err <= bound), float(np.max(err / bound))
+
+
+def _check_down(Wd, h_rows, Y_rows):
+    y, sy = M.matvec_with_scale(Wd, h_rows)
+    assert np.all(np.abs(Y_rows - y) <= 1e-3 * sy + 1e-5), float(np.max(np.abs(Y_rows - y) / (1e-3 * sy + 1e-5)))
+
+
+def _check_layer(r, T, H, I, E, k, experts=None):
+    P = T * k
+    counts, offsets, perm, inv = M.permute(r["ids"], E)
+    assert np.array_equal(r["perm"], perm) and np.array_equal(r["inv"], inv)
+    xd = r["x"].float().double().cpu().numpy()
+    touched = np.flatnonzero(counts)
+    if experts is None:
+        experts = touched
+    gw = r["gw"]
+    for e in experts:
+        pos = np.arange(offsets[e], offsets[e + 1])
+        toks = perm[pos] // k
+        Wg = gw[0][e * I:(e + 1) * I].double().cpu().numpy()
+        Wu = gw[1][e * I:(e + 1) * I].double().cpu().numpy()
+        Wd = gw[2][e * H:(e + 1) * H].double().cpu().numpy()
+        _check_gate_up(Wg, Wu, xd[toks], r["h"][pos])
+        _check_down(Wd, r["h"][pos], r["Y"][pos])
+    if r["sh"] is not None:
+        sg, su, sd = (m.float().double().cpu().numpy() for m in r["sh"])
+        _check_gate_up(sg, su, xd, r["h"][P:P + T])
+        _check_down(sd, r["h"][P:P + T], r["Y"][P:P + T])
+    # combine of the GPU's own expert outputs
+    yc = np.zeros((T, H))
+    for t in range(T):
+        for s in range(k):
+            yc[t] += r["tw"][t, s] * r["Y"][inv[t * k + s]]
+        if r["sh"] is not None:
+            yc[t] += r["Y"][P + t]
+    scale = np.abs(yc) + np.max(np.abs(r["Y"]), axis=0)[None, :] * 1e-6
+    assert np.all(np.abs(r["y"] - yc) <= 1e-5 * scale + 1e-6)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,shared", [(1, 256, 256, 1, 1, False), (5, 512, 256, 8, 2, True),
+                                               (13, 768, 512, 16, 4, True), (40, 512, 256, 4, 4, False)])
+def test_moe_stq_small_full_check(S, T, H, I, E, k, shared):
+    r = _run_layer(S, T, H, I, E, k, shared, ("small", T, H, I, E, k))
+    _check_layer(r, T, H, I, E, k)
+
+
+def test_moe_stq_decode_config_sampled(S):
+    """Decode MoE layer, STQ1_0: 256 experts, 6144/2048, 8 tokens, top-8, shared."""
+    T, H, I, E, k = 8, 6144, 2048, 256, 8
+    r = _run_layer(S, T, H, I, E, k, True, "decode")
+    counts = np.bincount(r["ids"].reshape(-1), minlength=E)
+    touched = np.flatnonzero(counts)
+    busiest = touched[np.argsort(-counts[touched], kind="stable")[:2]]
+    sample = np.unique(np.concatenate([busiest, touched[:: max(1, touched.size // 3)]]))
+    _check_layer(r, T, H, I, E, k, experts=sample)
+
+
+def test_moe_stq_residual_and_bf16_output(S):
+    T, H, I, E, k = 6, 512, 256, 8, 2
+    gw, packs, sh, wr, x = _make_layer(S, T, H, I, E, k, True, "res")
+    ids, tw, _ = S.moe_router_topk(x, wr, k)
+    ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, None, None, None, *sh)
+    out = {}
+    for fp32, res in [(True, False), (True, True), (False, True)]:
+        desc = S.make_desc(T, H, I, E, k, out_fp32=fp32, add_residual=res)
+        ws = torch.zeros(S.moe_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+        y = torch.empty((T, H), dtype=torch.float32 if fp32 else torch.bfloat16, device=DEV)
+        S.moe_expert_forward(desc, x, ids, tw, ew, y, ws)
+        out[(fp32, res)] = y.float().cpu().double().numpy()
+    xd = x.float().double().cpu().numpy()
+    assert np.allclose(out[(True, True)], out[(True, False)] + xd, rtol=1e-6, atol=1e-6)
+    ref_b = F.bf16_decode(F.bf16_encode_rne(out[(True, True)]))
+    assert np.array_equal(out[(False, True)], ref_b)
+
+
+def test_moe_bad_expert_id_reports_and_skips(S):
+    T, H, I, E, k = 2, 256, 256, 4, 2
+    gw, packs, sh, wr, x = _make_layer(S, T, H, I, E, k, False, "bad")
+    ids = torch.tensor([[0, 9], [1, 2]], dtype=torch.int32, device=DEV)
+    tw = torch.full((T, k), 0.5, device=DEV)
+    desc = S.make_desc(T, H, I, E, k, out_fp32=True)
+    ws = torch.zeros(S.moe_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
+    y = torch.empty((T, H), dtype=torch.float32, device=DEV)
+    S.moe_expert_forward(desc, x, ids, tw, S.ExpertWeights(S.FMT_STQ1_0, *packs), y, ws)
+    assert S.moe_get_device_error(ws) == -6
+    assert torch.isfinite(y).all()

@@ -132,7 +132,7 @@ def _read_code_by_loops(packed, rows, K, r, j):
     b, jj = divmod(j, 64)
     base = (tile * nb + b) * 672
     g, h = rr % 8, rr // 8
-    t, s = jj % 4, jj // 4
+    t, s = jj // 16, jj % 16
     lane = 4 * g + t
     i = 2 * s + h
     words = [int.from_bytes(bytes(packed[base + 32 + 16 * lane + 4 * w: base + 36 + 16 * lane + 4 * w]), "little") for w in range(4)]
