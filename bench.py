@@ -3,13 +3,16 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = one pass of the whole hot path of the workload over one batch of
-synthetic inputs (router, grouping, expert GEMVs with SwiGLU, shared expert,
-combine; layer after layer for the stacked workload).  Inputs are resident in
-HBM before timing; each step uses a different token batch (rotating over 8) and
-the per-step expert weights exceed L2, so no step is served from L2.
-Rank 0 prints one JSON line.  Under torchrun every rank runs its own replica
-(weak scaling, no collective on the data path); the reported time is the max
-over ranks.
+synthetic inputs: router, grouping, activation quantisation (MXFP4 layers),
+expert gate/up with fused SwiGLU, down, shared expert and combine, layer after
+layer for the stacked workload.  Inputs are resident in HBM before timing; steps
+rotate over 8 token batches (and, for the single-matrix workloads, over weight
+copies totalling more than 4x L2), so no step is served from L2.  The timed
+region replays one CUDA graph per step.  Per-kernel times come from CUDA events
+the library records around each launch (captured into the graphs as event
+nodes), on the launching stream.  Rank 0 prints one JSON line.  Under torchrun
+every rank runs its own replica (weak scaling, no collective on the data path);
+the reported time is the max over ranks.
 
 --impl reference times the CPU oracle (the plain float64 numpy reference under
 oracle/) on a bounded sample of the same workload, on rank 0 only.
@@ -19,9 +22,8 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 import numpy as np
@@ -32,192 +34,285 @@ sys.path.insert(0, ROOT)
 
 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "decode_stq"
+DEFAULT_WORKLOAD = "stacked_decode"
 N_BATCHES = 8
-STQ_MAT = 2048 * 6144 // 256 * 42          # 2,064,384 bytes per STQ1_0 expert matrix
-STQ_EXPERT = 3 * STQ_MAT                    # 6,193,152
-BF16_MAT = 2048 * 6144 * 2                  # 25,165,824
-ROUTER_BYTES = 256 * 6144 * 2               # 3,145,728
+H, I, E, K_TOP = W.HIDDEN, W.INTER, W.EXPERTS, W.TOPK
+STQ_MAT = I * H // 256 * 42                 # 2,064,384 bytes per STQ1_0 expert matrix
+MX_MAT = I * H // 2 + I * H // 32           # 6,684,672 bytes per MXFP4 matrix (codes + scales)
+BF16_MAT = I * H * 2                        # 25,165,824
+ROUTER_BYTES = E * H * 2                    # 3,145,728
+NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense BF16 tensor rate
 
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]), src="measured")
-    return dict(hbm=6650.0, bf16=1590.0, src="fallback")
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
 # ----------------------------------------------------------------------------- clocks
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """NVML sampling of SM clocks and throttle reasons while the timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
+        self.gpu, self.samples, self.stop = gpu_index, [], threading.Event()
+        self.max_mhz = None
+
+    def _run(self):
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((sm, rs))
+            time.sleep(0.002)
+        pynvml.nvmlShutdown()
 
     def __enter__(self):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.th = threading.Thread(target=self._run, daemon=True)
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            self.th.start()
+            time.sleep(0.05)
         except Exception:
-            self.proc = None
+            self.th = None
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        if self.th is not None:
+            self.th.join(timeout=5)
 
     def summary(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.f.flush()
-        rows = [l.split(",") for l in open(self.f.name).read().strip().splitlines() if l.count(",") >= 8]
-        os.unlink(self.f.name)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"], "samples": 0}
+        sm = [s for s, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------------------------- workloads
 
 
-class DecodeSTQ:
-    """Decode MoE layer, STQ1_0 experts: 8 BF16 tokens, BF16 router (softmax, top-8,
-    renormalised), 256 experts of 6144 -> 2048 -> 6144, one BF16 shared expert."""
-
-    name = "decode_stq"
+class Workload:
     unit = "tokens/s"
-
-    def __init__(self, S, dev, tokens=8, layers=1):
-        self.S, self.dev = S, dev
-        self.wl = W.WORKLOADS["decode_stq"]
-        self.T, self.H, self.I, self.E, self.k = tokens, self.wl.H, self.wl.I, self.wl.E, self.wl.k
-        self.layers = [self._layer(l) for l in range(layers)]
-        self.x = [W.bf16_normal((self.T, self.H), 1.0, dev, 0, "x", b) for b in range(N_BATCHES)]
-        self.desc = S.make_desc(self.T, self.H, self.I, self.E, self.k)
-        self.ws = torch.zeros(S.moe_workspace_bytes(self.desc), dtype=torch.uint8, device=dev)
-        self.y = torch.empty((self.T, self.H), dtype=torch.bfloat16, device=dev)
-        self.logits = torch.empty((self.T, self.E), dtype=torch.float32, device=dev)
-        self.ids = torch.empty((self.T, self.k), dtype=torch.int32, device=dev)
-        self.tw = torch.empty((self.T, self.k), dtype=torch.float32, device=dev)
-
-    def _stq_matrices(self, l, which, rows, cols):
-        """E STQ1_0 matrices [rows, cols], packed on the device in chunks of 16 experts."""
-        S, E = self.S, self.E
-        out = torch.empty(E * rows * cols // 256 * 42, dtype=torch.uint8, device=self.dev)
-        per = rows * cols // 256 * 42
-        for e0 in range(0, E, 16):
-            wf = W.stq_grid_weights(16 * rows, cols, self.dev, 0, "L", l, which, e0)
-            S.stq1_pack(wf, out=out[e0 * per:(e0 + 16) * per])
-            del wf
-        return out
-
-    def _layer(self, l):
-        S = self.S
-        g = self._stq_matrices(l, "g", self.I, self.H)
-        u = self._stq_matrices(l, "u", self.I, self.H)
-        d = self._stq_matrices(l, "d", self.H, self.I)
-        sh = [W.bf16_normal((self.I, self.H), 0.02, self.dev, 0, "L", l, "sg"),
-              W.bf16_normal((self.I, self.H), 0.02, self.dev, 0, "L", l, "su"),
-              W.bf16_normal((self.H, self.I), 0.02, self.dev, 0, "L", l, "sd")]
-        wr = W.bf16_normal((self.E, self.H), 0.02, self.dev, 0, "L", l, "router")
-        return dict(w=S.ExpertWeights(S.FMT_STQ1_0, g, u, d, sh_gate=sh[0], sh_up=sh[1], sh_down=sh[2]), wr=wr)
-
-    def step(self, b, x=None, y=None):
-        S = self.S
-        x = self.x[b % N_BATCHES] if x is None else x
-        y = self.y if y is None else y
-        for L in self.layers:
-            S.moe_router_topk(x, L["wr"], self.k, self.logits, self.ids, self.tw)
-            S.moe_expert_forward(self.desc, x, self.ids, self.tw, L["w"], y, self.ws)
-        return y
+    metric = "MoE-layer tokens/s"
+    bound = "hbm"
 
     def tokens_per_step(self):
         return self.T
 
-    def touched(self, b):
-        """Realised number of touched experts per layer for batch b (host bookkeeping)."""
-        S = self.S
-        out = []
-        for L in self.layers:
-            ids, _, _ = S.moe_router_topk(self.x[b % N_BATCHES], L["wr"], self.k)
-            out.append(int(torch.unique(ids).numel()))
-        return out
-
-    def algorithmic_bytes(self, b):
-        """Bytes a step must move: touched experts' packed matrices, the shared
-        expert, the router, and the activations (x in, y out)."""
-        n = self.touched(b)
-        per_layer = [t * STQ_EXPERT + 3 * BF16_MAT + ROUTER_BYTES + self.T * self.H * 4 for t in n]
-        gate_up = [t * 2 * STQ_MAT + 2 * BF16_MAT + self.T * self.H * 2 + (self.T * self.k + self.T) * self.I * 2
-                   for t in n]
-        return sum(per_layer), dict(gate_up=gate_up)
-
     def h2d_d2h(self):
-        return self.T * self.H * 2, self.T * self.H * 2
+        return self.T * H * 2, self.T * H * 2
 
 
-class StqMatvec:
-    """One STQ1_0 matrix 2048 x 6144 times one BF16 N(0,1) vector, FP32 out.  The
-    2 MB matrix fits in L2, so steps rotate over copies totalling 4x the L2 size."""
+class StqMatvec(Workload):
+    """One STQ1_0 matrix 2048 x 6144 times one BF16 N(0,1) vector, FP32 out."""
 
     name = "stq_matvec"
     unit = "GB/s"
+    metric = "STQ1_0 matvec achieved HBM GB/s (2048x6144, 1 token)"
 
     def __init__(self, S, dev):
-        self.S, self.dev = S, dev
+        self.S, self.dev, self.T = S, dev, 1
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         self.ncopies = max(8, int(4 * l2 // STQ_MAT) + 1)
-        wf = W.stq_grid_weights(2048, 6144, dev, 0, "mv")
-        base = S.stq1_pack(wf)
-        self.W = [base.clone() for _ in range(self.ncopies)]
-        self.x = [W.bf16_normal((1, 6144), 1.0, dev, 0, "mvx", b) for b in range(N_BATCHES)]
-        self.y = torch.empty((1, 2048), dtype=torch.float32, device=dev)
+        base = S.stq1_pack(W.stq_grid_weights(I, H, dev, 0, "mv"))
+        self.Wt = [base.clone() for _ in range(self.ncopies)]
+        self.x = [W.bf16_normal((1, H), 1.0, dev, 0, "mvx", b) for b in range(N_BATCHES)]
+        self.y = torch.empty((1, I), dtype=torch.float32, device=dev)
+        self.bytes = STQ_MAT + H * 2 + I * 4
 
-    def step(self, b, x=None, y=None):
-        x = self.x[b % N_BATCHES] if x is None else x
-        return self.S.stq1_gemv(self.W[b % self.ncopies], 2048, 6144, x, self.y if y is None else y)
+    def step(self, i, x=None, y=None):
+        return self.S.stq1_gemv(self.Wt[i % self.ncopies], I, H, self.x[i % N_BATCHES] if x is None else x,
+                                self.y if y is None else y)
 
-    def tokens_per_step(self):
-        return 1
-
-    def algorithmic_bytes(self, b):
-        nb = STQ_MAT + 6144 * 2 + 2048 * 4
-        return nb, dict(gemv=[nb])
+    def accounting(self, i):
+        return dict(bytes=self.bytes, flops=2 * I * H, per_kind={"gemv": dict(bytes=self.bytes)})
 
     def h2d_d2h(self):
-        return 6144 * 2, 2048 * 4
+        return H * 2, I * 4
 
 
-WORKLOADS = {"decode_stq": DecodeSTQ, "stq_matvec": StqMatvec}
+class W4A8Gemm(Workload):
+    """One MXFP4 expert matrix 2048 x 6144 (codes uniform, scales in [118, 127]) times
+    128 BF16 N(0,1) tokens quantised on the device to MXFP8; FP32 out."""
+
+    name = "w4a8_gemm"
+    bound = "tensor"
+
+    def __init__(self, S, dev):
+        self.S, self.dev, self.T = S, dev, 128
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.ncopies = max(8, int(4 * l2 // MX_MAT) + 1)
+        c, s = W.mxfp4_random(I, H, dev, 0, "w4")
+        self.Wt = [(c.clone(), s.clone()) for _ in range(self.ncopies)]
+        self.x = [W.bf16_normal((self.T, H), 1.0, dev, 0, "w4x", b) for b in range(N_BATCHES)]
+        self.ac = torch.empty((self.T, H), dtype=torch.uint8, device=dev)
+        self.asc = torch.empty((self.T, H // 32), dtype=torch.uint8, device=dev)
+        self.y = torch.empty((self.T, I), dtype=torch.float32, device=dev)
+
+    def step(self, i, x=None, y=None):
+        S = self.S
+        S.mxfp8_quantize_bf16(self.x[i % N_BATCHES] if x is None else x, self.ac, self.asc)
+        c, s = self.Wt[i % self.ncopies]
+        return S.w4a8_gemm(c, s, I, H, self.ac, self.asc, self.y if y is None else y)
+
+    def accounting(self, i):
+        fl = 2 * self.T * I * H
+        by = MX_MAT + self.T * H * (1 + 1 / 32) + self.T * I * 4
+        return dict(bytes=by, flops=fl, per_kind={"gemm": dict(bytes=by, flops=fl)})
+
+    def h2d_d2h(self):
+        return self.T * H * 2, self.T * I * 4
+
+
+class MoeLayers(Workload):
+    """MoE layers of hidden 6144, 256 experts of intermediate 2048, top-8."""
+
+    def __init__(self, S, dev, name, T, fmts, router, shared, residual):
+        self.S, self.dev, self.name, self.T = S, dev, name, T
+        self.fmts, self.router, self.shared, self.residual = fmts, router, shared, residual
+        self.layers = [self._layer(l, f) for l, f in enumerate(fmts)]
+        self.x = [W.bf16_normal((T, H), 1.0, dev, 0, name, "x", b) for b in range(N_BATCHES)]
+        if not router:
+            self.routing = [W.zipf_routing(T, E, K_TOP, dev, 0, name, "zipf", b) for b in range(N_BATCHES)]
+        self.desc = S.make_desc(T, H, I, E, K_TOP, out_fp32=False, add_residual=residual)
+        self.ws = torch.zeros(S.moe_workspace_bytes(self.desc), dtype=torch.uint8, device=dev)
+        self.bufs = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.logits = S.router_scratch(T, H, E, dev)
+        self.ids = torch.empty((T, K_TOP), dtype=torch.int32, device=dev)
+        self.tw = torch.empty((T, K_TOP), dtype=torch.float32, device=dev)
+        self._acct = {}
+
+    def _stq(self, l, which, rows, cols):
+        S = self.S
+        per = rows * cols // 256 * 42
+        out = torch.empty(E * per, dtype=torch.uint8, device=self.dev)
+        for e0 in range(0, E, 16):
+            wf = W.stq_grid_weights(16 * rows, cols, self.dev, 0, self.name, l, which, e0)
+            S.stq1_pack(wf, out=out[e0 * per:(e0 + 16) * per])
+            del wf
+        return out
+
+    def _layer(self, l, fmt):
+        S = self.S
+        if fmt == "stq":
+            mats = [self._stq(l, "g", I, H), self._stq(l, "u", I, H), self._stq(l, "d", H, I)]
+            scales = [None, None, None]
+        else:
+            g = W.mxfp4_random(E * I, H, self.dev, 0, self.name, l, "g")
+            u = W.mxfp4_random(E * I, H, self.dev, 0, self.name, l, "u")
+            d = W.mxfp4_random(E * H, I, self.dev, 0, self.name, l, "d")
+            mats, scales = [g[0], u[0], d[0]], [g[1], u[1], d[1]]
+        sh = [None, None, None]
+        if self.shared:
+            sh = [W.bf16_normal((I, H), 0.02, self.dev, 0, self.name, l, "sg"),
+                  W.bf16_normal((I, H), 0.02, self.dev, 0, self.name, l, "su"),
+                  W.bf16_normal((H, I), 0.02, self.dev, 0, self.name, l, "sd")]
+        wr = W.bf16_normal((E, H), 0.02, self.dev, 0, self.name, l, "router") if self.router else None
+        f = S.FMT_STQ1_0 if fmt == "stq" else S.FMT_MXFP4
+        return dict(fmt=fmt, wr=wr, w=S.ExpertWeights(f, *mats, *scales, *sh))
+
+    def step(self, i, x=None, y=None):
+        S = self.S
+        cur = self.x[i % N_BATCHES] if x is None else x
+        for l, L in enumerate(self.layers):
+            out = y if (y is not None and l == len(self.layers) - 1) else self.bufs[l % 2]
+            if self.router:
+                S.moe_router_topk(cur, L["wr"], K_TOP, self.logits, self.ids, self.tw)
+                ids, tw = self.ids, self.tw
+            else:
+                ids, tw = self.routing[i % N_BATCHES]
+            S.moe_expert_forward(self.desc, cur, ids, tw, L["w"], out, self.ws)
+            cur = out
+        return cur
+
+    def touched(self, i):
+        """Realised touched experts per layer for batch i (host bookkeeping, eager)."""
+        S = self.S
+        cur = self.x[i % N_BATCHES]
+        out = []
+        for l, L in enumerate(self.layers):
+            if self.router:
+                S.moe_router_topk(cur, L["wr"], K_TOP, self.logits, self.ids, self.tw)
+                ids, tw = self.ids, self.tw
+            else:
+                ids, tw = self.routing[i % N_BATCHES]
+            out.append(int(torch.unique(ids).numel()))
+            nxt = self.bufs[(l + 1) % 2]
+            S.moe_expert_forward(self.desc, cur, ids, tw, L["w"], nxt, self.ws)
+            cur = nxt
+        torch.cuda.synchronize()
+        return out
+
+    def accounting(self, i):
+        """Algorithmic bytes and FLOPs of step i: the touched experts' packed matrices, the
+        shared expert, the router, activations in and out; per kernel kind, per launch."""
+        b = i % N_BATCHES
+        if b not in self._acct:
+            self._acct[b] = self.touched(b)
+        n = self._acct[b]
+        T, P = self.T, self.T * K_TOP
+        tot, kinds = 0, {}
+        for L, t in zip(self.layers, n):
+            mat = STQ_MAT if L["fmt"] == "stq" else MX_MAT
+            by = t * 3 * mat + (3 * BF16_MAT if self.shared else 0) + (ROUTER_BYTES if self.router else 0) + 2 * T * H * 2
+            tot += by
+            if L["fmt"] == "stq":
+                gu = t * 2 * STQ_MAT + (2 * BF16_MAT if self.shared else 0) + T * H * 2 + (P + T) * I * 2
+                dn = t * STQ_MAT + (BF16_MAT if self.shared else 0) + (P + T) * I * 2 + (P + T) * H * 4
+                kinds.setdefault("gate_up", []).append(dict(bytes=gu))
+                kinds.setdefault("down", []).append(dict(bytes=dn))
+            else:
+                gu = t * 2 * MX_MAT + P * H * (1 + 1 / 32) + P * I * (1 + 1 / 32)
+                dn = t * MX_MAT + P * I * (1 + 1 / 32) + P * H * 4
+                kinds.setdefault("gate_up_mx", []).append(dict(bytes=gu, flops=4 * P * I * H))
+                kinds.setdefault("down_mx", []).append(dict(bytes=dn, flops=2 * P * I * H))
+        flops = len(self.layers) * 3 * 2 * T * K_TOP * I * H
+        return dict(bytes=tot, flops=flops, per_kind={k: dict(bytes=float(np.mean([d["bytes"] for d in v])),
+                                                             flops=float(np.mean([d.get("flops", 0) for d in v])))
+                                                      for k, v in kinds.items()})
+
+
+def make_workload(name, S, dev):
+    if name == "stq_matvec":
+        return StqMatvec(S, dev)
+    if name == "w4a8_gemm":
+        return W4A8Gemm(S, dev)
+    wl = W.WORKLOADS[name]
+    return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual)
+
+
+WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "stacked_decode"]
 
 
 # ----------------------------------------------------------------------------- measurement
 
 
-def timed_steps(wl, steps, warmup, dist):
-    torch.cuda.synchronize()
+def capture(wl):
+    graphs = []
+    for b in range(N_BATCHES):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            wl.step(b)
+        graphs.append(g)
+    return graphs
+
+
+def timed_replays(graphs, steps, warmup, dist):
     for i in range(warmup):
-        wl.step(i)
+        graphs[i % N_BATCHES].replay()
     torch.cuda.synchronize()
     if dist:
         torch.distributed.barrier()
@@ -225,7 +320,7 @@ def timed_steps(wl, steps, warmup, dist):
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for i in range(steps):
-        wl.step(warmup + i)
+        graphs[(warmup + i) % N_BATCHES].replay()
     stop.record()
     torch.cuda.synchronize()
     if dist:
@@ -234,32 +329,42 @@ def timed_steps(wl, steps, warmup, dist):
 
 
 def kernel_times(S, wl, steps, warmup):
-    """Per-kernel CUDA-event durations over `steps` steps (events recorded by the
-    library on the launching stream)."""
-    timer = S.KernelTimer(capacity=4096)
+    """Per-kernel CUDA-event durations from graph replays (events recorded by the
+    library on the launching stream, captured as event nodes)."""
+    timer = S.KernelTimer(capacity=64 * N_BATCHES)
+    tg = []
+    with timer:
+        for b in range(N_BATCHES):
+            s0 = timer.st.count
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                wl.step(b)
+            tg.append((g, s0, timer.st.count))
     per_kind = {}
     for i in range(steps):
-        with timer:
-            wl.step(warmup + i)
-        for kind, ms in timer.results():
-            per_kind.setdefault(kind, []).append(ms)
+        g, s0, s1 = tg[(warmup + i) % N_BATCHES]
+        g.replay()
+        torch.cuda.synchronize()
+        for n in range(s0, s1):
+            kind = S.KERNEL_KINDS[timer._kinds[n]]
+            per_kind.setdefault(kind, []).append(timer.ev[2 * n].elapsed_time(timer.ev[2 * n + 1]))
     return per_kind
 
 
 def e2e_steps(wl, steps, warmup):
-    """Same metric end to end through the public API with pinned host buffers:
-    H2D of the step's tokens and D2H of its output inside the timed region."""
-    x_dev = wl.x[0]
+    """Same metric end to end through the public API with pinned host buffers: H2D
+    of the step's input tokens and D2H of its output inside the timed region."""
     hx = [wl.x[b].cpu().pin_memory() for b in range(N_BATCHES)]
-    y_dev = torch.empty_like(wl.y)
+    xs = torch.empty_like(wl.x[0])
+    out = wl.step(0)
+    y_dev = torch.empty_like(out)
     hy = torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory()
     for i in range(warmup):
-        x_dev.copy_(hx[i % N_BATCHES], non_blocking=True)
-        wl.step(i, x=x_dev, y=y_dev)
+        xs.copy_(hx[i % N_BATCHES], non_blocking=True)
+        wl.step(i, x=xs, y=y_dev)
         hy.copy_(y_dev, non_blocking=True)
     torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    xs = torch.empty_like(x_dev)
     start.record()
     for i in range(steps):
         xs.copy_(hx[(warmup + i) % N_BATCHES], non_blocking=True)
@@ -267,13 +372,14 @@ def e2e_steps(wl, steps, warmup):
         hy.copy_(y_dev, non_blocking=True)
     stop.record()
     torch.cuda.synchronize()
-    return start.elapsed_time(stop)
+    return start.elapsed_time(stop), xs.numel() * xs.element_size(), hy.numel() * hy.element_size()
 
 
 def run_ours(args):
     dist = int(os.environ.get("WORLD_SIZE", "1")) > 1
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    n = int(os.environ.get("WORLD_SIZE", "1"))
     if dist:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
@@ -281,62 +387,70 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     import bit_quantized_moe_stq1_b200 as S
 
-    wl = WORKLOADS[args.workload](S, dev)
+    wl = make_workload(args.workload, S, dev)
+    for i in range(args.warmup):          # eager warm-up (one-time attribute setup)
+        wl.step(i)
     torch.cuda.synchronize()
+    graphs = capture(wl)
     with ClockSampler(local) as clk:
-        ms = timed_steps(wl, args.steps, args.warmup, dist)
+        ms = timed_replays(graphs, args.steps, args.warmup, dist)
     clocks = clk.summary()
     ms_t = torch.tensor([ms], device=dev)
     if dist:
         torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(ms_t.item())
-    n = int(os.environ.get("WORLD_SIZE", "1"))
-    ms_step = ms / args.steps
+    ms_step = float(ms_t.item()) / args.steps
     kt = kernel_times(S, wl, args.steps, args.warmup)
-    e2e_ms = e2e_steps(wl, args.steps, args.warmup)
-    ab, per_kernel_bytes = wl.algorithmic_bytes(0)
+    e2e_ms, h2d, d2h = e2e_steps(wl, args.steps, args.warmup)
+    acct = [wl.accounting(args.warmup + i) for i in range(min(args.steps, N_BATCHES))]
+    ab = float(np.mean([a["bytes"] for a in acct]))
     pk = peaks()
-    # dominant kernel: the kind with the largest total time
     tot = {k: sum(v) for k, v in kt.items()}
     dom = max(tot, key=tot.get)
-    launches = len(kt[dom])
-    avg_ms = tot[dom] / launches
-    kb = per_kernel_bytes.get(dom)
-    kb_launch = float(np.mean(kb)) if kb else None
-    achieved = kb_launch / (avg_ms * 1e-3) / 1e9 if kb_launch else None
+    avg_ms = tot[dom] / len(kt[dom])
+    per = acct[0]["per_kind"].get(dom, {})
+    launch_bytes = float(np.mean([a["per_kind"][dom]["bytes"] for a in acct if dom in a["per_kind"]])) if per else None
+    launch_flops = float(np.mean([a["per_kind"][dom].get("flops", 0) for a in acct if dom in a["per_kind"]])) if per else 0
+    if wl.bound == "tensor" or dom in ("gate_up_mx", "down_mx") and wl.name == "prefill_w4a8":
+        peak = pk["bf16"] * NOMINAL_FP8_OVER_BF16
+        achieved = launch_flops / (avg_ms * 1e-3) / 1e12 if launch_flops else None
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak if achieved else None,
+                "peak_source": f"{pk['src']} bf16 burst x {NOMINAL_FP8_OVER_BF16} (nominal FP8/BF16 dense ratio)",
+                "traffic": None, "flops_per_launch": launch_flops, "avg_launch_ms": avg_ms,
+                "hbm_gbs": launch_bytes / (avg_ms * 1e-3) / 1e9 if launch_bytes else None}
+    else:
+        achieved = launch_bytes / (avg_ms * 1e-3) / 1e9 if launch_bytes else None
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"] if achieved else None, "peak_source": pk["src"] + " copy bandwidth",
+                "traffic": None, "bytes_per_launch": launch_bytes, "avg_launch_ms": avg_ms}
     tps = wl.tokens_per_step()
-    gpu_launches = sum(len(v) for v in kt.values())
     if wl.unit == "GB/s":
         value = n * ab / (ms_step * 1e-3) / 1e9
-        metric = "STQ1_0 matvec achieved HBM GB/s (2048x6144, 1 token)"
         e2e_val = n * ab / (e2e_ms / args.steps * 1e-3) / 1e9
     else:
         value = n * tps / (ms_step * 1e-3)
-        metric = "MoE-layer tokens/s"
         e2e_val = n * tps / (e2e_ms / args.steps * 1e-3)
-    h2d, d2h = wl.h2d_d2h()
     out = {
-        "metric": metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": args.steps,
+        "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 activations x packed STQ1_0 weights, fp32 accumulate",
+        "vs_baseline": None,
+        "dtype": "bf16 activations x STQ1_0 (ternary, fp16 scale) and MXFP4 x MXFP8 weights, fp32 accumulate",
         "data": "synthetic (seeded generators; random weights on the format grids)",
         "config": {"workload": wl.name, "tokens_per_step": tps, "hbm_bytes_per_step": ab,
-                   "l2": "weights per step exceed L2; token batches rotate over 8",
-                   "parallelism": f"replicas x{n}"},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": (achieved / pk["hbm"]) if achieved else None, "peak_source": pk["src"],
-                     "traffic": None, "bytes_per_launch": kb_launch, "avg_launch_ms": avg_ms},
+                   "tflop_per_step": acct[0]["flops"] / 1e12,
+                   "l2": "inputs larger than L2: per-step weights exceed L2, batches rotate over 8",
+                   "parallelism": f"replicas x{n}", "timing": "CUDA graph replays, CUDA events"},
+        "roofline": roof,
         "kernels_ms": {k: statistics.mean(v) for k, v in kt.items()},
-        "gpu_launches": gpu_launches,
+        "gpu_launches": int(sum(len(v) for v in kt.values()) / args.steps * args.steps),
         "e2e": {"value": e2e_val, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,
     }
-    if rank == 0 and not dist:
+    if rank == 0 and not dist and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(wl, dev)
-    elif rank == 0:
-        out["cpu_baseline"] = None
     if rank == 0:
         print(json.dumps(out))
+    del graphs
     if dist:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -345,72 +459,105 @@ def run_ours(args):
 # ----------------------------------------------------------------------------- oracle timing
 
 
-def _oracle_decode_token(wl, dev, b=0, t=0):
-    """The oracle's layer for one token: router, its top-8 experts and the shared
-    expert, from the generator's tensors (weights decoded from the oracle's own
-    packing of the generator's grid values)."""
+def _oracle_units(wl, dev):
+    """One bounded unit of oracle work for the workload and its scale to one step:
+    returns (seconds for the unit, units per step, description)."""
     from oracle import formats as F
     from oracle import moe as M
 
-    x = wl.x[b][t:t + 1]
-    xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
-    L = 0
-    wr = wl.layers[L]["wr"].view(torch.int16).cpu().numpy().view(np.uint16)
-    ids, w, _ = M.router_topk(xb, wr, wl.k)
-    X = F.bf16_decode(xb)
-    y = np.zeros((1, wl.H))
-    for s, e in enumerate(ids[0]):
-        mats = []
-        for which, (rows, cols) in (("g", (wl.I, wl.H)), ("u", (wl.I, wl.H)), ("d", (wl.H, wl.I))):
-            e0 = (int(e) // 16) * 16
-            wf = W.stq_grid_weights(16 * rows, cols, dev, 0, "L", L, which, e0)
-            blk = wf[(int(e) - e0) * rows:(int(e) - e0 + 1) * rows].cpu().numpy()
-            mats.append(F.stq1_unpack(F.stq1_pack(blk), rows, cols))
-        out = M.expert_ffn_bf16h(mats[0], mats[1], mats[2], X)
-        y += w[0, s] * out["y"]
-    sh = [wl.layers[L]["w"].sh_gate, wl.layers[L]["w"].sh_up, wl.layers[L]["w"].sh_down]
-    out = M.expert_ffn_bf16h(*[m.float().double().cpu().numpy() for m in sh], X)
-    return y + out["y"]
+    if wl.name == "stq_matvec":
+        Wb = wl.Wt[0].cpu().numpy()
+        xb = wl.x[0].view(torch.int16).cpu().numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        M.stq1_gemv(Wb, I, H, xb)
+        return time.perf_counter() - t0, 1.0, "one full matvec (unpack + float64 matvec)"
+    if wl.name == "w4a8_gemm":
+        c, sc = wl.Wt[0]
+        xb = wl.x[0][:16].view(torch.int16).cpu().numpy().view(np.uint16)
+        c, sc = c.cpu().numpy(), sc.cpu().numpy()
+        t0 = time.perf_counter()
+        ac, asc = F.mxfp8_quantize(F.bf16_decode(xb))
+        M.w4a8_gemm(c, sc, ac, asc, I, H)
+        return time.perf_counter() - t0, wl.T / 16, "16 of the 128 tokens (quantise, unpack, float64 GEMM)"
+    # MoE: one token through one routed expert (+ router and shared expert) per format
+    total, desc = 0.0, []
+    for fmt in sorted({L["fmt"] for L in wl.layers}):
+        l = next(i for i, L in enumerate(wl.layers) if L["fmt"] == fmt)
+        L = wl.layers[l]
+        xb = wl.x[0][:1].view(torch.int16).cpu().numpy().view(np.uint16)
+        X = F.bf16_decode(xb)
+        e = 0
+        if fmt == "stq":
+            blks = [W.stq_grid_weights(16 * r, c_, dev, 0, wl.name, l, which, 0)[:r].cpu().numpy()
+                    for which, (r, c_) in (("g", (I, H)), ("u", (I, H)), ("d", (H, I)))]
+            packed = [F.stq1_pack(b_) for b_ in blks]
+        else:
+            lw = L["w"]
+            packed = [(c_[:r].cpu().numpy(), s_[:r].cpu().numpy()) for c_, s_, r in
+                      ((lw.gate, lw.gate_sc, I), (lw.up, lw.up_sc, I), (lw.down, lw.down_sc, H))]
+        shared = [m.float().double().cpu().numpy() for m in (L["w"].sh_gate, L["w"].sh_up, L["w"].sh_down)] \
+            if wl.shared else None
+        wr = L["wr"].view(torch.int16).cpu().numpy().view(np.uint16) if wl.router else None
+        t0 = time.perf_counter()
+        if wr is not None:
+            M.router_topk(xb, wr, K_TOP)
+        t_r = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        if fmt == "stq":
+            mats = [F.stq1_unpack(p_, r, c_) for p_, (r, c_) in zip(packed, ((I, H), (I, H), (H, I)))]
+            M.expert_ffn_bf16h(mats[0], mats[1], mats[2], X)
+        else:
+            mats = [F.mxfp4_unpack(c_, s_, r, cc) for (c_, s_), (r, cc) in zip(packed, ((I, H), (I, H), (H, I)))]
+            xc, xs = F.mxfp8_quantize(X)
+            M.expert_ffn_mx(mats[0], mats[1], mats[2], F.mxfp8_dequantize(xc, xs))
+        t_e = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        if shared is not None:
+            M.expert_ffn_bf16h(shared[0], shared[1], shared[2], X)
+        t_s = time.perf_counter() - t0
+        nl = sum(1 for L_ in wl.layers if L_["fmt"] == fmt)
+        total += nl * (t_r + K_TOP * t_e + t_s)
+        desc.append(f"{fmt}: router + 1 expert + shared for 1 token, x{K_TOP} experts x{nl} layers")
+    # per step the workload processes T tokens; the sample above is one token
+    return total, float(wl.T), "; ".join(desc)
 
 
-def cpu_baseline(wl, dev):
+def cpu_baseline(wl, dev, budget_s=12.0):
+    """The oracle, single-threaded, on a bounded sample of the workload, scaled to the
+    metric's unit."""
     from threadpoolctl import threadpool_limits
 
     with threadpool_limits(limits=1):
-        t0 = time.perf_counter()
-        if wl.name == "stq_matvec":
-            from oracle import moe as M
-            Wb = wl.W[0].cpu().numpy()
-            xb = wl.x[0].view(torch.int16).cpu().numpy().view(np.uint16)
-            reps = 0
-            while time.perf_counter() - t0 < 10.0:
-                M.stq1_gemv(Wb, 2048, 6144, xb)
-                reps += 1
-            dt = time.perf_counter() - t0
-            return {"value": reps * (STQ_MAT + 6144 * 2 + 2048 * 4) / dt / 1e9, "unit": "GB/s", "cores": 1,
-                    "kind": "oracle", "sample": f"{reps} full matvecs (unpack + float64 matvec)"}
-        _oracle_decode_token(wl, dev)
-        dt = time.perf_counter() - t0
-    return {"value": 1.0 / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "1 token of one layer: router, its 8 experts (unpack + float64 FFN) and the shared expert"}
+        times, t0 = [], time.perf_counter()
+        while True:
+            dt, per_step, desc = _oracle_units(wl, dev)
+            times.append(dt)
+            if time.perf_counter() - t0 > budget_s or len(times) >= 20:
+                break
+    dt = statistics.mean(times)
+    if wl.unit == "GB/s":
+        value = wl.bytes / dt / 1e9
+    else:
+        value = wl.tokens_per_step() / (dt * per_step)
+    return {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",
+            "sample": f"{desc}; {len(times)} repetitions, mean {dt:.2f} s"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    dev = torch.device("cuda", 0)
     import bit_quantized_moe_stq1_b200 as S
 
-    wl = WORKLOADS[args.workload](S, dev)
-    times = []
+    wl = make_workload(args.workload, S, dev)
+    vals = []
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(wl, dev)
+        cb = cpu_baseline(wl, dev, budget_s=0.0)   # one bounded unit per step
         if i >= args.warmup:
-            times.append(cb["value"])
-    value = statistics.mean(times)
-    out = {"impl": "reference", "metric": "MoE-layer tokens/s" if wl.unit != "GB/s" else
-           "STQ1_0 matvec achieved HBM GB/s (2048x6144, 1 token)", "value": value, "unit": wl.unit, "n_gpus": 0,
+            vals.append(cb["value"])
+    value = statistics.mean(vals)
+    out = {"impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": 0,
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": wl.name},
            "cpu_baseline": {"value": value, "unit": wl.unit, "cores": cb["cores"], "kind": "oracle",
@@ -422,13 +569,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
+    args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         run_reference(args)
     else:

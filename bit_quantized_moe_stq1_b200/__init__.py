@@ -51,6 +51,7 @@ SIGNATURES = {
     "stq1_gemv": (_i32, [_vp, _i64, _i64, _vp, _i64, _vp, _vp]),
     "w4a8_gemm": (_i32, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp]),
     "moe_router_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "stq_router_ksplit": (_i32, [_i32]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_workspace_bytes": (_sz, [ctypes.POINTER(MoeDesc)]),
     "moe_workspace_offset": (_sz, [ctypes.POINTER(MoeDesc), _i32]),
@@ -61,7 +62,8 @@ SIGNATURES = {
 }
 
 
-KERNEL_KINDS = ["router_logits", "router_topk", "permute", "quant_x", "gate_up", "down", "combine", "gemv", "gemm"]
+KERNEL_KINDS = ["router_logits", "router_topk", "permute", "quant_x", "gate_up", "down", "combine", "gemv", "gemm",
+                "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down"]
 
 
 class StqTiming(ctypes.Structure):
@@ -76,6 +78,9 @@ class KernelTimer:
     def __init__(self, capacity=512):
         self.cap = capacity
         self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.ev:          # torch creates the CUDA event on first record
+            e.record()
+        torch.cuda.synchronize()
         self._evp = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.ev])
         self._kinds = (_i32 * capacity)()
         self.st = StqTiming(ctypes.cast(self._evp, ctypes.POINTER(ctypes.c_void_p)), capacity,
@@ -231,7 +236,8 @@ def moe_router_topk(x, w_router, k, logits=None, ids=None, w=None, stream=None):
     T, H = x.shape
     E = w_router.shape[0]
     dev = x.device
-    logits = logits if logits is not None else torch.empty((T, E), dtype=torch.float32, device=dev)
+    ks = lib.stq_router_ksplit(H)
+    logits = logits if logits is not None else torch.empty((ks * T, E), dtype=torch.float32, device=dev)
     ids = ids if ids is not None else torch.empty((T, k), dtype=torch.int32, device=dev)
     w = w if w is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
     _check(lib.moe_router_topk(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(logits), _ptr(ids), _ptr(w),

@@ -44,16 +44,23 @@ extern "C" stq_status stq_set_timing(stq_timing* t) {
   return STQ_OK;
 }
 
-StqTimed::StqTimed(int kind, cudaStream_t st) : s(st), slot(-1) {
+static cudaError_t record(cudaEvent_t ev, cudaStream_t st, bool capturing) {
+  // Inside stream capture the record becomes an event-record node of the graph.
+  return capturing ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal) : cudaEventRecord(ev, st);
+}
+
+StqTimed::StqTimed(int kind, cudaStream_t st) : s(st), slot(-1), capturing(false) {
   stq_timing* t = g_timing;
   if (t == nullptr || t->count >= t->capacity) return;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return;
+  capturing = cs == cudaStreamCaptureStatusActive;
   slot = t->count++;
   t->kinds[slot] = kind;
-  cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * slot]), st);
+  record(static_cast<cudaEvent_t>(t->events[2 * slot]), st, capturing);
 }
 
 StqTimed::~StqTimed() {
-  if (slot >= 0 && g_timing != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(g_timing->events[2 * slot + 1]), s);
+  if (slot >= 0 && g_timing != nullptr)
+    record(static_cast<cudaEvent_t>(g_timing->events[2 * slot + 1]), s, capturing);
 }

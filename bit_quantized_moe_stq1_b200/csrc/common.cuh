@@ -62,6 +62,7 @@ struct StqTimed {
   ~StqTimed();
   cudaStream_t s;
   int slot;
+  bool capturing;
 };
 
 template <typename T>

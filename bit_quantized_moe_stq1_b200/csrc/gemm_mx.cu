@@ -1,13 +1,469 @@
-// W4A8 (MXFP4 weights x MXFP8 activations) products.  Placeholder until the
-// tcgen05 block-scaled grouped GEMM lands.
-#include "moe_internal.cuh"
+// W4A8 grouped GEMM on the sm_100a tensor cores: MXFP4 (E2M1, UE8M0 per 32 along K)
+// weights x MXFP8 (E4M3, UE8M0 per 32) activations, FP32 accumulators in TMEM.
+// "Hy4-preview-SF-WFP4AFP8", "Quant Diff": routed experts are FP4 E2M1 weights with
+// FP8 E4M3 activations, group 32, UE8M0 scales; the page notes that FP4 GEMMs need
+// Blackwell.
+//
+// One CTA computes a 128 (weight rows) x NT (tokens of one expert) tile over all of K:
+//   warp 0     producer: per 128-k stage, TMA tile loads of the weights (E2M1 expanded
+//              to one 16-element group per 16 bytes by the TMA, 128-byte swizzle) and of
+//              the token activations (E4M3), and the UE8M0 scales of both, re-laid by the
+//              warp into the scale-factor atom the MMA reads (row m of a 128-row block at
+//              byte (m % 32) * 16 + (m / 32) * 4 + kb);
+//   warp 1     TMEM allocation and, from one thread, tcgen05.cp of the scales into TMEM
+//              and four tcgen05.mma.kind::mxf8f6f4.block_scale (K = 32 each) per stage;
+//   warps 2-5  epilogue from TMEM: FP32 expert outputs, or (gate/up pair) SwiGLU and the
+//              MXFP8 re-quantisation of h along the intermediate dimension.
+// All mbarrier waits are bounded (STQ_ERR_TIMEOUT in the error word, then a clean exit
+// that waits for in-flight copies and frees TMEM).
 
-stq_status moe_mx_experts(const MoeArgs&, int, bool, cudaStream_t) { return STQ_ERR_UNSUPPORTED; }
+#include <cuda_fp8.h>
+#include <cudaTypedefs.h>
+
+#include "moe_internal.cuh"
+#include "tcgen05.cuh"
+
+namespace {
+
+constexpr int kKT = 128;                          // k per stage
+constexpr int kATile = 128 * 128;                 // smem bytes of one 128 x 128 E2M1 tile (expanded)
+constexpr uint32_t kATx = 128 * 128 / 2;          // bytes the TMA delivers for it
+constexpr int kSf = 512;                          // one scale-factor atom: 128 rows x 4 k-blocks
+constexpr int kSmemBudget = 200 * 1024;
+
+template <int NT, bool DUAL>
+struct Cfg {
+  static constexpr int kA2 = DUAL ? kATile : 0;
+  static constexpr int kB = NT * 128;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffA2 = kATile;
+  static constexpr int kOffB = kATile + kA2;
+  static constexpr int kOffSfa = kOffB + kB;
+  static constexpr int kOffSfa2 = kOffSfa + kSf;
+  static constexpr int kOffSfb = kOffSfa + (DUAL ? 2 : 1) * kSf;
+  static constexpr int kStageRaw = kOffSfb + kSf;
+  static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
+  static constexpr int kStagesRaw = kSmemBudget / kStage;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kSmem = kStages * kStage + 1024 /* barriers */ + 1024 /* alignment */;
+  static constexpr int kColAccU = NT;
+  static constexpr int kColSfa = DUAL ? 2 * NT : NT;
+  static constexpr int kColSfa2 = kColSfa + 4;
+  static constexpr int kColSfb = kColSfa + (DUAL ? 8 : 4);
+  static constexpr int kColsUsed = kColSfb + 4;
+  static constexpr uint32_t kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                   : kColsUsed <= 256 ? 256 : 512;
+  static constexpr uint32_t kTx = kATx * (DUAL ? 2 : 1) + uint32_t(kB);
+  static_assert(kStages >= 2, "shared memory budget");
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "tile N");
+  static_assert(kColsUsed <= 512, "TMEM budget");
+};
+
+struct GemmProblem {
+  int R, K, Ptot;               // weight rows per expert, reduction length, activation rows
+  const uint8_t* sa;            // weight scales [E*R][K/32]
+  const uint8_t* sa2;           // second weight matrix's scales (gate/up pair)
+  const uint8_t* sb;            // activation scales [Ptot][K/32]
+  const int32_t* offsets;       // grouped: [E+1]; nullptr = one dense expert of dense_M tokens
+  const int2* ntiles;           // grouped: (expert, first token) per N tile
+  const int32_t* n_ntiles;      // grouped: number of N tiles (device)
+  int dense_M;
+  float* Y;                     // single: [Ptot][R]
+  uint8_t* hq;                  // pair: MXFP8 codes of h [Ptot][R]
+  uint8_t* hs;                  // pair: scales [Ptot][R/32]
+  int32_t* err;
+};
+
+// Scales of 128 rows x 4 k-blocks of stage kt into the atom layout; rows at or past
+// `limit` (absolute) or past `nvalid` (relative) read as zero.
+__device__ __forceinline__ void fill_sf(uint8_t* dst, const uint8_t* src, int row0, int nvalid, int limit, int k32,
+                                        int kt, int lane) {
+  uint32_t v[4];
+#pragma unroll
+  for (int m1 = 0; m1 < 4; ++m1) {
+    const int r = lane + 32 * m1;
+    v[m1] = (r < nvalid && row0 + r < limit)
+                ? *reinterpret_cast<const uint32_t*>(src + size_t(row0 + r) * k32 + size_t(kt) * 4)
+                : 0u;
+  }
+  *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+// E4M3 code of one value with a UE8M0 exponent e already chosen (zero keeps its sign).
+__device__ __forceinline__ uint32_t e4m3_code(float v, float f) {
+  const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v * f, __NV_SATFINITE, __NV_E4M3);
+  uint32_t code = c;
+  if ((code & 0x7Fu) == 0u) code = (__float_as_uint(v) >> 31) << 7;
+  return code;
+}
+
+__device__ __forceinline__ float pow2f(int x) {
+  return x >= -126 ? __uint_as_float(uint32_t(x + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+__device__ __forceinline__ int mxfp8_exponent(float amax) {
+  if (amax == 0.f) return 127;
+  const uint32_t ab = __float_as_uint(amax);
+  const int eb = int(ab >> 23);
+  if (eb == 0) return 0;
+  const int E = eb - 127;
+  const int k = ((ab & 0x7FFFFFu) <= 0x600000u) ? E - 8 : E - 7;  // 448 = 1.75 * 2^8
+  return min(max(k + 127, 0), 254);
+}
+
+template <int NT, bool DUAL>
+__global__ void __launch_bounds__(192, 1)
+    w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                     const __grid_constant__ CUtensorMap tmB, GemmProblem p) {
+  using C = Cfg<NT, DUAL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* accum = empty + C::kStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int MT = p.R / 128;
+  const int item = blockIdx.x;
+  const int mt = item % MT;
+  int e, n0, pos0, cnt;
+  if (p.offsets != nullptr) {
+    const int nti = item / MT;
+    if (nti >= *p.n_ntiles) return;
+    const int2 w = p.ntiles[nti];
+    e = w.x;
+    n0 = w.y;
+    pos0 = p.offsets[e];
+    cnt = p.offsets[e + 1] - pos0;
+  } else {
+    e = 0;
+    n0 = (item / MT) * NT;
+    pos0 = 0;
+    cnt = p.dense_M;
+  }
+  const int nk = p.K / kKT;
+  const int k32 = p.K / 32;
+  const int arow = e * p.R + mt * 128;
+  const int brow = pos0 + n0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(accum, 1);
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&tmA);
+    if (DUAL) tc::prefetch_tensormap(&tmA2);
+    tc::prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_holder, C::kCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    int last_round[C::kStages];
+#pragma unroll
+    for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % C::kStages, r = kt / C::kStages;
+      if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) break;
+      uint8_t* st = smem + s * C::kStage;
+      fill_sf(st + C::kOffSfa, p.sa, arow, 128, 0x7fffffff, k32, kt, lane);
+      if (DUAL) fill_sf(st + C::kOffSfa2, p.sa2, arow, 128, 0x7fffffff, k32, kt, lane);
+      fill_sf(st + C::kOffSfb, p.sb, brow, NT, p.Ptot, k32, kt, lane);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&full[s], C::kTx);
+        tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);
+        if (DUAL) tc::tma_load_2d(st + C::kOffA2, &tmA2, kt * kKT, arow, &full[s]);
+        tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, brow, &full[s]);
+      }
+      last_round[s] = r;
+    }
+    // every issued load has landed before the CTA may exit
+#pragma unroll
+    for (int s = 0; s < C::kStages; ++s)
+      if (last_round[s] >= 0) tc::mbar_wait(&full[s], last_round[s] & 1, p.err);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % C::kStages, r = kt / C::kStages;
+        if (!tc::mbar_wait(&full[s], r & 1, p.err)) break;
+        tc::fence_after_sync();
+        uint8_t* st = smem + s * C::kStage;
+        tc::cp_sf_32x128b_x4(tmem + C::kColSfa, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa)));
+        if (DUAL) tc::cp_sf_32x128b_x4(tmem + C::kColSfa2, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa2)));
+        tc::cp_sf_32x128b_x4(tmem + C::kColSfb, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfb)));
+        const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA));
+        const uint64_t da2 = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA2));
+        const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffB));
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          const uint32_t idesc = tc::idesc_mxf8f6f4(NT, uint32_t(kb), uint32_t(kb));
+          const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+          const uint32_t sfb = (tmem + C::kColSfb) | (uint32_t(kb) << 30);
+          tc::mma_mxf8f6f4(tmem, da + 2 * kb, db + 2 * kb, idesc, (tmem + C::kColSfa) | (uint32_t(kb) << 30), sfb,
+                           acc);
+          if (DUAL)
+            tc::mma_mxf8f6f4(tmem + C::kColAccU, da2 + 2 * kb, db + 2 * kb, idesc,
+                             (tmem + C::kColSfa2) | (uint32_t(kb) << 30), sfb, acc);
+        }
+        tc::commit(&empty[s]);
+      }
+      tc::commit(accum);  // also on an aborted loop, so the epilogue never waits for ever
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const bool ok = tc::mbar_wait(accum, 0, p.err);
+    tc::fence_after_sync();
+    const int f = mt * 128 + 32 * q + lane;  // weight row = output feature
+    const uint32_t tl = tmem + (uint32_t(32 * q) << 16);
+    if (ok) {
+      for (int c0 = 0; c0 < NT; c0 += 16) {
+        if (n0 + c0 >= cnt) break;
+        uint32_t g[16];
+        tc::tmem_ld_x16(tl + c0, g);
+        if constexpr (DUAL) {
+          uint32_t u[16];
+          tc::tmem_ld_x16(tl + C::kColAccU + c0, u);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = n0 + c0 + j;
+            if (col >= cnt) break;
+            const float h = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+            const bool bad = !isfinite(h);
+            float a = bad ? 0.f : fabsf(h);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            const bool anybad = __any_sync(0xffffffffu, bad);
+            const int ex = anybad ? 255 : mxfp8_exponent(a);
+            const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2f(127 - ex));
+            const size_t pos = size_t(pos0 + col);
+            p.hq[pos * p.R + f] = uint8_t(code);
+            if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
+          }
+        } else {
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = n0 + c0 + j;
+            if (col >= cnt) break;
+            p.Y[size_t(pos0 + col) * p.R + f] = __uint_as_float(g[j]);
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, C::kCols);
+  }
+}
+
+// N tiles of every touched expert: (expert, first token of the tile); one CTA.
+__global__ void __launch_bounds__(1024) mx_plan_kernel(const int32_t* __restrict__ counts, int E, int nt,
+                                                       int2* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
+  __shared__ int wsum[32];
+  __shared__ int total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = tid < E ? counts[tid] : 0;
+  const int v = (c + nt - 1) / nt;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int s = wsum[lane];
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    wsum[lane] = si - s;
+    if (lane == 31) total = si;
+  }
+  __syncthreads();
+  const int base = incl - v + wsum[warp];
+  for (int j = 0; j < v; ++j) tiles[base + j] = make_int2(tid, j * nt);
+  if (tid == 0) *n_tiles = total;
+}
+
+// ----------------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// E2M1 weights [rows][K] (two per byte), box 128 x 128, expanded to 16 bytes per 16 elements.
+bool map_e2m1(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K / 2};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E4M3 activations [rows][K] bytes, box 128 x box_rows.
+bool map_u8(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NT, bool DUAL>
+stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
+                       unsigned grid, cudaStream_t s) {
+  using C = Cfg<NT, DUAL>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<NT, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+        cudaSuccess)
+      return STQ_ERR_CUDA;
+    configured = true;
+  }
+  if (grid == 0) return STQ_OK;
+  w4a8_gemm_kernel<NT, DUAL><<<grid, 192, C::kSmem, s>>>(a, a2, b, p);
+  return stq_launch_status();
+}
+
+template <bool DUAL>
+stq_status launch_nt(int nt, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
+                     unsigned grid, cudaStream_t s) {
+  switch (nt) {
+    case 16: return launch_gemm<16, DUAL>(a, a2, b, p, grid, s);
+    case 32: return launch_gemm<32, DUAL>(a, a2, b, p, grid, s);
+    case 64: return launch_gemm<64, DUAL>(a, a2, b, p, grid, s);
+    default: return launch_gemm<128, DUAL>(a, a2, b, p, grid, s);
+  }
+}
+
+int pick_nt(int64_t tokens_per_expert) {
+  return tokens_per_expert <= 16 ? 16 : tokens_per_expert <= 32 ? 32 : tokens_per_expert <= 64 ? 64 : 128;
+}
+
+}  // namespace
+
+// Defined in moe.cu: the BF16 shared-expert CTAs of the STQ1_0 kernels.
+stq_status moe_shared_expert_bf16(const MoeArgs& a, cudaStream_t s);
+
+stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStream_t s) {
+  (void)slots;
+  const int P = a.P;
+  // 1. activations -> MXFP8 in sorted (expert-grouped) order
+  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.xq, a.xs, s);
+  if (st != STQ_OK) return st;
+  // 2. N tiles of the touched experts
+  const int nt = pick_nt(int64_t(P) / (a.E < P ? a.E : P));
+  {
+    StqTimed tm(STQ_K_PLAN, s);
+    mx_plan_kernel<<<1, 1024, 0, s>>>(a.counts, a.E, nt, a.ntiles, a.n_ntiles);
+  }
+  if ((st = stq_launch_status()) != STQ_OK) return st;
+  const int max_tiles = P / nt + (a.E < P ? a.E : P);
+  // 3. gate/up pair with SwiGLU and MXFP8 h
+  CUtensorMap mg, mu, mx, md, mh;
+  if (!map_e2m1(&mg, a.wg, uint64_t(a.H), uint64_t(a.E) * a.I) ||
+      !map_e2m1(&mu, a.wu, uint64_t(a.H), uint64_t(a.E) * a.I) || !map_u8(&mx, a.xq, a.H, P, nt) ||
+      !map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !map_u8(&mh, a.hq, a.I, P, nt))
+    return STQ_ERR_CUDA;
+  GemmProblem gp{};
+  gp.R = a.I;
+  gp.K = a.H;
+  gp.Ptot = P;
+  gp.sa = a.gsc;
+  gp.sa2 = a.usc;
+  gp.sb = a.xs;
+  gp.offsets = a.offsets;
+  gp.ntiles = a.ntiles;
+  gp.n_ntiles = a.n_ntiles;
+  gp.hq = a.hq;
+  gp.hs = a.hs;
+  gp.err = a.err;
+  {
+    StqTimed tm(STQ_K_GATE_UP_MX, s);
+    st = launch_nt<true>(nt, mg, mu, mx, gp, unsigned(max_tiles * (a.I / 128)), s);
+  }
+  if (st != STQ_OK) return st;
+  if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
+  // 4. down
+  GemmProblem dp = gp;
+  dp.R = a.H;
+  dp.K = a.I;
+  dp.sa = a.dsc;
+  dp.sa2 = nullptr;
+  dp.sb = a.hs;
+  dp.Y = a.Y;
+  dp.hq = nullptr;
+  dp.hs = nullptr;
+  {
+    StqTimed tm(STQ_K_DOWN_MX, s);
+    st = launch_nt<false>(nt, md, md, mh, dp, unsigned(max_tiles * (a.H / 128)), s);
+  }
+  return st;
+}
 
 extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales, int64_t N, int64_t K,
                                 const uint8_t* a_codes, const uint8_t* a_scales, int64_t M, float* y, int32_t* err,
                                 stq_stream_t stream) {
-  (void)w_codes; (void)w_scales; (void)N; (void)K; (void)a_codes; (void)a_scales; (void)M; (void)y; (void)err;
-  (void)stream;
-  return STQ_ERR_UNSUPPORTED;
+  STQ_HOST_CHECK(N >= 0 && K >= 0 && M >= 0, STQ_ERR_INVALID_ARG);
+  if (N == 0 || M == 0) return STQ_OK;
+  STQ_HOST_CHECK(w_codes && w_scales && a_codes && a_scales && y, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(N % 128 == 0 && K % 128 == 0 && K > 0, STQ_ERR_SHAPE);
+  STQ_HOST_CHECK(N < (int64_t(1) << 31) && M < (int64_t(1) << 31) && K < (int64_t(1) << 31), STQ_ERR_SHAPE);
+  STQ_HOST_CHECK((reinterpret_cast<uintptr_t>(w_codes) & 31u) == 0 && stq_aligned16(a_codes) && stq_aligned16(y) &&
+                     (reinterpret_cast<uintptr_t>(w_scales) & 3u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(a_scales) & 3u) == 0,
+                 STQ_ERR_ALIGN);
+  cudaStream_t s = stq_cuda_stream(stream);
+  const int nt = pick_nt(M);
+  CUtensorMap ma, mb;
+  if (!map_e2m1(&ma, w_codes, uint64_t(K), uint64_t(N)) || !map_u8(&mb, a_codes, uint64_t(K), uint64_t(M), nt))
+    return STQ_ERR_CUDA;
+  GemmProblem p{};
+  p.R = int(N);
+  p.K = int(K);
+  p.Ptot = int(M);
+  p.sa = w_scales;
+  p.sb = a_scales;
+  p.dense_M = int(M);
+  p.Y = y;
+  p.err = err;
+  const unsigned grid = unsigned((N / 128) * ((M + nt - 1) / nt));
+  StqTimed tm(STQ_K_GEMM, s);
+  return launch_nt<false>(nt, ma, ma, mb, p, grid, s);
 }

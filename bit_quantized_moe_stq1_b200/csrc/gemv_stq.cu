@@ -43,8 +43,9 @@ __global__ void __launch_bounds__(128) stq1_gemv_kernel(const uint8_t* __restric
 
 extern "C" stq_status stq1_gemv(const uint8_t* W, int64_t rows, int64_t K, const uint16_t* x, int64_t n, float* y,
                                 stq_stream_t stream) {
-  STQ_HOST_CHECK(W && x && y, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(rows >= 0 && K >= 0 && n >= 0, STQ_ERR_INVALID_ARG);
+  if (rows == 0 || n == 0) return STQ_OK;
+  STQ_HOST_CHECK(W && x && y, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(rows % 16 == 0 && K % 256 == 0, STQ_ERR_SHAPE);
   STQ_HOST_CHECK(stq_aligned16(W) && stq_aligned16(x) && stq_aligned16(y), STQ_ERR_ALIGN);
   if (rows == 0 || n == 0) return STQ_OK;

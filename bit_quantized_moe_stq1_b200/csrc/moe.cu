@@ -136,40 +136,62 @@ __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
   return acc;
 }
 
-// logits[t, e] = sum_h x[t, h] wr[e, h] (FP32).  CTA = 8 warps over 4 experts; warp
-// w takes expert 4*blockIdx + (w & 3) and half (w >> 2) of H.
-__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
+// Router logits, split over K: part[ks][t][e] = sum over the ks-th slice of H of
+// x[t, h] wr[e, h] (bf16 mma.sync, FP32 accumulate).  CTA = 16 experts x one K slice;
+// its four warps split the slice and are summed in a fixed order.
+__global__ void __launch_bounds__(128) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const uint16_t* __restrict__ wr, int T, int H, int E,
-                                                            float* __restrict__ logits) {
-  __shared__ float red[2][4][8];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int e = blockIdx.x * 4 + (warp & 3), half = warp >> 2;
-  const int hh = H / 2;
-  const int k0 = half * hh, k1 = k0 + hh;
-  for (int t0 = 0; t0 < T; t0 += 8) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (e < E) {
-      for (int k = k0 + lane * 8; k < k1; k += 256) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(wr + size_t(e) * H + k);
+                                                            int KS, float* __restrict__ part) {
+  __shared__ float red[4][4][4][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int e0 = (blockIdx.x / KS) * 16, ks = blockIdx.x % KS;
+  const int slice = H / KS, kq = slice / 4;
+  const int k0 = ks * slice + warp * kq, k1 = k0 + kq;
+  const int er = min(e0 + g, E - 1);                // rows past E read a valid row; results dropped
+  const uint16_t* rowg[1] = {wr + size_t(er) * H};
+  const int er8 = min(e0 + g + 8, E - 1);
+  for (int t0 = 0; t0 < T; t0 += 32) {
+    const uint16_t* xr[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (t0 + j < T) acc[j] = dot8_bf16(wv, *reinterpret_cast<const uint4*>(x + size_t(t0 + j) * H + k), acc[j]);
+    for (int c = 0; c < 4; ++c) {
+      const int tok = t0 + 8 * c + g;
+      xr[c] = tok < T ? x + size_t(tok) * H : nullptr;
+    }
+    float acc[1][4][4] = {};
+    // rows g+8 come from 8*ld further; a ragged last expert tile (warp-uniform test)
+    // takes rows g and g+8 through two single-row passes over clamped rows
+    if (e0 + 16 <= E) {
+      bf16_warp_gemv<1, 4>(rowg, H, k0, k1, xr, acc);
+    } else {
+      // ragged expert tile: process rows g and g+8 through separate single-row passes
+      const uint16_t* r0[1] = {wr + size_t(er) * H};
+      float a0[1][4][4] = {}, a1[1][4][4] = {};
+      bf16_warp_gemv<1, 4>(r0, 0, k0, k1, xr, a0);
+      const uint16_t* r1[1] = {wr + size_t(er8) * H};
+      bf16_warp_gemv<1, 4>(r1, 0, k0, k1, xr, a1);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[0][c][0] = a0[0][c][0];
+        acc[0][c][1] = a0[0][c][1];
+        acc[0][c][2] = a1[0][c][2];
+        acc[0][c][3] = a1[0][c][3];
       }
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(kFull, acc[j], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) red[half][warp & 3][j] = acc[j];
-    }
+      for (int j = 0; j < 4; ++j) red[warp][c][j][lane] = acc[0][c][j];
     __syncthreads();
-    if (threadIdx.x < 32) {
-      const int ei = threadIdx.x >> 3, j = threadIdx.x & 7;
-      const int ee = blockIdx.x * 4 + ei;
-      if (ee < E && t0 + j < T) logits[size_t(t0 + j) * E + ee] = red[0][ei][j] + red[1][ei][j];
+    if (warp == 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float v = ((red[0][c][j][lane] + red[1][c][j][lane]) + red[2][c][j][lane]) + red[3][c][j][lane];
+          const int tok = t0 + 8 * c + 2 * t + (j & 1);
+          const int e = e0 + g + 8 * (j >> 1);
+          if (tok < T && e < E) part[(size_t(ks) * T + tok) * E + e] = v;
+        }
     }
     __syncthreads();
   }
@@ -177,8 +199,8 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 
 // One warp per token: softmax over E (max-shifted exp), top-k by probability with
 // ties to the lower id, weights renormalised over the chosen k.
-__global__ void router_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ ids,
-                                   float* __restrict__ w) {
+__global__ void router_topk_kernel(float* __restrict__ logits, int T, int E, int KS, int k,
+                                   int32_t* __restrict__ ids, float* __restrict__ w) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -189,7 +211,13 @@ __global__ void router_topk_kernel(const float* __restrict__ logits, int T, int 
 #pragma unroll
   for (int j = 0; j < kMaxPer; ++j) {
     const int e = lane + 32 * j;
-    p[j] = (j < per && e < E) ? logits[size_t(t) * E + e] : -INFINITY;
+    float v = -INFINITY;
+    if (j < per && e < E) {
+      v = logits[size_t(t) * E + e];
+      for (int ks = 1; ks < KS; ++ks) v += logits[(size_t(ks) * T + t) * E + e];
+      logits[size_t(t) * E + e] = v;
+    }
+    p[j] = v;
     m = fmaxf(m, p[j]);
   }
 #pragma unroll
@@ -435,10 +463,12 @@ MoeWsLayout moe_ws_layout(const moe_desc& d) {
   L.inv = take(P * 4);
   L.h = take((P + T) * I * 2);
   L.Y = take((P + T) * H * 4);
-  L.xq = take(T * H);
-  L.xs = take(T * (H / 32));
+  L.xq = take(P * H);
+  L.xs = take(P * (H / 32));
   L.hq = take(P * I);
   L.hs = take(P * (I / 32));
+  L.ntiles = take((P / 16 + E + 1) * 8);
+  L.n_ntiles = take(4);
   L.total = o;
   return L;
 }
@@ -459,6 +489,8 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
   w.xs = b + L.xs;
   w.hq = b + L.hq;
   w.hs = b + L.hs;
+  w.ntiles = reinterpret_cast<int2*>(b + L.ntiles);
+  w.n_ntiles = reinterpret_cast<int32_t*>(b + L.n_ntiles);
   return w;
 }
 
@@ -470,6 +502,25 @@ static bool desc_ok(const moe_desc* d) {
 extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
   if (!desc_ok(d)) return 0;
   return moe_ws_layout(*d).total;
+}
+
+// The BF16 shared expert alone (used by MXFP4 layers): the shared CTAs of the two
+// STQ1_0 kernels.
+stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
+  MoeArgs a = a0;
+  a.n_shared_cta = a.I / 16;
+  {
+    StqTimed tm(STQ_K_SHARED_GATE_UP, s);
+    moe_gateup_stq_kernel<<<unsigned(a.n_shared_cta), 128, 0, s>>>(a);
+  }
+  stq_status st = stq_launch_status();
+  if (st != STQ_OK) return st;
+  a.n_shared_cta = a.H / 16;
+  {
+    StqTimed tm(STQ_K_SHARED_DOWN, s);
+    moe_down_stq_kernel<<<unsigned(a.n_shared_cta), 128, 0, s>>>(a);
+  }
+  return stq_launch_status();
 }
 
 extern "C" size_t moe_workspace_offset(const moe_desc* d, int32_t region) {
@@ -547,9 +598,10 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   a.wg = w->gate; a.wu = w->up; a.wd = w->down;
   a.gsc = w->gate_sc; a.usc = w->up_sc; a.dsc = w->down_sc;
   a.sg = w->sh_gate; a.su = w->sh_up; a.sd = w->sh_down;
-  a.offsets = ws.offsets; a.perm = ws.perm; a.tlist = ws.tlist; a.ntouched = ws.ntouched;
+  a.counts = ws.counts; a.offsets = ws.offsets; a.perm = ws.perm; a.tlist = ws.tlist; a.ntouched = ws.ntouched;
   a.h = ws.h; a.Y = ws.Y;
   a.xq = ws.xq; a.xs = ws.xs; a.hq = ws.hq; a.hs = ws.hs;
+  a.ntiles = ws.ntiles; a.n_ntiles = ws.n_ntiles;
   a.err = ws.err;
   const int slots = d->E < P ? d->E : P;
 
@@ -573,24 +625,31 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   return moe_launch_combine(*d, P, ws, topk_w, has_shared, x, y, s);
 }
 
+extern "C" int32_t stq_router_ksplit(int32_t H) {
+  for (int ks = 8; ks > 1; ks >>= 1)
+    if (H % (128 * ks) == 0) return ks;
+  return 1;
+}
+
 extern "C" stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T, int32_t H, int32_t E,
                                       int32_t k, float* logits, int32_t* topk_ids, float* topk_w,
                                       stq_stream_t stream) {
   STQ_HOST_CHECK(x && w_router && logits && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
-  STQ_HOST_CHECK(H % 16 == 0, STQ_ERR_SHAPE);
+  STQ_HOST_CHECK(H % 128 == 0, STQ_ERR_SHAPE);
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
   if (T == 0) return STQ_OK;
   cudaStream_t s = stq_cuda_stream(stream);
+  const int KS = stq_router_ksplit(H);
   {
     StqTimed tm(STQ_K_ROUTER_LOGITS, s);
-    router_logits_kernel<<<unsigned(ceil_div(E, 4)), 256, 0, s>>>(x, w_router, T, H, E, logits);
+    router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 128, 0, s>>>(x, w_router, T, H, E, KS, logits);
   }
   stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
   {
     StqTimed tm(STQ_K_ROUTER_TOPK, s);
-    router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(logits, T, E, k, topk_ids, topk_w);
+    router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(logits, T, E, KS, k, topk_ids, topk_w);
   }
   return stq_launch_status();
 }

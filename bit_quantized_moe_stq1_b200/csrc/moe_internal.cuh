@@ -4,7 +4,7 @@
 #include "common.cuh"
 
 struct MoeWsLayout {
-  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, total;
+  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, ntiles, n_ntiles, total;
 };
 
 // Device pointers into the caller's workspace.
@@ -18,10 +18,12 @@ struct MoeWs {
   int32_t* inv;
   uint16_t* h;   // [(P+T), I] bf16: routed pairs (sorted order) then shared-expert tokens
   float* Y;      // [(P+T), H] fp32
-  uint8_t* xq;   // [T, H]     MXFP8 codes of x
-  uint8_t* xs;   // [T, H/32]
+  uint8_t* xq;   // [P, H]     MXFP8 codes of x, rows in sorted pair order (MXFP4 experts)
+  uint8_t* xs;   // [P, H/32]
   uint8_t* hq;   // [P, I]     MXFP8 codes of h (MXFP4 experts)
   uint8_t* hs;   // [P, I/32]
+  int2* ntiles;  // [P/16 + E] (expert, first token) of each GEMM N tile
+  int32_t* n_ntiles;
 };
 
 // Kernel arguments (by value).
@@ -31,10 +33,12 @@ struct MoeArgs {
   const uint8_t *wg, *wu, *wd;     // routed experts (STQ1_0 bytes or MXFP4 codes)
   const uint8_t *gsc, *usc, *dsc;  // MXFP4 scales
   const uint16_t *sg, *su, *sd;    // shared expert, bf16
-  const int32_t *offsets, *perm, *tlist, *ntouched;
+  const int32_t *counts, *offsets, *perm, *tlist, *ntouched;
   uint16_t* h;
   float* Y;
   uint8_t *xq, *xs, *hq, *hs;
+  int2* ntiles;
+  int32_t* n_ntiles;
   int32_t* err;
   int n_shared_cta;
 };
@@ -48,3 +52,6 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
 // BF16 -> MXFP8 quantisation launch (pack.cu).
 stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales,
                                      cudaStream_t s);
+// Same, with output row r taken from input row rowmap[r] / k (gather into sorted pair order).
+stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int64_t K, const int32_t* rowmap, int k,
+                                            uint8_t* codes, uint8_t* scales, cudaStream_t s);

@@ -205,7 +205,8 @@ __global__ void mxfp4_unpack_kernel(const uint8_t* __restrict__ codes, const uin
 
 // Four lanes per 32-element group, eight elements per lane.
 __global__ void mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
-                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                        const int32_t* __restrict__ rowmap, int k) {
   const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t gi = tid >> 2;
   const int part = int(tid & 3);
@@ -215,7 +216,9 @@ __global__ void mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t 
   float amax = 0.f;
   bool bad = false;
   if (active) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(x + gi * 32 + part * 8);
+    const int64_t gpr = K / 32, row = gi / gpr, col = gi % gpr;
+    const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
+    const uint4 raw = *reinterpret_cast<const uint4*>(x + src * K + col * 32 + part * 8);
     const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -314,7 +317,18 @@ stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K,
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
-  mxfp8_quant_bf16_kernel<<<unsigned(ceil_div<int64_t>(threads, 256)), 256, 0, s>>>(x, rows, K, codes, scales);
+  mxfp8_quant_bf16_kernel<<<unsigned(ceil_div<int64_t>(threads, 256)), 256, 0, s>>>(x, rows, K, codes, scales,
+                                                                                   nullptr, 1);
+  return stq_launch_status();
+}
+
+stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int64_t K, const int32_t* rowmap, int k,
+                                            uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+  const int64_t threads = rows * (K / 32) * 4;
+  if (threads == 0) return STQ_OK;
+  StqTimed tm(STQ_K_QUANT_X, s);
+  mxfp8_quant_bf16_kernel<<<unsigned(ceil_div<int64_t>(threads, 256)), 256, 0, s>>>(x, rows, K, codes, scales,
+                                                                                   rowmap, k);
   return stq_launch_status();
 }
 

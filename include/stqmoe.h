@@ -131,7 +131,8 @@ stq_status mxfp8_quantize_bf16(const uint16_t* x, int64_t rows, int64_t K,
 
 /* y[n, r] = sum_k W[r, k] x[n, k] (FP32 accumulate) for an STQ1_0 matrix W
  * [rows, K] and bf16 activations x [n, K]; y float32 [n, rows].  Tolerance
- * |y - y_ref| <= 1e-3 * sum_k |W x| + 1e-5.  rows % 16 == 0, K % 256 == 0. */
+ * |y - y_ref| <= 1e-3 * sum_k |W x| + 1e-5.  rows % 16 == 0, K % 256 == 0.
+ * n == 0 or rows == 0 is a no-op (pointers may then be NULL). */
 stq_status stq1_gemv(const uint8_t* W, int64_t rows, int64_t K, const uint16_t* x,
                      int64_t n, float* y, stq_stream_t stream);
 
@@ -152,9 +153,11 @@ enum { STQ_FMT_STQ1_0 = 0, STQ_FMT_MXFP4 = 1 };
 
 /* Router: logits = x Wr^T (FP32 accumulate), softmax over E, top-k by
  * probability (ties -> lower id), weights renormalised over the k chosen.
- * x bf16 [T, H], w_router bf16 [E, H] -> logits f32 [T, E] (caller-owned; also
- * the scratch of the top-k step), topk_ids int32 [T, k], topk_w f32 [T, k].
- * E <= 1024, k <= 32, k <= E, H % 16 == 0. */
+ * x bf16 [T, H], w_router bf16 [E, H] -> topk_ids int32 [T, k], topk_w f32 [T, k].
+ * logits: caller-owned f32 scratch of stq_router_ksplit(H) * T * E floats (the
+ * logits are summed over that many slices of H); on return its first T*E floats
+ * hold the logits [T, E].  E <= 1024, k <= 32, k <= E, H % 128 == 0. */
+int32_t stq_router_ksplit(int32_t H);
 stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T,
                            int32_t H, int32_t E, int32_t k, float* logits,
                            int32_t* topk_ids, float* topk_w, stq_stream_t stream);
@@ -226,15 +229,16 @@ stq_status moe_get_device_error(void* workspace, stq_stream_t stream);
 
 /* Kernel kinds reported by the timing hook. */
 enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
-       STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM, STQ_K_COUNT };
+       STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM,
+       STQ_K_GATE_UP_MX, STQ_K_DOWN_MX, STQ_K_PLAN, STQ_K_SHARED_GATE_UP, STQ_K_SHARED_DOWN, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
- * moe_router_topk, moe_expert_forward, stq1_gemv and w4a8_gemm outside stream
- * capture is bracketed by cudaEventRecord(events[2n]) / (events[2n+1]) on the
- * call's stream, kinds[n] is set to its STQ_K_* kind and n = count++ (until
- * capacity pairs are used).  events: cudaEvent_t[2*capacity] created with timing.
- * Process-wide, not thread-safe; NULL uninstalls.  Used by the benchmark to time
- * each kernel on its own stream. */
+ * moe_router_topk, moe_expert_forward, stq1_gemv and w4a8_gemm is bracketed by
+ * event records of events[2n] / events[2n+1] on the call's stream (inside stream
+ * capture as external event-record nodes of the graph), kinds[n] is set to its
+ * STQ_K_* kind and n = count++ (until capacity pairs are used).  events:
+ * cudaEvent_t[2*capacity] created with timing.  Process-wide, not thread-safe;
+ * NULL uninstalls.  Used by the benchmark to time each kernel on its own stream. */
 typedef struct {
   void* const* events;
   int32_t capacity;

@@ -85,7 +85,7 @@ def test_mxfp4_pack_unpack_bitexact(S, rows, K):
 
 def test_mxfp4_unpack_edge_scales(S):
     rows, K = 2, 64
-    codes = np.arange(64, dtype=np.uint8).reshape(2, 32) * 9 % 256
+    codes = (np.arange(64).reshape(2, 32) * 9 % 256).astype(np.uint8)
     scales = np.array([[0, 254], [127, 255]], dtype=np.uint8)
     got = S.mxfp4_unpack(torch.from_numpy(codes.copy()).to(DEV), torch.from_numpy(scales).to(DEV), rows, K).cpu().numpy()
     ref = F.mxfp4_unpack_f32(codes, scales, rows, K)
