@@ -517,14 +517,15 @@ def _oracle_units(wl, dev):
         t_s = time.perf_counter() - t0
         nl = sum(1 for L_ in wl.layers if L_["fmt"] == fmt)
         total += nl * (t_r + K_TOP * t_e + t_s)
-        desc.append(f"{fmt}: router + 1 expert + shared for 1 token, x{K_TOP} experts x{nl} layers")
+        desc.append(f"{fmt}: 1 token through the router ({t_r:.2f} s), one expert ({t_e:.2f} s) and the shared "
+                    f"expert ({t_s:.2f} s), scaled to {K_TOP} experts x {nl} layers")
     # per step the workload processes T tokens; the sample above is one token
     return total, float(wl.T), "; ".join(desc)
 
 
 def cpu_baseline(wl, dev, budget_s=12.0):
     """The oracle, single-threaded, on a bounded sample of the workload, scaled to the
-    metric's unit."""
+    metric's unit.  Small units repeat until budget_s has passed."""
     from threadpoolctl import threadpool_limits
 
     with threadpool_limits(limits=1):
@@ -532,7 +533,7 @@ def cpu_baseline(wl, dev, budget_s=12.0):
         while True:
             dt, per_step, desc = _oracle_units(wl, dev)
             times.append(dt)
-            if time.perf_counter() - t0 > budget_s or len(times) >= 20:
+            if time.perf_counter() - t0 > budget_s or len(times) >= 20 or isinstance(wl, MoeLayers):
                 break
     dt = statistics.mean(times)
     if wl.unit == "GB/s":

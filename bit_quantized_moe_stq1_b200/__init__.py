@@ -242,7 +242,12 @@ def moe_router_topk(x, w_router, k, logits=None, ids=None, w=None, stream=None):
     w = w if w is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
     _check(lib.moe_router_topk(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(logits), _ptr(ids), _ptr(w),
                                _stream(stream)), "moe_router_topk")
-    return ids, w, logits
+    return ids, w, logits[:T]
+
+
+def router_scratch(T, H, E, device):
+    """Logits scratch of the router: stq_router_ksplit(H) * T rows of E floats."""
+    return torch.empty((lib.stq_router_ksplit(H) * T, E), dtype=torch.float32, device=device)
 
 
 def moe_permute(topk_ids, E, err=None, stream=None):

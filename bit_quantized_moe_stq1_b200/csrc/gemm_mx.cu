@@ -74,18 +74,22 @@ struct GemmProblem {
   int32_t* err;
 };
 
-// Scales of 128 rows x 4 k-blocks of stage kt into the atom layout; rows at or past
-// `limit` (absolute) or past `nvalid` (relative) read as zero.
-__device__ __forceinline__ void fill_sf(uint8_t* dst, const uint8_t* src, int row0, int nvalid, int limit, int k32,
-                                        int kt, int lane) {
-  uint32_t v[4];
+// Scales of stage kt for the four 32-row slices m1 of a 128-row block: lane m0 reads
+// the 4 bytes (4 k-blocks) of rows m0 + 32*m1.  Rows at or past `limit` (absolute)
+// or `nvalid` (relative), and stages past nk, read as zero.
+__device__ __forceinline__ void load_sf(uint32_t (&v)[4], const uint8_t* src, int row0, int nvalid, int limit,
+                                        int k32, int kt, int nk, int lane) {
 #pragma unroll
   for (int m1 = 0; m1 < 4; ++m1) {
     const int r = lane + 32 * m1;
-    v[m1] = (r < nvalid && row0 + r < limit)
-                ? *reinterpret_cast<const uint32_t*>(src + size_t(row0 + r) * k32 + size_t(kt) * 4)
+    v[m1] = (kt < nk && r < nvalid && row0 + r < limit)
+                ? __ldg(reinterpret_cast<const uint32_t*>(src + size_t(row0 + r) * k32 + size_t(kt) * 4))
                 : 0u;
   }
+}
+
+// Store them into the scale-factor atom: row m = m0 + 32*m1 at byte m0*16 + m1*4 + kb.
+__device__ __forceinline__ void store_sf(uint8_t* dst, const uint32_t (&v)[4], int lane) {
   *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
@@ -166,25 +170,47 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
+    // Scale factors are read kPf stages ahead into a register ring, so no stage waits
+    // for a global load before its TMA is issued.
+    constexpr int kPf = 4;
     int last_round[C::kStages];
 #pragma unroll
     for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % C::kStages, r = kt / C::kStages;
-      if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) break;
-      uint8_t* st = smem + s * C::kStage;
-      fill_sf(st + C::kOffSfa, p.sa, arow, 128, 0x7fffffff, k32, kt, lane);
-      if (DUAL) fill_sf(st + C::kOffSfa2, p.sa2, arow, 128, 0x7fffffff, k32, kt, lane);
-      fill_sf(st + C::kOffSfb, p.sb, brow, NT, p.Ptot, k32, kt, lane);
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tc::mbar_arrive_expect_tx(&full[s], C::kTx);
-        tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);
-        if (DUAL) tc::tma_load_2d(st + C::kOffA2, &tmA2, kt * kKT, arow, &full[s]);
-        tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, brow, &full[s]);
+    uint32_t ra[kPf][4], ra2[kPf][4], rb[kPf][4];
+#pragma unroll
+    for (int d = 0; d < kPf; ++d) {
+      load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, d, nk, lane);
+      if (DUAL) load_sf(ra2[d], p.sa2, arow, 128, 0x7fffffff, k32, d, nk, lane);
+      load_sf(rb[d], p.sb, brow, NT, p.Ptot, k32, d, nk, lane);
+    }
+    bool ok = true;
+    for (int k0 = 0; k0 < nk && ok; k0 += kPf) {
+#pragma unroll
+      for (int d = 0; d < kPf; ++d) {
+        const int kt = k0 + d;
+        if (kt >= nk) break;
+        const int s = kt % C::kStages, r = kt / C::kStages;
+        if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * C::kStage;
+        store_sf(st + C::kOffSfa, ra[d], lane);
+        if (DUAL) store_sf(st + C::kOffSfa2, ra2[d], lane);
+        store_sf(st + C::kOffSfb, rb[d], lane);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(&full[s], C::kTx);
+          tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);
+          if (DUAL) tc::tma_load_2d(st + C::kOffA2, &tmA2, kt * kKT, arow, &full[s]);
+          tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, brow, &full[s]);
+        }
+        last_round[s] = r;
+        load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
+        if (DUAL) load_sf(ra2[d], p.sa2, arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
+        load_sf(rb[d], p.sb, brow, NT, p.Ptot, k32, kt + kPf, nk, lane);
       }
-      last_round[s] = r;
     }
     // every issued load has landed before the CTA may exit
 #pragma unroll
@@ -450,7 +476,8 @@ extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales,
                      (reinterpret_cast<uintptr_t>(a_scales) & 3u) == 0,
                  STQ_ERR_ALIGN);
   cudaStream_t s = stq_cuda_stream(stream);
-  const int nt = pick_nt(M);
+  int nt = pick_nt(M);
+  while (nt > 16 && (N / 128) * ((M + nt - 1) / nt) < 148) nt /= 2;  // fill the SMs
   CUtensorMap ma, mb;
   if (!map_e2m1(&ma, w_codes, uint64_t(K), uint64_t(N)) || !map_u8(&mb, a_codes, uint64_t(K), uint64_t(M), nt))
     return STQ_ERR_CUDA;
