@@ -52,6 +52,7 @@ SIGNATURES = {
     "w4a8_gemm": (_i32, [_vp, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp]),
     "moe_router_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
     "stq_router_ksplit": (_i32, [_i32]),
+    "moe_router_topk_static": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_workspace_bytes": (_sz, [ctypes.POINTER(MoeDesc)]),
     "moe_workspace_offset": (_sz, [ctypes.POINTER(MoeDesc), _i32]),
@@ -243,6 +244,19 @@ def moe_router_topk(x, w_router, k, logits=None, ids=None, w=None, stream=None):
     _check(lib.moe_router_topk(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(logits), _ptr(ids), _ptr(w),
                                _stream(stream)), "moe_router_topk")
     return ids, w, logits[:T]
+
+
+def moe_router_topk_static(x, w_router, k, ids=None, w=None, stream=None):
+    """Router whose logits scratch is the library's own fixed per-GPU array (no
+    scratch argument; see moe_router_topk_static in include/stqmoe.h)."""
+    _dev(x, w_router)
+    T, H = x.shape
+    E = w_router.shape[0]
+    ids = ids if ids is not None else torch.empty((T, k), dtype=torch.int32, device=x.device)
+    w = w if w is not None else torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _check(lib.moe_router_topk_static(_ptr(x), _ptr(w_router), T, H, E, k, _ptr(ids), _ptr(w), _stream(stream)),
+           "moe_router_topk_static")
+    return ids, w
 
 
 def router_scratch(T, H, E, device):

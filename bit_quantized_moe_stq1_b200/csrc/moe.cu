@@ -667,3 +667,58 @@ extern "C" stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k,
   ws.tlist = tlist; ws.ntouched = ntouched;
   return moe_launch_permute(topk_ids, int(P64), E, ws, stq_cuda_stream(stream));
 }
+
+// ----------------------------------------------------------------------------- router, no allocation
+//
+// The same two router kernels as moe_router_topk, for callers that cannot hand the
+// library a scratch buffer: the logits partial sums live in a fixed array compiled
+// into this module, one copy on every GPU that loads the library, kept until the
+// process exits.  Host code may not pass the array's name to a kernel (on the host
+// it is only a stand-in for the symbol), so its device address is looked up once
+// per device with cudaGetSymbolAddress and cached.
+
+constexpr size_t kRouterStaticFloats = size_t(1) << 19;  // 524,288 floats = 2 MiB per GPU
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) float g_router_scratch[kRouterStaticFloats];
+
+namespace {
+
+// Device address of g_router_scratch on the current device (looked up on first use).
+stq_status router_static_scratch(float** out) {
+  static float* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return STQ_ERR_CUDA;
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_router_scratch) != cudaSuccess || p == nullptr) return STQ_ERR_CUDA;
+    addr[dev] = static_cast<float*>(p);
+  }
+  *out = addr[dev];
+  return STQ_OK;
+}
+
+}  // namespace
+
+extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router, int32_t T, int32_t H,
+                                             int32_t E, int32_t k, int32_t* topk_ids, float* topk_w,
+                                             stq_stream_t stream) {
+  STQ_HOST_CHECK(x && w_router && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(H % 128 == 0, STQ_ERR_SHAPE);
+  STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
+  const int KS = stq_router_ksplit(H);
+  STQ_HOST_CHECK(size_t(KS) * size_t(T) * size_t(E) <= kRouterStaticFloats, STQ_ERR_WORKSPACE);
+  float* scratch = nullptr;
+  const stq_status st0 = router_static_scratch(&scratch);
+  if (st0 != STQ_OK) return st0;
+  if (T == 0) return STQ_OK;
+  cudaStream_t s = stq_cuda_stream(stream);
+  // Every entry the top-k step reads is written first by the logits step, so the
+  // array needs no clearing between calls.
+  router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 128, 0, s>>>(x, w_router, T, H, E, KS, scratch);
+  stq_status st = stq_launch_status();
+  if (st != STQ_OK) return st;
+  router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(scratch, T, E, KS, k, topk_ids, topk_w);
+  return stq_launch_status();
+}

@@ -173,6 +173,25 @@ stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                        int32_t* tlist, int32_t* ntouched, int32_t* err,
                        stq_stream_t stream);
 
+/* Router without a scratch argument (no counterpart on the pages; a convenience of
+ * this library).  Same result as moe_router_topk, for callers that cannot allocate
+ * device memory for scratch: code that must not call cudaMalloc (for instance a
+ * host program whose device memory is all owned by its own pool, or one that runs
+ * where allocation is not allowed) and so has no buffer to pass as `logits`.
+ * The logits' partial sums go to a fixed 2 MiB array inside the library instead,
+ * one per GPU that loads the library, held until the process exits.  Limit:
+ * stq_router_ksplit(H) * T * E <= 524288 (e.g. T <= 256 for H = 6144, E = 256);
+ * larger requests return STQ_ERR_WORKSPACE before any launch.  The array's device
+ * address is looked up on the first call on each device (cudaGetSymbolAddress,
+ * with that device current): make that first call before any stream capture.
+ * Every call shares the array and leaves its last contents there (each call
+ * writes every entry it reads, so nothing needs clearing); calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race on it.  Allocates
+ * nothing.  Outputs: topk_ids int32 [T, k], topk_w f32 [T, k]. */
+stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router,
+                                  int32_t T, int32_t H, int32_t E, int32_t k,
+                                  int32_t* topk_ids, float* topk_w, stq_stream_t stream);
+
 typedef struct {
   int32_t fmt;              /* STQ_FMT_STQ1_0 or STQ_FMT_MXFP4 (routed experts) */
   const uint8_t* gate;      /* E matrices [I, H], expert-major, contiguous      */
