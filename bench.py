@@ -180,7 +180,9 @@ class W4A8Gemm(Workload):
 class MoeLayers(Workload):
     """MoE layers of hidden 6144, 256 experts of intermediate 2048, top-8."""
 
-    def __init__(self, S, dev, name, T, fmts, router, shared, residual):
+    def __init__(self, S, dev, name, T, fmts, router, shared, residual, experts=E):
+        global E
+        E = experts
         self.S, self.dev, self.name, self.T = S, dev, name, T
         self.fmts, self.router, self.shared, self.residual = fmts, router, shared, residual
         self.layers = [self._layer(l, f) for l, f in enumerate(fmts)]
@@ -267,7 +269,7 @@ class MoeLayers(Workload):
         tot, kinds = 0, {}
         for L, t in zip(self.layers, n):
             mat = STQ_MAT if L["fmt"] == "stq" else MX_MAT
-            by = t * 3 * mat + (3 * BF16_MAT if self.shared else 0) + (ROUTER_BYTES if self.router else 0) + 2 * T * H * 2
+            by = t * 3 * mat + (3 * BF16_MAT if self.shared else 0) + (E * H * 2 if self.router else 0) + 2 * T * H * 2
             tot += by
             if L["fmt"] == "stq":
                 gu = t * 2 * STQ_MAT + (2 * BF16_MAT if self.shared else 0) + T * H * 2 + (P + T) * I * 2
@@ -285,16 +287,19 @@ class MoeLayers(Workload):
                                                       for k, v in kinds.items()})
 
 
-def make_workload(name, S, dev):
+def make_workload(name, S, dev, experts=256):
     if name == "stq_matvec":
         return StqMatvec(S, dev)
     if name == "w4a8_gemm":
         return W4A8Gemm(S, dev)
+    if name == "decode_mx":
+        # one MXFP4 layer of the stacked workload (a small case for profiler captures)
+        return MoeLayers(S, dev, name, 32, ("mx",), True, True, True, experts)
     wl = W.WORKLOADS[name]
-    return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual)
+    return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual, experts)
 
 
-WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "stacked_decode"]
+WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "stacked_decode", "decode_mx"]
 
 
 # ----------------------------------------------------------------------------- measurement
@@ -387,7 +392,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     import bit_quantized_moe_stq1_b200 as S
 
-    wl = make_workload(args.workload, S, dev)
+    wl = make_workload(args.workload, S, dev, args.experts)
     for i in range(args.warmup):          # eager warm-up (one-time attribute setup)
         wl.step(i)
     torch.cuda.synchronize()
@@ -436,7 +441,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16 activations x STQ1_0 (ternary, fp16 scale) and MXFP4 x MXFP8 weights, fp32 accumulate",
         "data": "synthetic (seeded generators; random weights on the format grids)",
-        "config": {"workload": wl.name, "tokens_per_step": tps, "hbm_bytes_per_step": ab,
+        "config": {"workload": wl.name, "experts": E, "tokens_per_step": tps, "hbm_bytes_per_step": ab,
                    "tflop_per_step": acct[0]["flops"] / 1e12,
                    "l2": "inputs larger than L2: per-step weights exceed L2, batches rotate over 8",
                    "parallelism": f"replicas x{n}", "timing": "CUDA graph replays, CUDA events"},
@@ -551,7 +556,7 @@ def run_reference(args):
     dev = torch.device("cuda", 0)
     import bit_quantized_moe_stq1_b200 as S
 
-    wl = make_workload(args.workload, S, dev)
+    wl = make_workload(args.workload, S, dev, args.experts)
     vals = []
     for i in range(args.warmup + args.steps):
         cb = cpu_baseline(wl, dev, budget_s=0.0)   # one bounded unit per step
@@ -575,6 +580,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--experts", type=int, default=256,
+                    help="routed experts per layer (256 = the workloads; fewer only for small profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
