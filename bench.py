@@ -237,6 +237,8 @@ class MoeLayers(Workload):
             else:
                 ids, tw = self.routing[i % N_BATCHES]
             S.moe_expert_forward(self.desc, cur, ids, tw, L["w"], out, self.ws)
+            if self.residual:
+                S.rmsnorm_bf16(out, W.STACK_RMS_EPS, y=out)
             cur = out
         return cur
 
@@ -254,6 +256,8 @@ class MoeLayers(Workload):
             out.append(int(torch.unique(ids).numel()))
             nxt = self.bufs[(l + 1) % 2]
             S.moe_expert_forward(self.desc, cur, ids, tw, L["w"], nxt, self.ws)
+            if self.residual:
+                S.rmsnorm_bf16(nxt, W.STACK_RMS_EPS, y=nxt)
             cur = nxt
         torch.cuda.synchronize()
         return out
@@ -442,6 +446,7 @@ def run_ours(args):
         "dtype": "bf16 activations x STQ1_0 (ternary, fp16 scale) and MXFP4 x MXFP8 weights, fp32 accumulate",
         "data": "synthetic (seeded generators; random weights on the format grids)",
         "config": {"workload": wl.name, "experts": E, "tokens_per_step": tps, "hbm_bytes_per_step": ab,
+                   "touched_experts_per_layer": getattr(wl, "_acct", {}).get((args.warmup) % N_BATCHES),
                    "tflop_per_step": acct[0]["flops"] / 1e12,
                    "l2": "inputs larger than L2: per-step weights exceed L2, batches rotate over 8",
                    "parallelism": f"replicas x{n}", "timing": "CUDA graph replays, CUDA events"},
@@ -519,6 +524,8 @@ def _oracle_units(wl, dev):
         t0 = time.perf_counter()
         if shared is not None:
             M.expert_ffn_bf16h(shared[0], shared[1], shared[2], X)
+        if wl.residual:
+            M.rms_norm(X, W.STACK_RMS_EPS)
         t_s = time.perf_counter() - t0
         nl = sum(1 for L_ in wl.layers if L_["fmt"] == fmt)
         total += nl * (t_r + K_TOP * t_e + t_s)

@@ -60,11 +60,12 @@ SIGNATURES = {
                                   _vp, _vp, _sz, _vp]),
     "moe_get_device_error": (_i32, [_vp, _vp]),
     "stq_set_timing": (_i32, [_vp]),
+    "stq_rmsnorm_bf16": (_i32, [_vp, _i64, _i64, ctypes.c_float, _vp, _vp]),
 }
 
 
 KERNEL_KINDS = ["router_logits", "router_topk", "permute", "quant_x", "gate_up", "down", "combine", "gemv", "gemm",
-                "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down"]
+                "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down", "rmsnorm"]
 
 
 class StqTiming(ctypes.Structure):
@@ -198,6 +199,17 @@ def mxfp8_quantize_bf16(x, codes=None, scales=None, stream=None):
     _check(lib.mxfp8_quantize_bf16(_ptr(x), rows, K, _ptr(codes), _ptr(scales), _stream(stream)),
            "mxfp8_quantize_bf16")
     return codes, scales
+
+
+def rmsnorm_bf16(x, eps=1e-6, y=None, stream=None):
+    """bf16 [T, H] -> bf16 [T, H]: each row times 1/sqrt(mean(row^2) + eps); y may be x."""
+    _dev(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.is_contiguous()
+    if y is None:
+        y = torch.empty_like(x)
+    _check(lib.stq_rmsnorm_bf16(_ptr(x), x.shape[0], x.shape[1], float(eps), _ptr(y), _stream(stream)),
+           "stq_rmsnorm_bf16")
+    return y
 
 
 def read_error(err, stream=None):

@@ -29,40 +29,42 @@ constexpr int kKT = 128;                          // k per stage
 constexpr int kATile = 128 * 128;                 // smem bytes of one 128 x 128 E2M1 tile (expanded)
 constexpr uint32_t kATx = 128 * 128 / 2;          // bytes the TMA delivers for it
 constexpr int kSf = 512;                          // one scale-factor atom: 128 rows x 4 k-blocks
-constexpr int kSmemBudget = 200 * 1024;
+// Decode-size tiles (N <= 32) use half the shared memory so two CTAs share an SM and one
+// CTA's prologue and epilogue overlap the other's main loop.
+constexpr int smem_budget(int nt) { return nt <= 32 ? 100 * 1024 : 200 * 1024; }
 
-template <int NT, bool DUAL>
+// PAIR = the gate/up pair of one expert: the 128-row A tile holds 64 gate rows (TMEM
+// lanes 0-63) and the same 64 rows of the up projection (lanes 64-127), so one MMA per
+// k-block produces both and the epilogue pairs lane r with lane r + 64.
+template <int NT, bool PAIR>
 struct Cfg {
-  static constexpr int kA2 = DUAL ? kATile : 0;
   static constexpr int kB = NT * 128;
   static constexpr int kOffA = 0;
-  static constexpr int kOffA2 = kATile;
-  static constexpr int kOffB = kATile + kA2;
+  static constexpr int kOffB = kATile;
   static constexpr int kOffSfa = kOffB + kB;
-  static constexpr int kOffSfa2 = kOffSfa + kSf;
-  static constexpr int kOffSfb = kOffSfa + (DUAL ? 2 : 1) * kSf;
+  static constexpr int kOffSfb = kOffSfa + kSf;
   static constexpr int kStageRaw = kOffSfb + kSf;
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kStagesRaw = kSmemBudget / kStage;
+  static constexpr int kCtasPerSm = NT <= 32 ? 2 : 1;
+  static constexpr int kUBuf = PAIR ? 64 * 17 * 4 : 0;   // up-projection staging (row pitch 17 words)
+  static constexpr int kStagesRaw = (smem_budget(NT) - 2048 - kUBuf) / kStage;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kSmem = kStages * kStage + 1024 /* barriers */ + 1024 /* alignment */;
-  static constexpr int kColAccU = NT;
-  static constexpr int kColSfa = DUAL ? 2 * NT : NT;
-  static constexpr int kColSfa2 = kColSfa + 4;
-  static constexpr int kColSfb = kColSfa + (DUAL ? 8 : 4);
-  static constexpr int kColsUsed = kColSfb + 4;
+  static constexpr int kSmem = kStages * kStage + kUBuf + 1024 /* barriers */ + 1024 /* alignment */;
+  static constexpr int kRowsPerTile = PAIR ? 64 : 128;   // output features per CTA
+  static constexpr int kColSfa = NT;
+  static constexpr int kColSfb = NT + 4;
+  static constexpr int kColsUsed = NT + 8;
   static constexpr uint32_t kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-  static constexpr uint32_t kTx = kATx * (DUAL ? 2 : 1) + uint32_t(kB);
+  static constexpr uint32_t kTx = kATx + uint32_t(kB);
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "tile N");
-  static_assert(kColsUsed <= 512, "TMEM budget");
 };
 
 struct GemmProblem {
   int R, K, Ptot;               // weight rows per expert, reduction length, activation rows
-  const uint8_t* sa;            // weight scales [E*R][K/32]
-  const uint8_t* sa2;           // second weight matrix's scales (gate/up pair)
+  const uint8_t* sa;            // weight scales [E*R][K/32] (gate scales for a pair)
+  const uint8_t* sa2;           // up-projection scales (gate/up pair)
   const uint8_t* sb;            // activation scales [Ptot][K/32]
   const int32_t* offsets;       // grouped: [E+1]; nullptr = one dense expert of dense_M tokens
   const int2* ntiles;           // grouped: (expert, first token) per N tile
@@ -85,6 +87,18 @@ __device__ __forceinline__ void load_sf(uint32_t (&v)[4], const uint8_t* src, in
     v[m1] = (kt < nk && r < nvalid && row0 + r < limit)
                 ? __ldg(reinterpret_cast<const uint32_t*>(src + size_t(row0 + r) * k32 + size_t(kt) * 4))
                 : 0u;
+  }
+}
+
+// Pair tile: slices m1 = 0, 1 are gate rows row0 + lane + 32*m1, slices 2, 3 the same
+// rows of the up projection.
+__device__ __forceinline__ void load_sf_pair(uint32_t (&v)[4], const uint8_t* gsrc, const uint8_t* usrc, int row0,
+                                             int k32, int kt, int nk, int lane) {
+#pragma unroll
+  for (int m1 = 0; m1 < 4; ++m1) {
+    const uint8_t* src = m1 < 2 ? gsrc : usrc;
+    const int r = row0 + lane + 32 * (m1 & 1);
+    v[m1] = kt < nk ? __ldg(reinterpret_cast<const uint32_t*>(src + size_t(r) * k32 + size_t(kt) * 4)) : 0u;
   }
 }
 
@@ -115,20 +129,21 @@ __device__ __forceinline__ int mxfp8_exponent(float amax) {
   return min(max(k + 127, 0), 254);
 }
 
-template <int NT, bool DUAL>
-__global__ void __launch_bounds__(192, 1)
+template <int NT, bool PAIR>
+__global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, GemmProblem p) {
-  using C = Cfg<NT, DUAL>;
+  using C = Cfg<NT, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
+  float* ubuf = reinterpret_cast<float*>(smem + C::kStages * C::kStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage + C::kUBuf);
   uint64_t* empty = full + C::kStages;
   uint64_t* accum = empty + C::kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int MT = p.R / 128;
+  const int MT = p.R / C::kRowsPerTile;
   const int item = blockIdx.x;
   const int mt = item % MT;
   int e, n0, pos0, cnt;
@@ -148,7 +163,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   const int nk = p.K / kKT;
   const int k32 = p.K / 32;
-  const int arow = e * p.R + mt * 128;
+  const int arow = e * p.R + mt * C::kRowsPerTile;  // first A row (both matrices for a pair)
   const int brow = pos0 + n0;
 
   if (threadIdx.x == 0) {
@@ -159,7 +174,7 @@ __global__ void __launch_bounds__(192, 1)
     tc::mbar_init(accum, 1);
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&tmA);
-    if (DUAL) tc::prefetch_tensormap(&tmA2);
+    if (PAIR) tc::prefetch_tensormap(&tmA2);
     tc::prefetch_tensormap(&tmB);
   }
   if (warp == 1) tc::tmem_alloc(tmem_holder, C::kCols);
@@ -176,11 +191,11 @@ __global__ void __launch_bounds__(192, 1)
     int last_round[C::kStages];
 #pragma unroll
     for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;
-    uint32_t ra[kPf][4], ra2[kPf][4], rb[kPf][4];
+    uint32_t ra[kPf][4], rb[kPf][4];
 #pragma unroll
     for (int d = 0; d < kPf; ++d) {
-      load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, d, nk, lane);
-      if (DUAL) load_sf(ra2[d], p.sa2, arow, 128, 0x7fffffff, k32, d, nk, lane);
+      if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, arow, k32, d, nk, lane);
+      else load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, d, nk, lane);
       load_sf(rb[d], p.sb, brow, NT, p.Ptot, k32, d, nk, lane);
     }
     bool ok = true;
@@ -196,19 +211,22 @@ __global__ void __launch_bounds__(192, 1)
         }
         uint8_t* st = smem + s * C::kStage;
         store_sf(st + C::kOffSfa, ra[d], lane);
-        if (DUAL) store_sf(st + C::kOffSfa2, ra2[d], lane);
         store_sf(st + C::kOffSfb, rb[d], lane);
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           tc::mbar_arrive_expect_tx(&full[s], C::kTx);
-          tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);
-          if (DUAL) tc::tma_load_2d(st + C::kOffA2, &tmA2, kt * kKT, arow, &full[s]);
+          if (PAIR) {
+            tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);              // gate rows -> lanes 0-63
+            tc::tma_load_2d(st + C::kOffA + kATile / 2, &tmA2, kt * kKT, arow, &full[s]);  // up rows -> lanes 64-127
+          } else {
+            tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);
+          }
           tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, brow, &full[s]);
         }
         last_round[s] = r;
-        load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
-        if (DUAL) load_sf(ra2[d], p.sa2, arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
+        if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, arow, k32, kt + kPf, nk, lane);
+        else load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
         load_sf(rb[d], p.sb, brow, NT, p.Ptot, k32, kt + kPf, nk, lane);
       }
     }
@@ -225,21 +243,15 @@ __global__ void __launch_bounds__(192, 1)
         tc::fence_after_sync();
         uint8_t* st = smem + s * C::kStage;
         tc::cp_sf_32x128b_x4(tmem + C::kColSfa, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa)));
-        if (DUAL) tc::cp_sf_32x128b_x4(tmem + C::kColSfa2, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa2)));
         tc::cp_sf_32x128b_x4(tmem + C::kColSfb, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfb)));
         const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA));
-        const uint64_t da2 = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA2));
         const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffB));
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           const uint32_t idesc = tc::idesc_mxf8f6f4(NT, uint32_t(kb), uint32_t(kb));
           const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-          const uint32_t sfb = (tmem + C::kColSfb) | (uint32_t(kb) << 30);
-          tc::mma_mxf8f6f4(tmem, da + 2 * kb, db + 2 * kb, idesc, (tmem + C::kColSfa) | (uint32_t(kb) << 30), sfb,
-                           acc);
-          if (DUAL)
-            tc::mma_mxf8f6f4(tmem + C::kColAccU, da2 + 2 * kb, db + 2 * kb, idesc,
-                             (tmem + C::kColSfa2) | (uint32_t(kb) << 30), sfb, acc);
+          tc::mma_mxf8f6f4(tmem, da + 2 * kb, db + 2 * kb, idesc, (tmem + C::kColSfa) | (uint32_t(kb) << 30),
+                           (tmem + C::kColSfb) | (uint32_t(kb) << 30), acc);
         }
         tc::commit(&empty[s]);
       }
@@ -248,43 +260,62 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;
-    const bool ok = tc::mbar_wait(accum, 0, p.err);
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    bool ok = tc::mbar_wait(accum, 0, p.err);
+    if constexpr (PAIR) {
+      // the four epilogue warps meet at named barriers below, so they agree on ok first
+      uint32_t all;
+      asm volatile(
+          "{\n .reg .pred p, r;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred r, 1, 128, p;\n"
+          " selp.u32 %0, 1, 0, r;\n}"
+          : "=r"(all)
+          : "r"(ok ? 1u : 0u)
+          : "memory");
+      ok = all != 0u;
+    }
     tc::fence_after_sync();
-    const int f = mt * 128 + 32 * q + lane;  // weight row = output feature
     const uint32_t tl = tmem + (uint32_t(32 * q) << 16);
     if (ok) {
       for (int c0 = 0; c0 < NT; c0 += 16) {
         if (n0 + c0 >= cnt) break;
-        uint32_t g[16];
-        tc::tmem_ld_x16(tl + c0, g);
-        if constexpr (DUAL) {
-          uint32_t u[16];
-          tc::tmem_ld_x16(tl + C::kColAccU + c0, u);
-          tc::tmem_ld_wait();
+        uint32_t v[16];
+        tc::tmem_ld_x16(tl + c0, v);
+        tc::tmem_ld_wait();
+        if constexpr (PAIR) {
+          // lanes 64-127 (up) hand their values to lanes 0-63 (gate) through shared memory
+          if (q >= 2) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int col = n0 + c0 + j;
-            if (col >= cnt) break;
-            const float h = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
-            const bool bad = !isfinite(h);
-            float a = bad ? 0.f : fabsf(h);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            const bool anybad = __any_sync(0xffffffffu, bad);
-            const int ex = anybad ? 255 : mxfp8_exponent(a);
-            const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2f(127 - ex));
-            const size_t pos = size_t(pos0 + col);
-            p.hq[pos * p.R + f] = uint8_t(code);
-            if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
+            for (int j = 0; j < 16; ++j) ubuf[((q - 2) * 32 + lane) * 17 + j] = __uint_as_float(v[j]);
           }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (q < 2) {
+            const int f = mt * 64 + 32 * q + lane;  // output feature of this lane
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int col = n0 + c0 + j;
+              if (col >= cnt) break;
+              const float u = ubuf[(q * 32 + lane) * 17 + j];
+              const float h = silu_f32(__uint_as_float(v[j])) * u;
+              const bool bad = !isfinite(h);
+              float a = bad ? 0.f : fabsf(h);
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+              const bool anybad = __any_sync(0xffffffffu, bad);
+              const int ex = anybad ? 255 : mxfp8_exponent(a);
+              const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2f(127 - ex));
+              const size_t pos = size_t(pos0 + col);
+              p.hq[pos * p.R + f] = uint8_t(code);
+              if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
+            }
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
         } else {
-          tc::tmem_ld_wait();
+          const int f = mt * 128 + 32 * q + lane;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int col = n0 + c0 + j;
             if (col >= cnt) break;
-            p.Y[size_t(pos0 + col) * p.R + f] = __uint_as_float(g[j]);
+            p.Y[size_t(pos0 + col) * p.R + f] = __uint_as_float(v[j]);
           }
         }
       }
@@ -345,13 +376,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// E2M1 weights [rows][K] (two per byte), box 128 x 128, expanded to 16 bytes per 16 elements.
-bool map_e2m1(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows) {
+// E2M1 weights [rows][K] (two per byte), box 128 x box_rows, expanded to 16 bytes per 16 elements.
+bool map_e2m1(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {K, rows};
   const cuuint64_t strides[1] = {K / 2};
-  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -371,30 +402,30 @@ bool map_u8(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT, bool DUAL>
+template <int NT, bool PAIR>
 stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
                        unsigned grid, cudaStream_t s) {
-  using C = Cfg<NT, DUAL>;
+  using C = Cfg<NT, PAIR>;
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(w4a8_gemm_kernel<NT, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<NT, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
         cudaSuccess)
       return STQ_ERR_CUDA;
     configured = true;
   }
   if (grid == 0) return STQ_OK;
-  w4a8_gemm_kernel<NT, DUAL><<<grid, 192, C::kSmem, s>>>(a, a2, b, p);
+  w4a8_gemm_kernel<NT, PAIR><<<grid, 192, C::kSmem, s>>>(a, a2, b, p);
   return stq_launch_status();
 }
 
-template <bool DUAL>
+template <bool PAIR>
 stq_status launch_nt(int nt, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
                      unsigned grid, cudaStream_t s) {
   switch (nt) {
-    case 16: return launch_gemm<16, DUAL>(a, a2, b, p, grid, s);
-    case 32: return launch_gemm<32, DUAL>(a, a2, b, p, grid, s);
-    case 64: return launch_gemm<64, DUAL>(a, a2, b, p, grid, s);
-    default: return launch_gemm<128, DUAL>(a, a2, b, p, grid, s);
+    case 16: return launch_gemm<16, PAIR>(a, a2, b, p, grid, s);
+    case 32: return launch_gemm<32, PAIR>(a, a2, b, p, grid, s);
+    case 64: return launch_gemm<64, PAIR>(a, a2, b, p, grid, s);
+    default: return launch_gemm<128, PAIR>(a, a2, b, p, grid, s);
   }
 }
 
@@ -423,8 +454,8 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   const int max_tiles = P / nt + (a.E < P ? a.E : P);
   // 3. gate/up pair with SwiGLU and MXFP8 h
   CUtensorMap mg, mu, mx, md, mh;
-  if (!map_e2m1(&mg, a.wg, uint64_t(a.H), uint64_t(a.E) * a.I) ||
-      !map_e2m1(&mu, a.wu, uint64_t(a.H), uint64_t(a.E) * a.I) || !map_u8(&mx, a.xq, a.H, P, nt) ||
+  if (!map_e2m1(&mg, a.wg, uint64_t(a.H), uint64_t(a.E) * a.I, 64) ||
+      !map_e2m1(&mu, a.wu, uint64_t(a.H), uint64_t(a.E) * a.I, 64) || !map_u8(&mx, a.xq, a.H, P, nt) ||
       !map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !map_u8(&mh, a.hq, a.I, P, nt))
     return STQ_ERR_CUDA;
   GemmProblem gp{};
@@ -442,7 +473,7 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   gp.err = a.err;
   {
     StqTimed tm(STQ_K_GATE_UP_MX, s);
-    st = launch_nt<true>(nt, mg, mu, mx, gp, unsigned(max_tiles * (a.I / 128)), s);
+    st = launch_nt<true>(nt, mg, mu, mx, gp, unsigned(max_tiles * (a.I / 64)), s);
   }
   if (st != STQ_OK) return st;
   if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;

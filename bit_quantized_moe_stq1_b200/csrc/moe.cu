@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __rest
   __shared__ int total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += 1024) cnt[e] = 0;
+  if (ws.sched != nullptr && tid < 4) ws.sched[tid] = 0;
   __syncthreads();
   bool bad = false;
   for (int p = tid; p < P; p += 1024) {
@@ -138,14 +139,14 @@ __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
 
 // Router logits, split over K: part[ks][t][e] = sum over the ks-th slice of H of
 // x[t, h] wr[e, h] (bf16 mma.sync, FP32 accumulate).  CTA = 16 experts x one K slice;
-// its four warps split the slice and are summed in a fixed order.
-__global__ void __launch_bounds__(128) router_logits_kernel(const uint16_t* __restrict__ x,
+// its eight warps split the slice and are summed in a fixed order.
+__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const uint16_t* __restrict__ wr, int T, int H, int E,
                                                             int KS, float* __restrict__ part) {
-  __shared__ float red[4][4][4][32];
+  __shared__ float red[8][4][4][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int e0 = (blockIdx.x / KS) * 16, ks = blockIdx.x % KS;
-  const int slice = H / KS, kq = slice / 4;
+  const int slice = H / KS, kq = slice / 8;
   const int k0 = ks * slice + warp * kq, k1 = k0 + kq;
   const int er = min(e0 + g, E - 1);                // rows past E read a valid row; results dropped
   const uint16_t* rowg[1] = {wr + size_t(er) * H};
@@ -187,7 +188,9 @@ __global__ void __launch_bounds__(128) router_logits_kernel(const uint16_t* __re
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float v = ((red[0][c][j][lane] + red[1][c][j][lane]) + red[2][c][j][lane]) + red[3][c][j][lane];
+          float v = red[0][c][j][lane];
+#pragma unroll
+          for (int w = 1; w < 8; ++w) v += red[w][c][j][lane];
           const int tok = t0 + 8 * c + 2 * t + (j & 1);
           const int e = e0 + g + 8 * (j >> 1);
           if (tok < T && e < E) part[(size_t(ks) * T + tok) * E + e] = v;
@@ -205,25 +208,47 @@ __global__ void router_topk_kernel(float* __restrict__ logits, int T, int E, int
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   constexpr int kMaxPer = 32;  // E <= 1024
+  constexpr int kMaxKs = 8;
   float p[kMaxPer];
   const int per = (E + 31) / 32;
   float m = -INFINITY;
+  // Logits = sum of the KS partial slices, in slice order; all loads of a chunk of 8
+  // experts are issued before any add.
 #pragma unroll
-  for (int j = 0; j < kMaxPer; ++j) {
-    const int e = lane + 32 * j;
-    float v = -INFINITY;
-    if (j < per && e < E) {
-      v = logits[size_t(t) * E + e];
-      for (int ks = 1; ks < KS; ++ks) v += logits[(size_t(ks) * T + t) * E + e];
-      logits[size_t(t) * E + e] = v;
+  for (int j0 = 0; j0 < kMaxPer; j0 += 8) {
+    if (j0 >= per) break;
+    float part[kMaxKs][8];
+#pragma unroll
+    for (int ks = 0; ks < kMaxKs; ++ks)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int e = lane + 32 * (j0 + jj);
+        part[ks][jj] = (ks < KS && j0 + jj < per && e < E) ? logits[(size_t(ks) * T + t) * E + e] : 0.f;
+      }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int e = lane + 32 * (j0 + jj);
+      float v = part[0][jj];
+#pragma unroll
+      for (int ks = 1; ks < kMaxKs; ++ks) v += part[ks][jj];
+      const bool valid = j0 + jj < per && e < E;
+      if (valid) logits[size_t(t) * E + e] = v;
+      p[j0 + jj] = valid ? v : -INFINITY;
+      m = fmaxf(m, p[j0 + jj]);
     }
-    p[j] = v;
-    m = fmaxf(m, p[j]);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  for (int j = 0; j < kMaxPer; ++j)
+    if (j >= ((per + 7) / 8) * 8) p[j] = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < kMaxPer; ++j) p[j] = (p[j] == -INFINITY) ? -1.f : expf(p[j] - m);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  // Padding lanes get -1 (never chosen); a non-finite logit (or an infinite maximum)
+  // counts as probability 0, so a valid expert id is chosen in every round.
+#pragma unroll
+  for (int j = 0; j < kMaxPer; ++j) {
+    const float pv = expf(p[j] - m);
+    p[j] = (p[j] == -INFINITY && !(j < per && lane + 32 * j < E)) ? -1.f : (pv >= 0.f ? pv : 0.f);
+  }
   float sel_sum = 0.f;
   for (int r = 0; r < k; ++r) {
     float bp = -1.f;
@@ -239,7 +264,7 @@ __global__ void router_topk_kernel(float* __restrict__ logits, int T, int E, int
       const int oid = __shfl_xor_sync(kFull, bid, o);
       if (op > bp || (op == bp && oid < bid)) { bp = op; bid = oid; }
     }
-    if ((bid & 31) == lane) p[bid >> 5] = -1.f;  // remove the chosen expert
+    if (bid >= 0 && bid < E && (bid & 31) == lane) p[bid >> 5] = -1.f;  // remove the chosen expert
     sel_sum += bp;
     if (lane == 0) {
       ids[size_t(t) * k + r] = bid;
@@ -247,7 +272,7 @@ __global__ void router_topk_kernel(float* __restrict__ logits, int T, int E, int
     }
   }
   __syncwarp();
-  if (lane < k) w[size_t(t) * k + lane] = w[size_t(t) * k + lane] / sel_sum;
+  if (lane < k) w[size_t(t) * k + lane] = sel_sum > 0.f ? w[size_t(t) * k + lane] / sel_sum : 1.f / float(k);
 }
 
 // ----------------------------------------------------------------------------- expert GEMVs
@@ -325,83 +350,102 @@ __device__ __forceinline__ void shared_down(const MoeArgs& a, int bid, float (*r
   }
 }
 
-// Routed STQ1_0 gate/up + SwiGLU.  CTA = 128 features of one touched expert; warp =
-// 32 features = 2 gate tiles + 2 up tiles over all of H.
-__global__ void __launch_bounds__(128) moe_gateup_stq_kernel(MoeArgs a) {
+// Next work item of a persistent CTA (one atomic per item, broadcast through smem).
+__device__ __forceinline__ int next_item(int32_t* counter, int* slot) {
+  if (threadIdx.x == 0) *slot = atomicAdd(counter, 1);
+  __syncthreads();
+  const int item = *slot;
+  __syncthreads();
+  return item;
+}
+
+// Routed STQ1_0 gate/up + SwiGLU, persistent.  Items: first the shared expert's
+// 16-feature tiles (BF16, K split over the four warps), then, per touched expert,
+// 128-feature tiles (warp = 32 features = 2 gate tiles + 2 up tiles over all of H).
+__global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
   __shared__ float red[4][2][4][4][32];
-  int bid = blockIdx.x;
-  if (bid < a.n_shared_cta) {
-    shared_gateup(a, bid, red);
-    return;
-  }
-  bid -= a.n_shared_cta;
+  __shared__ int s_item;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int per_expert = a.I / 128;
-  const int slot = bid / per_expert, ct = bid % per_expert;
-  if (slot >= *a.ntouched) return;
-  const int e = a.tlist[slot];
-  const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+  const int n_items = a.n_shared_cta + (a.routed ? *a.ntouched * per_expert : 0);
   const int nb = a.H / 256;
   const size_t mat = size_t(a.I) * nb * 42;
-  const int f0 = ct * 128 + warp * 32;
-  const uint8_t* gb = a.wg + size_t(e) * mat;
-  const uint8_t* ub = a.wu + size_t(e) * mat;
   const size_t tstride = size_t(nb) * kTileBlockBytes;
-  const uint8_t* tb[4] = {gb + size_t(f0 / 16) * tstride, gb + size_t(f0 / 16 + 1) * tstride,
-                          ub + size_t(f0 / 16) * tstride, ub + size_t(f0 / 16 + 1) * tstride};
   const uint32_t lut = lut_entry(lane);
-  for (int c0 = 0; c0 < cnt; c0 += 8) {
-    const int j = c0 + g;
-    const uint16_t* xrow = j < cnt ? a.x + size_t(a.perm[pos0 + j] / a.k) * a.H : nullptr;
-    float acc[4][4] = {};
-    stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
+  for (;;) {
+    const int item = next_item(a.sched, &s_item);
+    if (item >= n_items) break;
+    if (item < a.n_shared_cta) {
+      shared_gateup(a, item, red);
+      continue;
+    }
+    const int bid = item - a.n_shared_cta;
+    const int slot = bid / per_expert, ct = bid % per_expert;
+    const int e = a.tlist[slot];
+    const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+    const int f0 = ct * 128 + warp * 32;
+    const uint8_t* gb = a.wg + size_t(e) * mat;
+    const uint8_t* ub = a.wu + size_t(e) * mat;
+    const uint8_t* tb[4] = {gb + size_t(f0 / 16) * tstride, gb + size_t(f0 / 16 + 1) * tstride,
+                            ub + size_t(f0 / 16) * tstride, ub + size_t(f0 / 16 + 1) * tstride};
+    for (int c0 = 0; c0 < cnt; c0 += 8) {
+      const int j = c0 + g;
+      const uint16_t* xrow = j < cnt ? a.x + size_t(a.perm[pos0 + j] / a.k) * a.H : nullptr;
+      float acc[4][4] = {};
+      stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
 #pragma unroll
-    for (int tp = 0; tp < 2; ++tp)
+      for (int tp = 0; tp < 2; ++tp)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int col = c0 + 2 * t + (q & 1);
-        const int f = f0 + 16 * tp + g + 8 * (q >> 1);
-        if (col < cnt) a.h[size_t(pos0 + col) * a.I + f] = float_to_bf16_bits(silu_f32(acc[tp][q]) * acc[tp + 2][q]);
-      }
+        for (int q = 0; q < 4; ++q) {
+          const int col = c0 + 2 * t + (q & 1);
+          const int f = f0 + 16 * tp + g + 8 * (q >> 1);
+          if (col < cnt) a.h[size_t(pos0 + col) * a.I + f] = float_to_bf16_bits(silu_f32(acc[tp][q]) * acc[tp + 2][q]);
+        }
+    }
   }
 }
 
-// Routed STQ1_0 down.  CTA = 256 rows of H of one touched expert; warp = 4 tiles.
-__global__ void __launch_bounds__(128) moe_down_stq_kernel(MoeArgs a) {
+// Routed STQ1_0 down, persistent.  Items: the shared expert's 16-row tiles, then per
+// touched expert 256-row tiles of H (warp = 4 tiles).
+__global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
   __shared__ float red[4][2][4][4][32];
-  int bid = blockIdx.x;
-  if (bid < a.n_shared_cta) {
-    shared_down(a, bid, red);
-    return;
-  }
-  bid -= a.n_shared_cta;
+  __shared__ int s_item;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int per_expert = a.H / 256;
-  const int slot = bid / per_expert, ct = bid % per_expert;
-  if (slot >= *a.ntouched) return;
-  const int e = a.tlist[slot];
-  const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+  const int n_items = a.n_shared_cta + (a.routed ? *a.ntouched * per_expert : 0);
   const int nb = a.I / 256;
   const size_t mat = size_t(a.H) * nb * 42;
-  const int r0 = ct * 256 + warp * 64;
-  const uint8_t* db = a.wd + size_t(e) * mat;
   const size_t tstride = size_t(nb) * kTileBlockBytes;
-  const uint8_t* tb[4] = {db + size_t(r0 / 16) * tstride, db + size_t(r0 / 16 + 1) * tstride,
-                          db + size_t(r0 / 16 + 2) * tstride, db + size_t(r0 / 16 + 3) * tstride};
   const uint32_t lut = lut_entry(lane);
-  for (int c0 = 0; c0 < cnt; c0 += 8) {
-    const int j = c0 + g;
-    const uint16_t* xrow = j < cnt ? a.h + size_t(pos0 + j) * a.I : nullptr;
-    float acc[4][4] = {};
-    stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
+  for (;;) {
+    const int item = next_item(a.sched, &s_item);
+    if (item >= n_items) break;
+    if (item < a.n_shared_cta) {
+      shared_down(a, item, red);
+      continue;
+    }
+    const int bid = item - a.n_shared_cta;
+    const int slot = bid / per_expert, ct = bid % per_expert;
+    const int e = a.tlist[slot];
+    const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+    const int r0 = ct * 256 + warp * 64;
+    const uint8_t* db = a.wd + size_t(e) * mat;
+    const uint8_t* tb[4] = {db + size_t(r0 / 16) * tstride, db + size_t(r0 / 16 + 1) * tstride,
+                            db + size_t(r0 / 16 + 2) * tstride, db + size_t(r0 / 16 + 3) * tstride};
+    for (int c0 = 0; c0 < cnt; c0 += 8) {
+      const int j = c0 + g;
+      const uint16_t* xrow = j < cnt ? a.h + size_t(pos0 + j) * a.I : nullptr;
+      float acc[4][4] = {};
+      stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int col = c0 + 2 * t + (q & 1);
-        const int r = r0 + 16 * i + g + 8 * (q >> 1);
-        if (col < cnt) a.Y[size_t(pos0 + col) * a.H + r] = acc[i][q];
-      }
+        for (int q = 0; q < 4; ++q) {
+          const int col = c0 + 2 * t + (q & 1);
+          const int r = r0 + 16 * i + g + 8 * (q >> 1);
+          if (col < cnt) a.Y[size_t(pos0 + col) * a.H + r] = acc[i][q];
+        }
+    }
   }
 }
 
@@ -449,6 +493,19 @@ __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __re
 
 // ----------------------------------------------------------------------------- host side
 
+// CTAs of a persistent GEMV launch: four per SM (the register-limited occupancy), never
+// more than the work items.
+int stq_persistent_grid(int items) {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  const int cap = 4 * sms;
+  return items < 1 ? 1 : (items < cap ? items : cap);
+}
+
 MoeWsLayout moe_ws_layout(const moe_desc& d) {
   MoeWsLayout L{};
   const size_t T = size_t(d.T), H = size_t(d.H), I = size_t(d.I), E = size_t(d.E), P = T * size_t(d.k);
@@ -469,6 +526,7 @@ MoeWsLayout moe_ws_layout(const moe_desc& d) {
   L.hs = take(P * (I / 32));
   L.ntiles = take((P / 16 + E + 1) * 8);
   L.n_ntiles = take(4);
+  L.sched = take(16);
   L.total = o;
   return L;
 }
@@ -491,6 +549,7 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
   w.hs = b + L.hs;
   w.ntiles = reinterpret_cast<int2*>(b + L.ntiles);
   w.n_ntiles = reinterpret_cast<int32_t*>(b + L.n_ntiles);
+  w.sched = reinterpret_cast<int32_t*>(b + L.sched);
   return w;
 }
 
@@ -508,17 +567,20 @@ extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
 // STQ1_0 kernels.
 stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
   MoeArgs a = a0;
+  a.routed = 0;
   a.n_shared_cta = a.I / 16;
+  a.sched = a0.sched + 2;
   {
     StqTimed tm(STQ_K_SHARED_GATE_UP, s);
-    moe_gateup_stq_kernel<<<unsigned(a.n_shared_cta), 128, 0, s>>>(a);
+    moe_gateup_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta)), 128, 0, s>>>(a);
   }
   stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
   a.n_shared_cta = a.H / 16;
+  a.sched = a0.sched + 3;
   {
     StqTimed tm(STQ_K_SHARED_DOWN, s);
-    moe_down_stq_kernel<<<unsigned(a.n_shared_cta), 128, 0, s>>>(a);
+    moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta)), 128, 0, s>>>(a);
   }
   return stq_launch_status();
 }
@@ -602,20 +664,24 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   a.h = ws.h; a.Y = ws.Y;
   a.xq = ws.xq; a.xs = ws.xs; a.hq = ws.hq; a.hs = ws.hs;
   a.ntiles = ws.ntiles; a.n_ntiles = ws.n_ntiles;
+  a.sched = ws.sched;
   a.err = ws.err;
   const int slots = d->E < P ? d->E : P;
 
   if (w->fmt == STQ_FMT_STQ1_0) {
+    a.routed = 1;
     a.n_shared_cta = has_shared ? d->I / 16 : 0;
+    a.sched = ws.sched;
     {
       StqTimed tm(STQ_K_GATE_UP, s);
-      moe_gateup_stq_kernel<<<unsigned(a.n_shared_cta + slots * (d->I / 128)), 128, 0, s>>>(a);
+      moe_gateup_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->I / 128))), 128, 0, s>>>(a);
     }
     if ((st = stq_launch_status()) != STQ_OK) return st;
     a.n_shared_cta = has_shared ? d->H / 16 : 0;
+    a.sched = ws.sched + 1;
     {
       StqTimed tm(STQ_K_DOWN, s);
-      moe_down_stq_kernel<<<unsigned(a.n_shared_cta + slots * (d->H / 256)), 128, 0, s>>>(a);
+      moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->H / 256))), 128, 0, s>>>(a);
     }
     if ((st = stq_launch_status()) != STQ_OK) return st;
   } else {
@@ -627,7 +693,7 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
 
 extern "C" int32_t stq_router_ksplit(int32_t H) {
   for (int ks = 8; ks > 1; ks >>= 1)
-    if (H % (128 * ks) == 0) return ks;
+    if (H % (256 * ks) == 0) return ks;
   return 1;
 }
 
@@ -636,14 +702,14 @@ extern "C" stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_route
                                       stq_stream_t stream) {
   STQ_HOST_CHECK(x && w_router && logits && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
-  STQ_HOST_CHECK(H % 128 == 0, STQ_ERR_SHAPE);
+  STQ_HOST_CHECK(H % 256 == 0, STQ_ERR_SHAPE);
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
   if (T == 0) return STQ_OK;
   cudaStream_t s = stq_cuda_stream(stream);
   const int KS = stq_router_ksplit(H);
   {
     StqTimed tm(STQ_K_ROUTER_LOGITS, s);
-    router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 128, 0, s>>>(x, w_router, T, H, E, KS, logits);
+    router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 256, 0, s>>>(x, w_router, T, H, E, KS, logits);
   }
   stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
@@ -705,7 +771,7 @@ extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* 
                                              stq_stream_t stream) {
   STQ_HOST_CHECK(x && w_router && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
-  STQ_HOST_CHECK(H % 128 == 0, STQ_ERR_SHAPE);
+  STQ_HOST_CHECK(H % 256 == 0, STQ_ERR_SHAPE);
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
   const int KS = stq_router_ksplit(H);
   STQ_HOST_CHECK(size_t(KS) * size_t(T) * size_t(E) <= kRouterStaticFloats, STQ_ERR_WORKSPACE);
@@ -716,7 +782,7 @@ extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* 
   cudaStream_t s = stq_cuda_stream(stream);
   // Every entry the top-k step reads is written first by the logits step, so the
   // array needs no clearing between calls.
-  router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 128, 0, s>>>(x, w_router, T, H, E, KS, scratch);
+  router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 256, 0, s>>>(x, w_router, T, H, E, KS, scratch);
   stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
   router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(scratch, T, E, KS, k, topk_ids, topk_w);

@@ -4,7 +4,7 @@
 #include "common.cuh"
 
 struct MoeWsLayout {
-  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, ntiles, n_ntiles, total;
+  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, ntiles, n_ntiles, sched, total;
 };
 
 // Device pointers into the caller's workspace.
@@ -24,6 +24,7 @@ struct MoeWs {
   uint8_t* hs;   // [P, I/32]
   int2* ntiles;  // [P/16 + E] (expert, first token) of each GEMM N tile
   int32_t* n_ntiles;
+  int32_t* sched;  // [4] work counters of the persistent GEMV kernels (zeroed by the permute kernel)
 };
 
 // Kernel arguments (by value).
@@ -40,7 +41,9 @@ struct MoeArgs {
   int2* ntiles;
   int32_t* n_ntiles;
   int32_t* err;
-  int n_shared_cta;
+  int32_t* sched;   // work counter of this launch
+  int n_shared_cta; // work items of the shared expert (first)
+  int routed;       // 1: routed STQ1_0 items follow the shared ones
 };
 
 MoeWsLayout moe_ws_layout(const moe_desc& d);

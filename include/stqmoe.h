@@ -156,7 +156,9 @@ enum { STQ_FMT_STQ1_0 = 0, STQ_FMT_MXFP4 = 1 };
  * x bf16 [T, H], w_router bf16 [E, H] -> topk_ids int32 [T, k], topk_w f32 [T, k].
  * logits: caller-owned f32 scratch of stq_router_ksplit(H) * T * E floats (the
  * logits are summed over that many slices of H); on return its first T*E floats
- * hold the logits [T, E].  E <= 1024, k <= 32, k <= E, H % 128 == 0. */
+ * hold the logits [T, E].  A non-finite logit counts as probability 0 (a token whose
+ * chosen probabilities are all 0 gets weights 1/k).  E <= 1024, k <= 32, k <= E,
+ * H % 256 == 0. */
 int32_t stq_router_ksplit(int32_t H);
 stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T,
                            int32_t H, int32_t E, int32_t k, float* logits,
@@ -243,16 +245,35 @@ size_t moe_workspace_offset(const moe_desc* d, int32_t region);
 stq_status moe_get_device_error(void* workspace, stq_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
+/* Layer stacking                                                            */
+/* ------------------------------------------------------------------------- */
+
+/* RMS normalisation of bf16 rows with unit gain:
+ *   y[t, :] = bf16_RNE( x[t, :] * 1 / sqrt(mean_j x[t, j]^2 + eps) ).
+ * The pages' stacked decode ("Hy4-preview-FlashMoE-STQ1_0", "Package details":
+ * consecutive MoE layers with a residual add between them) names no normalisation;
+ * without one, eight layers of random SwiGLU experts grow the residual stream past
+ * the FP32 range.  This library's reading puts one RMS normalisation after each
+ * layer's residual add (the next layer's input is stq_rmsnorm_bf16 of the previous
+ * layer's output).  Sum of squares, mean, scale and product in FP64 (fixed
+ * summation order: deterministic), rounded to FP32 and then to bf16; x, y bf16 [T, H] row-major, device, 16-byte aligned, caller-owned;
+ * y == x (in place) allowed.  H % 8 == 0; T == 0 is a no-op; eps >= 0 finite.  A row
+ * with a non-finite element gives non-finite outputs.  One kernel launch. */
+stq_status stq_rmsnorm_bf16(const uint16_t* x, int64_t T, int64_t H, float eps,
+                            uint16_t* y, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
 /* Instrumentation (no counterpart on the pages).                             */
 /* ------------------------------------------------------------------------- */
 
 /* Kernel kinds reported by the timing hook. */
 enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM,
-       STQ_K_GATE_UP_MX, STQ_K_DOWN_MX, STQ_K_PLAN, STQ_K_SHARED_GATE_UP, STQ_K_SHARED_DOWN, STQ_K_COUNT };
+       STQ_K_GATE_UP_MX, STQ_K_DOWN_MX, STQ_K_PLAN, STQ_K_SHARED_GATE_UP, STQ_K_SHARED_DOWN,
+       STQ_K_RMSNORM, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
- * moe_router_topk, moe_expert_forward, stq1_gemv and w4a8_gemm is bracketed by
+ * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm and stq_rmsnorm_bf16 is bracketed by
  * event records of events[2n] / events[2n+1] on the call's stream (inside stream
  * capture as external event-record nodes of the graph), kinds[n] is set to its
  * STQ_K_* kind and n = count++ (until capacity pairs are used).  events:

@@ -6,7 +6,8 @@ Shapes ("Hy4-preview-FlashMoE-STQ1_0", "Package details"): hidden H = 6144,
 MoE intermediate I = 2048, E = 256 routed experts, k = 8 selected per token,
 one shared expert.  Steps, in order: router (softmax over the E logits, top-k,
 renormalised), token-to-expert grouping, per expert gate/up projections, SwiGLU,
-down projection, weighted top-k combine plus the shared expert.
+down projection, weighted top-k combine plus the shared expert; between stacked
+layers, an RMS normalisation of the residual stream (a reading, see rms_norm).
 
 Every matrix product is a float64 numpy matmul of decoded values (a library
 primitive); every reduction bound S = sum |w * x| is returned beside the result
@@ -164,3 +165,21 @@ def combine(Y_pairs, S_pairs, topk_w, shared=None, shared_S=None, residual=None)
         y = y + residual
         s = s + np.abs(residual)
     return y, s
+
+
+# ----------------------------------------------------------------------------
+# Between stacked layers
+# ----------------------------------------------------------------------------
+
+
+def rms_norm(x, eps):
+    """y[t, :] = x[t, :] / sqrt(mean_j x[t, j]^2 + eps), float64, unit gain.
+
+    The stacked decode of "Hy4-preview-FlashMoE-STQ1_0" ("Package details") chains
+    MoE layers with a residual add and names no normalisation; the reading used
+    here applies this normalisation to each layer's output (residual included)
+    before it becomes the next layer's input, which keeps eight random layers
+    finite.  Callers round the result to BF16 to compare with a BF16 output."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps)

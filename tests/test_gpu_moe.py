@@ -80,6 +80,21 @@ def test_router_topk(S, T, H, E, k):
         assert abs(w[t].sum() - 1.0) < 1e-5
 
 
+def test_router_nonfinite_inputs_give_valid_ids(S):
+    T, H, E, k = 4, 512, 64, 8
+    x = W.bf16_normal((T, H), 1.0, DEV, 0, "rnf")
+    x[1, 7] = float("nan")
+    x[2, 3] = float("inf")
+    x[3, :] = float("nan")
+    wr = W.bf16_normal((E, H), 0.02, DEV, 0, "rnfw")
+    ids, w, _ = S.moe_router_topk(x, wr, k)
+    ids, w = ids.cpu().numpy(), w.cpu().numpy()
+    assert ids.min() >= 0 and ids.max() < E
+    for t in range(T):
+        assert len(set(ids[t])) == k
+    assert np.all(np.isfinite(w)) and np.allclose(w.sum(1), 1.0, atol=1e-5)
+
+
 # --------------------------------------------------------------------------- STQ1_0 MoE layer
 
 

@@ -187,3 +187,27 @@ def test_expert_ffn_stage_consistency():
     h = F.bf16_decode(F.bf16_encode_rne(M.silu(g.astype(np.float32).astype(np.float64)) * u.astype(np.float32)))
     assert np.array_equal(out["h"], h)
     assert np.allclose(out["y"], h @ wd.astype(np.float64).T, rtol=1e-13, atol=1e-15)
+
+
+def test_rms_norm_closed_forms():
+    """Constant rows: a / sqrt(a^2 + eps) (eps = 3, a = 1 gives exactly 1/2; eps = 0
+    gives sign(a)); a 3-4 row: mean square 12.5, so y = (3, 4) / sqrt(12.5)."""
+    y = M.rms_norm(np.array([[1.0] * 8, [-2.5] * 8]), 3.0)
+    assert np.all(y[0] == 0.5) and np.allclose(y[1], -2.5 / np.sqrt(6.25 + 3.0), rtol=0, atol=1e-15)
+    assert np.all(M.rms_norm(np.full((1, 16), -7.0), 0.0) == -1.0)
+    y = M.rms_norm(np.array([[3.0, 4.0]]), 0.0)
+    assert abs(y[0, 0] - 0.848528137423857) < 1e-14 and abs(y[0, 1] - 1.131370849898476) < 1e-14
+
+
+def test_rms_norm_invariants():
+    """With eps = 0 every output row has mean square 1 and the map ignores a positive
+    scale of its row; rows are independent of one another."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 96)) * np.array([[1e-3], [1.0], [7.0], [1e4], [0.5], [3.0]])
+    y = M.rms_norm(x, 0.0)
+    assert np.allclose(np.mean(y * y, axis=1), 1.0, rtol=0, atol=1e-13)
+    assert np.allclose(M.rms_norm(x * 2.0 ** 11, 0.0), y, rtol=1e-15, atol=0)
+    assert np.array_equal(M.rms_norm(x[2:3], 0.0), y[2:3])
+    # eps only lowers the output: |y_eps| < |y_0| elementwise where x != 0
+    ye = M.rms_norm(x, 1e-2)
+    assert np.all(np.abs(ye) <= np.abs(y))

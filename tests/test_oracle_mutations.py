@@ -85,3 +85,18 @@ def test_unstable_permute_is_caught(monkeypatch):
 
     monkeypatch.setattr(M, "permute", unstable)
     _fails(TM.test_permute_matches_stable_sort_by_loops)
+
+
+@pytest.mark.parametrize("mistake", ["sum", "eps_outside", "no_sqrt"])
+def test_rms_norm_mistakes_are_caught(monkeypatch, mistake):
+    def wrong(x, eps):
+        x = np.asarray(x, np.float64)
+        if mistake == "sum":
+            return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+        ms = np.mean(x * x, axis=-1, keepdims=True)
+        if mistake == "eps_outside":
+            return x / (np.sqrt(ms) + eps)
+        return x / (ms + eps)
+
+    monkeypatch.setattr(M, "rms_norm", wrong)
+    _fails(TM.test_rms_norm_closed_forms)

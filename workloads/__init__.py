@@ -14,7 +14,8 @@ hidden 6144, MoE intermediate 2048, 256 routed experts, top-8, 1 shared expert):
 * ``decode_stq``   one MoE layer, STQ1_0 experts, 8 tokens, BF16 router, shared expert.
 * ``prefill_w4a8`` one MoE layer, MXFP4 experts, 4096 tokens, Zipf(1.1) routing.
 * ``stacked_decode`` 8 MoE layers (odd layers STQ1_0, even layers MXFP4), 32
-  tokens, fresh router per layer, residual add.
+  tokens, fresh router per layer, residual add, then an RMS normalisation
+  (unit gain, eps ``STACK_RMS_EPS``) of each layer's output before the next layer.
 """
 
 import hashlib
@@ -83,14 +84,18 @@ def stq_grid_weights(rows, K, device, seed, *tag):
     return (pat.view(rows, K // 256, 256) * d.unsqueeze(-1)).view(rows, K).contiguous()
 
 
-def mxfp4_random(rows, K, device, seed, *tag):
+def mxfp4_random(rows, K, device, seed, *tag, emin=118, emax=127):
     """MXFP4 weights as stored: codes uniform over the 16 E2M1 codes (uniform
     bytes, two codes per byte) and one UE8M0 exponent per 32 along K uniform in
-    [118, 127]."""
+    [emin, emax] (the single-expert and prefill workloads use [118, 127])."""
     g = generator(device, seed, *tag)
     codes = torch.randint(0, 256, (rows, K // 2), generator=g, device=device, dtype=torch.int32).to(torch.uint8)
-    scales = torch.randint(118, 128, (rows, K // 32), generator=g, device=device, dtype=torch.int32).to(torch.uint8)
+    scales = torch.randint(emin, emax + 1, (rows, K // 32), generator=g, device=device, dtype=torch.int32).to(torch.uint8)
     return codes, scales
+
+
+# Stacked decode: eps of the RMS normalisation between layers.
+STACK_RMS_EPS = 1e-6
 
 
 def float_normal(shape, std, device, seed, *tag):
