@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "../../include/stqmoe.h"
@@ -51,7 +52,43 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D = A * B + D for one m16n8k32 E4M3 tile with FP32 accumulators.
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+
+// 2^x as a float for x in [-127, 127] (2^-127 is the binary32 subnormal 0x00400000).
+__device__ __forceinline__ float pow2_float(int x) {
+  return x >= -126 ? __uint_as_float(uint32_t(x + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// Biased UE8M0 exponent of the smallest power of two 2^k with amax <= limit * 2^k,
+// where limit = 1.m * 2^p is given by its mantissa bits (m_lim) and exponent p
+// (E4M3's 448 = 1.75 * 2^8: m_lim 0x600000, p 8; E2M1's 6 = 1.5 * 2^2: 0x400000, 2).
+__device__ __forceinline__ int mx_scale_exponent(float amax, uint32_t m_lim, int p) {
+  if (amax == 0.f) return 127;
+  const uint32_t ab = __float_as_uint(amax);
+  const int eb = int(ab >> 23);
+  if (eb == 0) return 0;  // subnormal amax: k + 127 < 0
+  const int E = eb - 127;
+  const int k = ((ab & 0x7FFFFFu) <= m_lim) ? E - p : E - p + 1;
+  return min(max(k + 127, 0), 254);
+}
+
+// E4M3 code (round to nearest even, saturating) of v * f; a zero result keeps v's sign.
+__device__ __forceinline__ uint32_t e4m3_code(float v, float f) {
+  const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v * f, __NV_SATFINITE, __NV_E4M3);
+  uint32_t code = c;
+  if ((code & 0x7Fu) == 0u) code = (__float_as_uint(v) >> 31) << 7;
+  return code;
+}
 
 // Round an FP32 value to the bf16 grid and back (for intermediates stored as bf16).
 __device__ __forceinline__ float round_bf16(float f) { return __bfloat162float(__float2bfloat16_rn(f)); }

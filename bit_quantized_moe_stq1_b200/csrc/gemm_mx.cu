@@ -29,9 +29,10 @@ constexpr int kKT = 128;                          // k per stage
 constexpr int kATile = 128 * 128;                 // smem bytes of one 128 x 128 E2M1 tile (expanded)
 constexpr uint32_t kATx = 128 * 128 / 2;          // bytes the TMA delivers for it
 constexpr int kSf = 512;                          // one scale-factor atom: 128 rows x 4 k-blocks
-// Decode-size tiles (N <= 32) use half the shared memory so two CTAs share an SM and one
-// CTA's prologue and epilogue overlap the other's main loop.
-constexpr int smem_budget(int nt) { return nt <= 32 ? 100 * 1024 : 200 * 1024; }
+// Two CTAs share an SM (half the shared memory each), so one CTA's prologue and
+// epilogue overlap the other's main loop.
+constexpr int ctas_per_sm(int nt) { return nt > 0 ? 2 : 1; }
+constexpr int smem_budget(int nt) { return ctas_per_sm(nt) == 2 ? 112 * 1024 : 200 * 1024; }
 
 // PAIR = the gate/up pair of one expert: the 128-row A tile holds 64 gate rows (TMEM
 // lanes 0-63) and the same 64 rows of the up projection (lanes 64-127), so one MMA per
@@ -45,8 +46,8 @@ struct Cfg {
   static constexpr int kOffSfb = kOffSfa + kSf;
   static constexpr int kStageRaw = kOffSfb + kSf;
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kCtasPerSm = NT <= 32 ? 2 : 1;
-  static constexpr int kUBuf = PAIR ? 64 * 17 * 4 : 0;   // up-projection staging (row pitch 17 words)
+  static constexpr int kCtasPerSm = ctas_per_sm(NT);
+  static constexpr int kUBuf = PAIR ? 4 * 32 * 9 * 4 : 0;   // gate/up exchange of the epilogue (pitch 9 words)
   static constexpr int kStagesRaw = (smem_budget(NT) - 2048 - kUBuf) / kStage;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kSmem = kStages * kStage + kUBuf + 1024 /* barriers */ + 1024 /* alignment */;
@@ -105,28 +106,6 @@ __device__ __forceinline__ void load_sf_pair(uint32_t (&v)[4], const uint8_t* gs
 // Store them into the scale-factor atom: row m = m0 + 32*m1 at byte m0*16 + m1*4 + kb.
 __device__ __forceinline__ void store_sf(uint8_t* dst, const uint32_t (&v)[4], int lane) {
   *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
-}
-
-// E4M3 code of one value with a UE8M0 exponent e already chosen (zero keeps its sign).
-__device__ __forceinline__ uint32_t e4m3_code(float v, float f) {
-  const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v * f, __NV_SATFINITE, __NV_E4M3);
-  uint32_t code = c;
-  if ((code & 0x7Fu) == 0u) code = (__float_as_uint(v) >> 31) << 7;
-  return code;
-}
-
-__device__ __forceinline__ float pow2f(int x) {
-  return x >= -126 ? __uint_as_float(uint32_t(x + 127) << 23) : __uint_as_float(0x00400000u);
-}
-
-__device__ __forceinline__ int mxfp8_exponent(float amax) {
-  if (amax == 0.f) return 127;
-  const uint32_t ab = __float_as_uint(amax);
-  const int eb = int(ab >> 23);
-  if (eb == 0) return 0;
-  const int E = eb - 127;
-  const int k = ((ab & 0x7FFFFFu) <= 0x600000u) ? E - 8 : E - 7;  // 448 = 1.75 * 2^8
-  return min(max(k + 127, 0), 254);
 }
 
 template <int NT, bool PAIR>
@@ -282,31 +261,39 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
         tc::tmem_ld_x16(tl + c0, v);
         tc::tmem_ld_wait();
         if constexpr (PAIR) {
-          // lanes 64-127 (up) hand their values to lanes 0-63 (gate) through shared memory
-          if (q >= 2) {
+          // Warps q and q+2 hold the gate and up values of the same 32 features; the gate
+          // warp takes columns 0-7 of the chunk and the up warp columns 8-15, each handing
+          // the other its half through shared memory.
+          const int pr = q & 1;
+          const bool gate = q < 2;
+          float* mine = ubuf + (2 * pr + (gate ? 0 : 1)) * (32 * 9);
+          const float* other = ubuf + (2 * pr + (gate ? 1 : 0)) * (32 * 9);
+          if (gate) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) ubuf[((q - 2) * 32 + lane) * 17 + j] = __uint_as_float(v[j]);
+            for (int j = 0; j < 8; ++j) mine[lane * 9 + j] = __uint_as_float(v[8 + j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mine[lane * 9 + j] = __uint_as_float(v[j]);
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (q < 2) {
-            const int f = mt * 64 + 32 * q + lane;  // output feature of this lane
+          const int f = mt * 64 + 32 * pr + lane;  // output feature of this lane
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int col = n0 + c0 + j;
-              if (col >= cnt) break;
-              const float u = ubuf[(q * 32 + lane) * 17 + j];
-              const float h = silu_f32(__uint_as_float(v[j])) * u;
-              const bool bad = !isfinite(h);
-              float a = bad ? 0.f : fabsf(h);
+          for (int j = 0; j < 8; ++j) {
+            const int col = n0 + c0 + (gate ? j : 8 + j);
+            if (col >= cnt) break;
+            const float g = gate ? __uint_as_float(v[j]) : other[lane * 9 + j];
+            const float u = gate ? other[lane * 9 + j] : __uint_as_float(v[8 + j]);
+            const float h = silu_f32(g) * u;
+            const bool bad = !isfinite(h);
+            float a = bad ? 0.f : fabsf(h);
 #pragma unroll
-              for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-              const bool anybad = __any_sync(0xffffffffu, bad);
-              const int ex = anybad ? 255 : mxfp8_exponent(a);
-              const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2f(127 - ex));
-              const size_t pos = size_t(pos0 + col);
-              p.hq[pos * p.R + f] = uint8_t(code);
-              if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
-            }
+            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            const bool anybad = __any_sync(0xffffffffu, bad);
+            const int ex = anybad ? 255 : mx_scale_exponent(a, 0x600000u, 8);
+            const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2_float(127 - ex));
+            const size_t pos = size_t(pos0 + col);
+            p.hq[pos * p.R + f] = uint8_t(code);
+            if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
         } else {

@@ -122,23 +122,6 @@ __global__ void stq1_unpack_kernel(const uint8_t* __restrict__ in, int64_t rows,
 
 // ----------------------------------------------------------------------------- MXFP4
 
-// 2^x as a float for x in [-127, 127] (2^-127 is the binary32 subnormal 0x00400000).
-__device__ __forceinline__ float pow2_float(int x) {
-  return x >= -126 ? __uint_as_float(uint32_t(x + 127) << 23) : __uint_as_float(0x00400000u);
-}
-
-// Biased UE8M0 exponent of the smallest power of two 2^k with amax <= limit * 2^k,
-// where limit = 1.m * 2^p is given by its mantissa bits (m_lim) and exponent p.
-__device__ __forceinline__ int mx_scale_exponent(float amax, uint32_t m_lim, int p) {
-  if (amax == 0.f) return 127;
-  const uint32_t ab = __float_as_uint(amax);
-  const int eb = int(ab >> 23);
-  if (eb == 0) return 0;  // subnormal amax: k + 127 < 0
-  const int E = eb - 127;
-  const int k = ((ab & 0x7FFFFFu) <= m_lim) ? E - p : E - p + 1;
-  return min(max(k + 127, 0), 254);
-}
-
 // E2M1 round to nearest, ties to the even code, of y in [0, 6].
 __device__ __forceinline__ uint32_t e2m1_rne_mag(float y) {
   return uint32_t(y > 0.25f) + uint32_t(y >= 0.75f) + uint32_t(y > 1.25f) + uint32_t(y >= 1.75f) +
