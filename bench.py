@@ -43,6 +43,12 @@ BF16_MAT = I * H * 2                        # 25,165,824
 ROUTER_BYTES = E * H * 2                    # 3,145,728
 NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense BF16 tensor rate
 
+# DRAM bytes (read + write) per touched expert of one decode-size launch, from one ncu
+# capture of the same kernel build on a smaller case (named profile under profiles/); a
+# launch's traffic grows with its touched experts, so the full launch's traffic is this
+# figure times its touched experts.  An entry is removed when its kernel changes.
+MEASURED_TRAFFIC_PER_EXPERT = {}
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -283,11 +289,12 @@ class MoeLayers(Workload):
             else:
                 gu = t * 2 * MX_MAT + P * H * (1 + 1 / 32) + P * I * (1 + 1 / 32)
                 dn = t * MX_MAT + P * I * (1 + 1 / 32) + P * H * 4
-                kinds.setdefault("gate_up_mx", []).append(dict(bytes=gu, flops=4 * P * I * H))
-                kinds.setdefault("down_mx", []).append(dict(bytes=dn, flops=2 * P * I * H))
+                kinds.setdefault("gate_up_mx", []).append(dict(bytes=gu, flops=4 * P * I * H, touched=t))
+                kinds.setdefault("down_mx", []).append(dict(bytes=dn, flops=2 * P * I * H, touched=t))
         flops = len(self.layers) * 3 * 2 * T * K_TOP * I * H
         return dict(bytes=tot, flops=flops, per_kind={k: dict(bytes=float(np.mean([d["bytes"] for d in v])),
-                                                             flops=float(np.mean([d.get("flops", 0) for d in v])))
+                                                             flops=float(np.mean([d.get("flops", 0) for d in v])),
+                                                             touched=float(np.mean([d.get("touched", 0) for d in v])))
                                                       for k, v in kinds.items()})
 
 
@@ -432,6 +439,10 @@ def run_ours(args):
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                 "frac": achieved / pk["hbm"] if achieved else None, "peak_source": pk["src"] + " copy bandwidth",
                 "traffic": None, "bytes_per_launch": launch_bytes, "avg_launch_ms": avg_ms}
+    if dom in MEASURED_TRAFFIC_PER_EXPERT and wl.name != "prefill_w4a8" and per.get("touched"):
+        touched = float(np.mean([a["per_kind"][dom]["touched"] for a in acct if dom in a["per_kind"]]))
+        roof["traffic"] = MEASURED_TRAFFIC_PER_EXPERT[dom] * touched
+        roof["traffic_source"] = "ncu dram bytes per touched expert (smaller case) x touched experts per launch"
     tps = wl.tokens_per_step()
     if wl.unit == "GB/s":
         value = n * ab / (ms_step * 1e-3) / 1e9
@@ -443,7 +454,8 @@ def run_ours(args):
         "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 activations x STQ1_0 (ternary, fp16 scale) and MXFP4 x MXFP8 weights, fp32 accumulate",
+        "dtype": "bf16 x bf16 (STQ1_0 patterns x activations) and e2m1 x e4m3 (MXFP4 x MXFP8) "
+                 "tensor-core products, fp32 accumulate",
         "data": "synthetic (seeded generators; random weights on the format grids)",
         "config": {"workload": wl.name, "experts": E, "tokens_per_step": tps, "hbm_bytes_per_step": ab,
                    "touched_experts_per_layer": getattr(wl, "_acct", {}).get((args.warmup) % N_BATCHES),

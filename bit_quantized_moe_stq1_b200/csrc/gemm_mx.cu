@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
     // ---------------------------------------------------------------- producer
     // Scale factors are read kPf stages ahead into a register ring, so no stage waits
     // for a global load before its TMA is issued.
-    constexpr int kPf = 4;
+    constexpr int kPf = 8;
     int last_round[C::kStages];
 #pragma unroll
     for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;

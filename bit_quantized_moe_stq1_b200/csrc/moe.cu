@@ -350,6 +350,53 @@ __device__ __forceinline__ void shared_down(const MoeArgs& a, int bid, float (*r
   }
 }
 
+// Shared expert gate/up on its own (the MXFP4 layers, whose routed experts run on the
+// tensor-core GEMM): CTA = 16 features of h with 16 warps splitting K in 32-wide chunks,
+// so that each SM keeps enough loads in flight; the warps' partial sums are added in warp
+// order through shared memory (deterministic), warp w finishing token-chunk/fragment slot
+// w.  NCH token chunks of 8 per pass.  (The down projection, K = I, keeps the 4-warp CTAs
+// of the persistent STQ1_0 kernel: there the 16-way split left too little work per warp.)
+constexpr int kWideWarps = 16;
+
+template <int NCH>
+__global__ void __launch_bounds__(kWideWarps * 32) shared_gateup_wide_kernel(MoeArgs a) {
+  extern __shared__ float red[];  // [warp][2][NCH][4][32]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  const int f0 = blockIdx.x * 16;
+  const int nch = a.H / 32;
+  const int k0 = 32 * (warp * nch / kWideWarps), k1 = 32 * ((warp + 1) * nch / kWideWarps);
+  const uint16_t* rowg[2] = {a.sg + size_t(f0 + g) * a.H, a.su + size_t(f0 + g) * a.H};
+  for (int t0 = 0; t0 < a.T; t0 += 8 * NCH) {
+    const uint16_t* xr[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int tok = t0 + 8 * c + g;
+      xr[c] = tok < a.T ? a.x + size_t(tok) * a.H : nullptr;
+    }
+    float acc[2][NCH][4] = {};
+    bf16_warp_gemv<2, NCH>(rowg, a.H, k0, k1, xr, acc);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[(((warp * 2 + i) * NCH + c) * 4 + j) * 32 + lane] = acc[i][c][j];
+    __syncthreads();
+    if (warp < NCH * 4) {
+      const int c = warp >> 2, j = warp & 3;
+      float gs = 0.f, us = 0.f;
+      for (int w = 0; w < kWideWarps; ++w) {
+        gs += red[(((w * 2 + 0) * NCH + c) * 4 + j) * 32 + lane];
+        us += red[(((w * 2 + 1) * NCH + c) * 4 + j) * 32 + lane];
+      }
+      const int tok = t0 + 8 * c + 2 * t + (j & 1);
+      const int f = f0 + g + 8 * (j >> 1);
+      if (tok < a.T) a.h[size_t(a.P + tok) * a.I + f] = float_to_bf16_bits(silu_f32(gs) * us);
+    }
+    __syncthreads();
+  }
+}
+
 // Next work item of a persistent CTA (one atomic per item, broadcast through smem).
 __device__ __forceinline__ int next_item(int32_t* counter, int* slot) {
   if (threadIdx.x == 0) *slot = atomicAdd(counter, 1);
@@ -565,17 +612,30 @@ extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
 
 // The BF16 shared expert alone (used by MXFP4 layers): the shared CTAs of the two
 // STQ1_0 kernels.
+template <int NCH>
+stq_status launch_shared_gateup_wide(const MoeArgs& a, cudaStream_t s) {
+  const int smem = kWideWarps * 2 * NCH * 4 * 32 * 4;
+  static int attr_device = -1;  // the >48 KB opt-in, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return STQ_ERR_CUDA;
+  if (attr_device != dev) {
+    if (cudaFuncSetAttribute(shared_gateup_wide_kernel<NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return STQ_ERR_CUDA;
+    attr_device = dev;
+  }
+  StqTimed tm(STQ_K_SHARED_GATE_UP, s);
+  shared_gateup_wide_kernel<NCH><<<unsigned(a.I / 16), kWideWarps * 32, smem, s>>>(a);
+  return stq_launch_status();
+}
+
 stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
+  stq_status st = a0.T <= 8    ? launch_shared_gateup_wide<1>(a0, s)
+                  : a0.T <= 16 ? launch_shared_gateup_wide<2>(a0, s)
+                               : launch_shared_gateup_wide<4>(a0, s);
+  if (st != STQ_OK) return st;
   MoeArgs a = a0;
   a.routed = 0;
-  a.n_shared_cta = a.I / 16;
-  a.sched = a0.sched + 2;
-  {
-    StqTimed tm(STQ_K_SHARED_GATE_UP, s);
-    moe_gateup_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta)), 128, 0, s>>>(a);
-  }
-  stq_status st = stq_launch_status();
-  if (st != STQ_OK) return st;
   a.n_shared_cta = a.H / 16;
   a.sched = a0.sched + 3;
   {

@@ -111,8 +111,9 @@ def _make_layer(S, T, H, I, E, k, shared, tag):
     return gw, packs, sh, wr, x
 
 
-def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None):
-    gw, packs, sh, wr, x = _make_layer(S, T, H, I, E, k, shared, tag)
+def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None, x=None):
+    gw, packs, sh, wr, x0 = _make_layer(S, T, H, I, E, k, shared, tag)
+    x = x0 if x is None else x
     if ids is None:
         ids, tw, _ = S.moe_router_topk(x, wr, k)
     desc = S.make_desc(T, H, I, E, k, out_fp32=True, add_residual=residual)
@@ -221,6 +222,18 @@ def test_moe_stq_residual_and_bf16_output(S):
     assert np.allclose(out[(True, True)], out[(True, False)] + xd, rtol=1e-6, atol=1e-6)
     ref_b = F.bf16_decode(F.bf16_encode_rne(out[(True, True)]))
     assert np.array_equal(out[(False, True)], ref_b)
+
+
+def test_moe_stq_wide_range_activations(S):
+    """Activations spanning 2^-30 .. 2^30 within each row, and a zero row."""
+    T, H, I, E, k = 6, 512, 256, 8, 2
+    g = W.generator(DEV, 0, "wide", "mag")
+    mag = torch.exp2(torch.randint(-30, 31, (T, H), generator=g, device=DEV).float())
+    x = (W.bf16_normal((T, H), 1.0, DEV, 0, "wide", "x").float() * mag).to(torch.bfloat16)
+    x[3] = 0
+    ids, tw = W.uniform_routing(T, E, k, DEV, 0, "wide", "ids")
+    r = _run_layer(S, T, H, I, E, k, True, "wide", ids=ids, tw=tw, x=x)
+    _check_layer(r, T, H, I, E, k)
 
 
 def test_moe_bad_expert_id_reports_and_skips(S):
