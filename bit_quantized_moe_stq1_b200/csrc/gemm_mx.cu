@@ -29,9 +29,9 @@ constexpr int kKT = 128;                          // k per stage
 constexpr int kATile = 128 * 128;                 // smem bytes of one 128 x 128 E2M1 tile (expanded)
 constexpr uint32_t kATx = 128 * 128 / 2;          // bytes the TMA delivers for it
 constexpr int kSf = 512;                          // one scale-factor atom: 128 rows x 4 k-blocks
-// Two CTAs share an SM (half the shared memory each), so one CTA's prologue and
-// epilogue overlap the other's main loop.
-constexpr int ctas_per_sm(int nt) { return nt > 0 ? 2 : 1; }
+// Two CTAs share an SM (half the shared memory each) unless the two accumulator buffers
+// of the 128-wide N tile need more than half of the SM's 512 TMEM columns.
+constexpr int ctas_per_sm(int nt) { return nt <= 64 ? 2 : 1; }
 constexpr int smem_budget(int nt) { return ctas_per_sm(nt) == 2 ? 112 * 1024 : 200 * 1024; }
 
 // PAIR = the gate/up pair of one expert: the 128-row A tile holds 64 gate rows (TMEM
@@ -52,14 +52,17 @@ struct Cfg {
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kSmem = kStages * kStage + kUBuf + 1024 /* barriers */ + 1024 /* alignment */;
   static constexpr int kRowsPerTile = PAIR ? 64 : 128;   // output features per CTA
-  static constexpr int kColSfa = NT;
-  static constexpr int kColSfb = NT + 4;
-  static constexpr int kColsUsed = NT + 8;
+  // TMEM: accumulator buffers at columns 0 and NT (tile i uses buffer i & 1), then the
+  // scale factors of the current k-block.
+  static constexpr int kColSfa = 2 * NT;
+  static constexpr int kColSfb = 2 * NT + 4;
+  static constexpr int kColsUsed = 2 * NT + 8;
   static constexpr uint32_t kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
   static constexpr uint32_t kTx = kATx + uint32_t(kB);
   static_assert(kStages >= 2, "shared memory budget");
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "tile N");
+  static_assert(kCtasPerSm * kCols <= 512, "TMEM columns");
 };
 
 struct GemmProblem {
@@ -71,6 +74,7 @@ struct GemmProblem {
   const int2* ntiles;           // grouped: (expert, first token) per N tile
   const int32_t* n_ntiles;      // grouped: number of N tiles (device)
   int dense_M;
+  int max_items;                // upper bound of the work items (N tiles x M tiles)
   float* Y;                     // single: [Ptot][R]
   uint8_t* hq;                  // pair: MXFP8 codes of h [Ptot][R]
   uint8_t* hs;                  // pair: scales [Ptot][R/32]
@@ -108,6 +112,44 @@ __device__ __forceinline__ void store_sf(uint8_t* dst, const uint32_t (&v)[4], i
   *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
+// One work item = (N tile, M tile); item i covers N tile i / MT and M tile i % MT.
+struct Item {
+  bool valid;
+  int mt, n0, pos0, cnt, arow, brow;
+};
+
+template <int NT>
+__device__ __forceinline__ Item get_item(const GemmProblem& p, int item, int MT, int rows_per_tile) {
+  Item t{};
+  const int nti = item / MT;
+  t.mt = item - nti * MT;
+  int e;
+  if (p.offsets != nullptr) {
+    t.valid = item < p.max_items && nti < *p.n_ntiles;
+    if (!t.valid) return t;
+    const int2 w = p.ntiles[nti];
+    e = w.x;
+    t.n0 = w.y;
+    t.pos0 = p.offsets[e];
+    t.cnt = p.offsets[e + 1] - t.pos0;
+  } else {
+    t.valid = item < p.max_items;
+    if (!t.valid) return t;
+    e = 0;
+    t.n0 = nti * NT;
+    t.pos0 = 0;
+    t.cnt = p.dense_M;
+  }
+  t.arow = e * p.R + t.mt * rows_per_tile;
+  t.brow = t.pos0 + t.n0;
+  return t;
+}
+
+// Persistent: CTA b takes items b, b + gridDim.x, ...  Warp roles: warp 0 loads (TMA
+// for the operands, a register ring kPf stages ahead for the scale factors), warp 1
+// issues the MMAs (one elected thread), warps 2-5 drain the accumulators.  The smem
+// ring and its barrier phases run on across items; the accumulator is double-buffered
+// in TMEM (tfull / tempty), so the epilogue of one item overlaps the MMAs of the next.
 template <int NT, bool PAIR>
 __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
@@ -118,39 +160,25 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
   float* ubuf = reinterpret_cast<float*>(smem + C::kStages * C::kStage);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage + C::kUBuf);
   uint64_t* empty = full + C::kStages;
-  uint64_t* accum = empty + C::kStages;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
+  uint64_t* tfull = empty + C::kStages;   // [2]
+  uint64_t* tempty = tfull + 2;           // [2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT = p.R / C::kRowsPerTile;
-  const int item = blockIdx.x;
-  const int mt = item % MT;
-  int e, n0, pos0, cnt;
-  if (p.offsets != nullptr) {
-    const int nti = item / MT;
-    if (nti >= *p.n_ntiles) return;
-    const int2 w = p.ntiles[nti];
-    e = w.x;
-    n0 = w.y;
-    pos0 = p.offsets[e];
-    cnt = p.offsets[e + 1] - pos0;
-  } else {
-    e = 0;
-    n0 = (item / MT) * NT;
-    pos0 = 0;
-    cnt = p.dense_M;
-  }
+  const int G = gridDim.x;
   const int nk = p.K / kKT;
   const int k32 = p.K / 32;
-  const int arow = e * p.R + mt * C::kRowsPerTile;  // first A row (both matrices for a pair)
-  const int brow = pos0 + n0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       tc::mbar_init(&full[s], 1);
       tc::mbar_init(&empty[s], 1);
     }
-    tc::mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&tfull[b], 1);
+      tc::mbar_init(&tempty[b], 4);
+    }
     tc::fence_barrier_init();
     tc::prefetch_tensormap(&tmA);
     if (PAIR) tc::prefetch_tensormap(&tmA2);
@@ -164,99 +192,124 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Scale factors are read kPf stages ahead into a register ring, so no stage waits
-    // for a global load before its TMA is issued.
     constexpr int kPf = 8;
     int last_round[C::kStages];
 #pragma unroll
     for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;
-    uint32_t ra[kPf][4], rb[kPf][4];
-#pragma unroll
-    for (int d = 0; d < kPf; ++d) {
-      if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, arow, k32, d, nk, lane);
-      else load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, d, nk, lane);
-      load_sf(rb[d], p.sb, brow, NT, p.Ptot, k32, d, nk, lane);
-    }
+    int s = 0, r = 0;  // stage and round of the next k-step (continuing across items)
     bool ok = true;
-    for (int k0 = 0; k0 < nk && ok; k0 += kPf) {
+    for (int it = 0; ok; ++it) {
+      const Item I = get_item<NT>(p, blockIdx.x + it * G, MT, C::kRowsPerTile);
+      if (!I.valid) break;
+      uint32_t ra[kPf][4], rb[kPf][4];
 #pragma unroll
       for (int d = 0; d < kPf; ++d) {
-        const int kt = k0 + d;
-        if (kt >= nk) break;
-        const int s = kt % C::kStages, r = kt / C::kStages;
-        if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = smem + s * C::kStage;
-        store_sf(st + C::kOffSfa, ra[d], lane);
-        store_sf(st + C::kOffSfb, rb[d], lane);
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tc::mbar_arrive_expect_tx(&full[s], C::kTx);
-          if (PAIR) {
-            tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);              // gate rows -> lanes 0-63
-            tc::tma_load_2d(st + C::kOffA + kATile / 2, &tmA2, kt * kKT, arow, &full[s]);  // up rows -> lanes 64-127
-          } else {
-            tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, arow, &full[s]);
+        if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, d, nk, lane);
+        else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, d, nk, lane);
+        load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, d, nk, lane);
+      }
+      for (int k0 = 0; k0 < nk && ok; k0 += kPf) {
+#pragma unroll
+        for (int d = 0; d < kPf; ++d) {
+          const int kt = k0 + d;
+          if (kt >= nk) break;
+          if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
+            ok = false;
+            break;
           }
-          tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, brow, &full[s]);
+          uint8_t* st = smem + s * C::kStage;
+          store_sf(st + C::kOffSfa, ra[d], lane);
+          store_sf(st + C::kOffSfb, rb[d], lane);
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc::mbar_arrive_expect_tx(&full[s], C::kTx);
+            if (PAIR) {
+              tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, I.arow, &full[s]);              // gate rows: lanes 0-63
+              tc::tma_load_2d(st + C::kOffA + kATile / 2, &tmA2, kt * kKT, I.arow, &full[s]);  // up rows: 64-127
+            } else {
+              tc::tma_load_2d(st + C::kOffA, &tmA, kt * kKT, I.arow, &full[s]);
+            }
+            tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, I.brow, &full[s]);
+          }
+          last_round[s] = r;
+          if (++s == C::kStages) {
+            s = 0;
+            ++r;
+          }
+          if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt + kPf, nk, lane);
+          else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
+          load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt + kPf, nk, lane);
         }
-        last_round[s] = r;
-        if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, arow, k32, kt + kPf, nk, lane);
-        else load_sf(ra[d], p.sa, arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
-        load_sf(rb[d], p.sb, brow, NT, p.Ptot, k32, kt + kPf, nk, lane);
       }
     }
     // every issued load has landed before the CTA may exit
-#pragma unroll
-    for (int s = 0; s < C::kStages; ++s)
-      if (last_round[s] >= 0) tc::mbar_wait(&full[s], last_round[s] & 1, p.err);
+    for (int q = 0; q < C::kStages; ++q)
+      if (last_round[q] >= 0) tc::mbar_wait(&full[q], last_round[q] & 1, p.err);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      for (int kt = 0; kt < nk; ++kt) {
-        const int s = kt % C::kStages, r = kt / C::kStages;
-        if (!tc::mbar_wait(&full[s], r & 1, p.err)) break;
+      int s = 0, r = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int item = blockIdx.x + it * G;
+        if (item >= p.max_items || (p.offsets != nullptr && item / MT >= *p.n_ntiles)) break;
+        const int buf = it & 1;
+        if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
-        uint8_t* st = smem + s * C::kStage;
-        tc::cp_sf_32x128b_x4(tmem + C::kColSfa, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa)));
-        tc::cp_sf_32x128b_x4(tmem + C::kColSfb, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfb)));
-        const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA));
-        const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffB));
+        const uint32_t acc_col = tmem + uint32_t(buf * NT);
+        for (int kt = 0; kt < nk; ++kt) {
+          if (!tc::mbar_wait(&full[s], r & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          uint8_t* st = smem + s * C::kStage;
+          tc::cp_sf_32x128b_x4(tmem + C::kColSfa, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa)));
+          tc::cp_sf_32x128b_x4(tmem + C::kColSfb, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfb)));
+          const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA));
+          const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffB));
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          const uint32_t idesc = tc::idesc_mxf8f6f4(NT, uint32_t(kb), uint32_t(kb));
-          const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-          tc::mma_mxf8f6f4(tmem, da + 2 * kb, db + 2 * kb, idesc, (tmem + C::kColSfa) | (uint32_t(kb) << 30),
-                           (tmem + C::kColSfb) | (uint32_t(kb) << 30), acc);
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t idesc = tc::idesc_mxf8f6f4(NT, uint32_t(kb), uint32_t(kb));
+            const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+            tc::mma_mxf8f6f4(acc_col, da + 2 * kb, db + 2 * kb, idesc, (tmem + C::kColSfa) | (uint32_t(kb) << 30),
+                             (tmem + C::kColSfb) | (uint32_t(kb) << 30), acc);
+          }
+          tc::commit(&empty[s]);
+          if (++s == C::kStages) {
+            s = 0;
+            ++r;
+          }
         }
-        tc::commit(&empty[s]);
+        tc::commit(&tfull[buf]);  // also after an aborted item, so the epilogue never waits for ever
       }
-      tc::commit(accum);  // also on an aborted loop, so the epilogue never waits for ever
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
-    bool ok = tc::mbar_wait(accum, 0, p.err);
-    if constexpr (PAIR) {
-      // the four epilogue warps meet at named barriers below, so they agree on ok first
-      uint32_t all;
-      asm volatile(
-          "{\n .reg .pred p, r;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred r, 1, 128, p;\n"
-          " selp.u32 %0, 1, 0, r;\n}"
-          : "=r"(all)
-          : "r"(ok ? 1u : 0u)
-          : "memory");
-      ok = all != 0u;
-    }
-    tc::fence_after_sync();
-    const uint32_t tl = tmem + (uint32_t(32 * q) << 16);
-    if (ok) {
+    for (int it = 0;; ++it) {
+      const Item I = get_item<NT>(p, blockIdx.x + it * G, MT, C::kRowsPerTile);
+      if (!I.valid) break;
+      const int buf = it & 1;
+      bool ok = tc::mbar_wait(&tfull[buf], (it >> 1) & 1, p.err);
+      if constexpr (PAIR) {
+        // the four epilogue warps meet at named barriers below, so they agree on ok first
+        uint32_t all;
+        asm volatile(
+            "{\n .reg .pred p, r;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred r, 1, 128, p;\n"
+            " selp.u32 %0, 1, 0, r;\n}"
+            : "=r"(all)
+            : "r"(ok ? 1u : 0u)
+            : "memory");
+        ok = all != 0u;
+      }
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * NT);
       for (int c0 = 0; c0 < NT; c0 += 16) {
-        if (n0 + c0 >= cnt) break;
+        if (I.n0 + c0 >= I.cnt) break;
         uint32_t v[16];
         tc::tmem_ld_x16(tl + c0, v);
         tc::tmem_ld_wait();
@@ -276,11 +329,11 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
             for (int j = 0; j < 8; ++j) mine[lane * 9 + j] = __uint_as_float(v[j]);
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
-          const int f = mt * 64 + 32 * pr + lane;  // output feature of this lane
+          const int f = I.mt * 64 + 32 * pr + lane;  // output feature of this lane
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int col = n0 + c0 + (gate ? j : 8 + j);
-            if (col >= cnt) break;
+            const int col = I.n0 + c0 + (gate ? j : 8 + j);
+            if (col >= I.cnt) break;
             const float g = gate ? __uint_as_float(v[j]) : other[lane * 9 + j];
             const float u = gate ? other[lane * 9 + j] : __uint_as_float(v[8 + j]);
             const float h = silu_f32(g) * u;
@@ -291,21 +344,25 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
             const bool anybad = __any_sync(0xffffffffu, bad);
             const int ex = anybad ? 255 : mx_scale_exponent(a, 0x600000u, 8);
             const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2_float(127 - ex));
-            const size_t pos = size_t(pos0 + col);
+            const size_t pos = size_t(I.pos0 + col);
             p.hq[pos * p.R + f] = uint8_t(code);
             if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
         } else {
-          const int f = mt * 128 + 32 * q + lane;
+          const int f = I.mt * 128 + 32 * q + lane;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int col = n0 + c0 + j;
-            if (col >= cnt) break;
-            p.Y[size_t(pos0 + col) * p.R + f] = __uint_as_float(v[j]);
+            const int col = I.n0 + c0 + j;
+            if (col >= I.cnt) break;
+            p.Y[size_t(I.pos0 + col) * p.R + f] = __uint_as_float(v[j]);
           }
         }
       }
+      // this warp's reads of the buffer are complete: hand it back to the MMA warp
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[buf]);
     }
   }
   tc::fence_before_sync();
@@ -389,9 +446,20 @@ bool map_u8(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  return sms;
+}
+
+// Persistent launch over p.max_items work items: at most kCtasPerSm CTAs per SM.
 template <int NT, bool PAIR>
 stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
-                       unsigned grid, cudaStream_t s) {
+                       cudaStream_t s) {
   using C = Cfg<NT, PAIR>;
   static bool configured = false;
   if (!configured) {
@@ -400,19 +468,21 @@ stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtens
       return STQ_ERR_CUDA;
     configured = true;
   }
-  if (grid == 0) return STQ_OK;
+  if (p.max_items <= 0) return STQ_OK;
+  const int cap = C::kCtasPerSm * sm_count();
+  const unsigned grid = unsigned(p.max_items < cap ? p.max_items : cap);
   w4a8_gemm_kernel<NT, PAIR><<<grid, 192, C::kSmem, s>>>(a, a2, b, p);
   return stq_launch_status();
 }
 
 template <bool PAIR>
 stq_status launch_nt(int nt, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
-                     unsigned grid, cudaStream_t s) {
+                     cudaStream_t s) {
   switch (nt) {
-    case 16: return launch_gemm<16, PAIR>(a, a2, b, p, grid, s);
-    case 32: return launch_gemm<32, PAIR>(a, a2, b, p, grid, s);
-    case 64: return launch_gemm<64, PAIR>(a, a2, b, p, grid, s);
-    default: return launch_gemm<128, PAIR>(a, a2, b, p, grid, s);
+    case 16: return launch_gemm<16, PAIR>(a, a2, b, p, s);
+    case 32: return launch_gemm<32, PAIR>(a, a2, b, p, s);
+    case 64: return launch_gemm<64, PAIR>(a, a2, b, p, s);
+    default: return launch_gemm<128, PAIR>(a, a2, b, p, s);
   }
 }
 
@@ -458,9 +528,10 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   gp.hq = a.hq;
   gp.hs = a.hs;
   gp.err = a.err;
+  gp.max_items = max_tiles * (a.I / 64);
   {
     StqTimed tm(STQ_K_GATE_UP_MX, s);
-    st = launch_nt<true>(nt, mg, mu, mx, gp, unsigned(max_tiles * (a.I / 64)), s);
+    st = launch_nt<true>(nt, mg, mu, mx, gp, s);
   }
   if (st != STQ_OK) return st;
   if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
@@ -474,9 +545,10 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   dp.Y = a.Y;
   dp.hq = nullptr;
   dp.hs = nullptr;
+  dp.max_items = max_tiles * (a.H / 128);
   {
     StqTimed tm(STQ_K_DOWN_MX, s);
-    st = launch_nt<false>(nt, md, md, mh, dp, unsigned(max_tiles * (a.H / 128)), s);
+    st = launch_nt<false>(nt, md, md, mh, dp, s);
   }
   return st;
 }
@@ -508,7 +580,9 @@ extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales,
   p.dense_M = int(M);
   p.Y = y;
   p.err = err;
-  const unsigned grid = unsigned((N / 128) * ((M + nt - 1) / nt));
+  const int64_t items = (N / 128) * ((M + nt - 1) / nt);
+  STQ_HOST_CHECK(items < (int64_t(1) << 31), STQ_ERR_SHAPE);
+  p.max_items = int(items);
   StqTimed tm(STQ_K_GEMM, s);
-  return launch_nt<false>(nt, ma, ma, mb, p, grid, s);
+  return launch_nt<false>(nt, ma, ma, mb, p, s);
 }
