@@ -22,6 +22,7 @@
 
 #include "moe_internal.cuh"
 #include "tcgen05.cuh"
+#include "tma.cuh"
 
 namespace {
 
@@ -408,43 +409,7 @@ __global__ void __launch_bounds__(1024) mx_plan_kernel(const int32_t* __restrict
 
 // ----------------------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
 
-// E2M1 weights [rows][K] (two per byte), box 128 x box_rows, expanded to 16 bytes per 16 elements.
-bool map_e2m1(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows = 128) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {K, rows};
-  const cuuint64_t strides[1] = {K / 2};
-  const cuuint32_t box[2] = {128, box_rows};
-  const cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// E4M3 activations [rows][K] bytes, box 128 x box_rows.
-bool map_u8(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {K, rows};
-  const cuuint64_t strides[1] = {K};
-  const cuuint32_t box[2] = {128, box_rows};
-  const cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 int sm_count() {
   static int sms = 0;
@@ -492,7 +457,7 @@ int pick_nt(int64_t tokens_per_expert) {
 
 }  // namespace
 
-// Defined in moe.cu: the BF16 shared-expert CTAs of the STQ1_0 kernels.
+// Defined in moe.cu: the shared BF16 expert on its own.
 stq_status moe_shared_expert_bf16(const MoeArgs& a, cudaStream_t s);
 
 stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStream_t s) {
@@ -511,9 +476,9 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   const int max_tiles = P / nt + (a.E < P ? a.E : P);
   // 3. gate/up pair with SwiGLU and MXFP8 h
   CUtensorMap mg, mu, mx, md, mh;
-  if (!map_e2m1(&mg, a.wg, uint64_t(a.H), uint64_t(a.E) * a.I, 64) ||
-      !map_e2m1(&mu, a.wu, uint64_t(a.H), uint64_t(a.E) * a.I, 64) || !map_u8(&mx, a.xq, a.H, P, nt) ||
-      !map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !map_u8(&mh, a.hq, a.I, P, nt))
+  if (!tma::map_e2m1(&mg, a.wg, uint64_t(a.H), uint64_t(a.E) * a.I, 64) ||
+      !tma::map_e2m1(&mu, a.wu, uint64_t(a.H), uint64_t(a.E) * a.I, 64) || !tma::map_u8(&mx, a.xq, a.H, P, nt) ||
+      !tma::map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !tma::map_u8(&mh, a.hq, a.I, P, nt))
     return STQ_ERR_CUDA;
   GemmProblem gp{};
   gp.R = a.I;
@@ -569,7 +534,7 @@ extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales,
   int nt = pick_nt(M);
   while (nt > 16 && (N / 128) * ((M + nt - 1) / nt) < 148) nt /= 2;  // fill the SMs
   CUtensorMap ma, mb;
-  if (!map_e2m1(&ma, w_codes, uint64_t(K), uint64_t(N)) || !map_u8(&mb, a_codes, uint64_t(K), uint64_t(M), nt))
+  if (!tma::map_e2m1(&ma, w_codes, uint64_t(K), uint64_t(N)) || !tma::map_u8(&mb, a_codes, uint64_t(K), uint64_t(M), nt))
     return STQ_ERR_CUDA;
   GemmProblem p{};
   p.R = int(N);
