@@ -4,8 +4,8 @@
 // FP8 E4M3 activations, group 32, UE8M0 scales; the page notes that FP4 GEMMs need
 // Blackwell.
 //
-// One CTA computes a 128 (weight rows) x NT (tokens of one expert) tile over all of K:
-//   warp 0     producer: per 128-k stage, TMA tile loads of the weights (E2M1 expanded
+// A work item is a 128 (weight rows) x NT (tokens of one expert) tile over all of K:
+//   warps 0, 6 producers (alternate stages): per 128-k stage, TMA tile loads of the weights (E2M1 expanded
 //              to one 16-element group per 16 bytes by the TMA, 128-byte swizzle) and of
 //              the token activations (E4M3), and the UE8M0 scales of both, re-laid by the
 //              warp into the scale-factor atom the MMA reads (row m of a 128-row block at
@@ -50,7 +50,10 @@ struct Cfg {
   static constexpr int kCtasPerSm = ctas_per_sm(NT);
   static constexpr int kUBuf = PAIR ? 4 * 32 * 9 * 4 : 0;   // gate/up exchange of the epilogue (pitch 9 words)
   static constexpr int kStagesRaw = (smem_budget(NT) - 2048 - kUBuf) / kStage;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // even: the two producer warps own alternate stages (producer p fills stages 2i + p);
+  // an odd count (one producer with a stage more than the other) measured slower
+  static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) & ~1;
+  static constexpr int stages_of(int) { return kStages / 2; }
   static constexpr int kSmem = kStages * kStage + kUBuf + 1024 /* barriers */ + 1024 /* alignment */;
   static constexpr int kRowsPerTile = PAIR ? 64 : 128;   // output features per CTA
   // TMEM: accumulator buffers at columns 0 and NT (tile i uses buffer i & 1), then the
@@ -61,7 +64,7 @@ struct Cfg {
   static constexpr uint32_t kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
   static constexpr uint32_t kTx = kATx + uint32_t(kB);
-  static_assert(kStages >= 2, "shared memory budget");
+  static_assert(kStages >= 2, "shared memory budget (one stage per producer at least)");
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "tile N");
   static_assert(kCtasPerSm * kCols <= 512, "TMEM columns");
 };
@@ -146,13 +149,17 @@ __device__ __forceinline__ Item get_item(const GemmProblem& p, int item, int MT,
   return t;
 }
 
-// Persistent: CTA b takes items b, b + gridDim.x, ...  Warp roles: warp 0 loads (TMA
-// for the operands, a register ring kPf stages ahead for the scale factors), warp 1
-// issues the MMAs (one elected thread), warps 2-5 drain the accumulators.  The smem
+// Persistent: CTA b takes items b, b + gridDim.x, ...  Warp roles: warps 0 and 6 load
+// (TMA for the operands, a register ring kPf of their stages ahead for the scale
+// factors), warp 1 issues the MMAs (one elected thread), warps 2-5 drain the
+// accumulators.  The smem
 // ring and its barrier phases run on across items; the accumulator is double-buffered
 // in TMEM (tfull / tempty), so the epilogue of one item overlaps the MMAs of the next.
+constexpr int kGemmThreads = 224;  // producer, MMA, 4 epilogue warps, second producer
+constexpr int kProducer2 = 6;
+
 template <int NT, bool PAIR>
-__global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
+__global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, GemmProblem p) {
   using C = Cfg<NT, PAIR>;
@@ -191,29 +198,37 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
+  if (warp == 0 || warp == kProducer2) {
+    // ---------------------------------------------------------------- producers
+    // Two producer warps take alternate k-steps (global step g = item * nk + kt, producer
+    // g & 1), so the scale-factor stores and proxy fences of one stage overlap the other's.
+    // Producer p's j-th step uses stage 2 (j % n_p) + p, round j / n_p, with n_p the number
+    // of stages of parity p: no stage is shared, so each warp's final wait for its own
+    // loads is exact.
     constexpr int kPf = 8;
+    const int pid = warp == 0 ? 0 : 1;
     int last_round[C::kStages];
 #pragma unroll
     for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;
-    int s = 0, r = 0;  // stage and round of the next k-step (continuing across items)
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const Item I = get_item<NT>(p, blockIdx.x + it * G, MT, C::kRowsPerTile);
       if (!I.valid) break;
+      const int kt0 = ((pid - it * nk) % 2 + 2) % 2;  // first k-step of this item for this producer
       uint32_t ra[kPf][4], rb[kPf][4];
 #pragma unroll
       for (int d = 0; d < kPf; ++d) {
-        if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, d, nk, lane);
-        else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, d, nk, lane);
-        load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, d, nk, lane);
+        if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt0 + 2 * d, nk, lane);
+        else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt0 + 2 * d, nk, lane);
+        load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt0 + 2 * d, nk, lane);
       }
-      for (int k0 = 0; k0 < nk && ok; k0 += kPf) {
+      for (int k0 = kt0; k0 < nk && ok; k0 += 2 * kPf) {
 #pragma unroll
         for (int d = 0; d < kPf; ++d) {
-          const int kt = k0 + d;
+          const int kt = k0 + 2 * d;
           if (kt >= nk) break;
+          const int j = (it * nk + kt) >> 1, np = C::stages_of(pid);
+          const int s = 2 * (j % np) + pid, r = j / np;
           if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
             ok = false;
             break;
@@ -234,23 +249,19 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
             tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, I.brow, &full[s]);
           }
           last_round[s] = r;
-          if (++s == C::kStages) {
-            s = 0;
-            ++r;
-          }
-          if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt + kPf, nk, lane);
-          else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt + kPf, nk, lane);
-          load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt + kPf, nk, lane);
+          if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt + 2 * kPf, nk, lane);
+          else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt + 2 * kPf, nk, lane);
+          load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt + 2 * kPf, nk, lane);
         }
       }
     }
-    // every issued load has landed before the CTA may exit
+    // every load this warp issued has landed before the CTA may exit
     for (int q = 0; q < C::kStages; ++q)
       if (last_round[q] >= 0) tc::mbar_wait(&full[q], last_round[q] & 1, p.err);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      int s = 0, r = 0;
+      int g = 0;  // global k-step
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int item = blockIdx.x + it * G;
@@ -259,7 +270,9 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
         if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
         const uint32_t acc_col = tmem + uint32_t(buf * NT);
-        for (int kt = 0; kt < nk; ++kt) {
+        for (int kt = 0; kt < nk; ++kt, ++g) {
+          const int j = g >> 1, np = C::stages_of(g & 1);
+          const int s = 2 * (j % np) + (g & 1), r = j / np;
           if (!tc::mbar_wait(&full[s], r & 1, p.err)) {
             ok = false;
             break;
@@ -278,10 +291,6 @@ __global__ void __launch_bounds__(192, Cfg<NT, PAIR>::kCtasPerSm)
                              (tmem + C::kColSfb) | (uint32_t(kb) << 30), acc);
           }
           tc::commit(&empty[s]);
-          if (++s == C::kStages) {
-            s = 0;
-            ++r;
-          }
         }
         tc::commit(&tfull[buf]);  // also after an aborted item, so the epilogue never waits for ever
       }
@@ -436,7 +445,7 @@ stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtens
   if (p.max_items <= 0) return STQ_OK;
   const int cap = C::kCtasPerSm * sm_count();
   const unsigned grid = unsigned(p.max_items < cap ? p.max_items : cap);
-  w4a8_gemm_kernel<NT, PAIR><<<grid, 192, C::kSmem, s>>>(a, a2, b, p);
+  w4a8_gemm_kernel<NT, PAIR><<<grid, kGemmThreads, C::kSmem, s>>>(a, a2, b, p);
   return stq_launch_status();
 }
 

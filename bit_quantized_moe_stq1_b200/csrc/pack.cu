@@ -187,59 +187,66 @@ __global__ void mxfp4_unpack_kernel(const uint8_t* __restrict__ codes, const uin
 // ----------------------------------------------------------------------------- MXFP8
 
 // Four lanes per 32-element group, eight elements per lane.
-__global__ void mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
-                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                        const int32_t* __restrict__ rowmap, int k) {
-  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t gi = tid >> 2;
-  const int part = int(tid & 3);
-  const int64_t ng = rows * (K / 32);
-  const bool active = gi < ng;
-  float v[8];
-  float amax = 0.f;
-  bool bad = false;
-  if (active) {
-    const int64_t gpr = K / 32, row = gi / gpr, col = gi % gpr;
-    const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
-    const uint4 raw = *reinterpret_cast<const uint4*>(x + src * K + col * 32 + part * 8);
-    const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+// Grid (column chunks of 2048 elements, rows; rows beyond 65535 loop): thread = 8
+// consecutive elements, 4 threads = one 32-element group, no 64-bit division per thread.
+__global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                               int64_t K, uint8_t* __restrict__ codes,
+                                                               uint8_t* __restrict__ scales,
+                                                               const int32_t* __restrict__ rowmap, int k) {
+  const int part = int(threadIdx.x & 3);
+  const int64_t col8 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // 8-element chunk of the row
+  const bool active = col8 < K / 8;                                     // whole 4-thread groups
+  for (int64_t row = blockIdx.y; row < rows; row += gridDim.y) {
+    const int64_t gi = row * (K / 32) + (col8 >> 2);
+    float v[8];
+    float amax = 0.f;
+    bool bad = false;
+    if (active) {
+      const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
+      const uint4 raw = *reinterpret_cast<const uint4*>(x + src * K + col8 * 8);
+      const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = bf16_bits_to_float(rw[i] & 0xFFFFu);
-      v[2 * i + 1] = bf16_bits_to_float(rw[i] >> 16);
-    }
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = bf16_bits_to_float(rw[i] & 0xFFFFu);
+        v[2 * i + 1] = bf16_bits_to_float(rw[i] >> 16);
+      }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      bad |= !isfinite(v[i]);
-      amax = fmaxf(amax, isfinite(v[i]) ? fabsf(v[i]) : 0.f);
+      for (int i = 0; i < 8; ++i) {
+        bad |= !isfinite(v[i]);
+        amax = fmaxf(amax, isfinite(v[i]) ? fabsf(v[i]) : 0.f);
+      }
     }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const unsigned badmask = __ballot_sync(0xffffffffu, bad);
+    if (!active) continue;
+    const bool gbad = (badmask >> (threadIdx.x & 28)) & 0xFu;
+    int e = mx_scale_exponent(amax, 0x600000u, 8);  // limit 448 = 1.75 * 2^8
+    uint32_t lo = 0u, hi = 0u;
+    if (gbad) {
+      e = 255;
+      lo = hi = 0x7F7F7F7Fu;
+    } else {
+      const float f = pow2_float(127 - e);
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const __nv_fp8x2_storage_t pr =
+            __nv_cvt_float2_to_fp8x2(make_float2(v[i] * f, v[i + 1] * f), __NV_SATFINITE, __NV_E4M3);
+        uint32_t c0 = pr & 0xFFu, c1 = (pr >> 8) & 0xFFu;
+        // zero results carry the sign of the input
+        if ((c0 & 0x7Fu) == 0u) c0 = (__float_as_uint(v[i]) >> 31) << 7;
+        if ((c1 & 0x7Fu) == 0u) c1 = (__float_as_uint(v[i + 1]) >> 31) << 7;
+        const uint32_t pair = c0 | (c1 << 8);
+        if (i < 4) lo |= pair << (8 * i); else hi |= pair << (8 * (i - 4));
+      }
+    }
+    *reinterpret_cast<uint2*>(codes + gi * 32 + part * 8) = make_uint2(lo, hi);
+    if (part == 0) scales[gi] = uint8_t(e);
   }
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  const unsigned badmask = __ballot_sync(0xffffffffu, bad);
-  if (!active) return;
-  const bool gbad = (badmask >> (threadIdx.x & 28)) & 0xFu;
-  int e = mx_scale_exponent(amax, 0x600000u, 8);  // limit 448 = 1.75 * 2^8
-  uint32_t lo = 0u, hi = 0u;
-  if (gbad) {
-    e = 255;
-    lo = hi = 0x7F7F7F7Fu;
-  } else {
-    const float f = pow2_float(127 - e);
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      const __nv_fp8x2_storage_t pr =
-          __nv_cvt_float2_to_fp8x2(make_float2(v[i] * f, v[i + 1] * f), __NV_SATFINITE, __NV_E4M3);
-      uint32_t c0 = pr & 0xFFu, c1 = (pr >> 8) & 0xFFu;
-      // zero results carry the sign of the input
-      if ((c0 & 0x7Fu) == 0u) c0 = (__float_as_uint(v[i]) >> 31) << 7;
-      if ((c1 & 0x7Fu) == 0u) c1 = (__float_as_uint(v[i + 1]) >> 31) << 7;
-      const uint32_t pair = c0 | (c1 << 8);
-      if (i < 4) lo |= pair << (8 * i); else hi |= pair << (8 * (i - 4));
-    }
-  }
-  *reinterpret_cast<uint2*>(codes + gi * 32 + part * 8) = make_uint2(lo, hi);
-  if (part == 0) scales[gi] = uint8_t(e);
+}
+
+dim3 quant_grid(int64_t rows, int64_t K) {
+  return dim3(unsigned(ceil_div<int64_t>(K / 8, 256)), unsigned(rows < 65535 ? rows : 65535));
 }
 
 }  // namespace
@@ -300,8 +307,7 @@ stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K,
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
-  mxfp8_quant_bf16_kernel<<<unsigned(ceil_div<int64_t>(threads, 256)), 256, 0, s>>>(x, rows, K, codes, scales,
-                                                                                   nullptr, 1);
+  mxfp8_quant_bf16_kernel<<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1);
   return stq_launch_status();
 }
 
@@ -310,8 +316,7 @@ stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
-  mxfp8_quant_bf16_kernel<<<unsigned(ceil_div<int64_t>(threads, 256)), 256, 0, s>>>(x, rows, K, codes, scales,
-                                                                                   rowmap, k);
+  mxfp8_quant_bf16_kernel<<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k);
   return stq_launch_status();
 }
 
