@@ -47,7 +47,10 @@ NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense
 # capture of the same kernel build on a smaller case (named profile under profiles/); a
 # launch's traffic grows with its touched experts, so the full launch's traffic is this
 # figure times its touched experts.  An entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_EXPERT = {}
+MEASURED_TRAFFIC_PER_EXPERT = {
+    # profiles/w4a8_gemm_decode_mx_64experts.md: 63 touched, 858,358,528 B read + 4,408,832 B written
+    "gate_up_mx": (858_358_528 + 4_408_832) / 63,
+}
 
 
 def peaks():
@@ -582,7 +585,7 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append(cb["value"])
     value = statistics.mean(vals)
-    out = {"impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": 0,
+    out = {"impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": wl.name},
            "cpu_baseline": {"value": value, "unit": wl.unit, "cores": cb["cores"], "kind": "oracle",
