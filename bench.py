@@ -394,6 +394,24 @@ def e2e_steps(wl, steps, warmup):
     return start.elapsed_time(stop), xs.numel() * xs.element_size(), hy.numel() * hy.element_size()
 
 
+def max_over_ranks(values, device, dist):
+    """Element-wise maximum of per-rank timings over all ranks (every rank calls this in
+    the same order); identity on one process."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(n_ranks, units_per_rank_step, ms_per_step):
+    """Units per second of the whole job: every rank processes its own units per step."""
+    return n_ranks * units_per_rank_step / (ms_per_step * 1e-3)
+
+
+def base_config(wl):
+    return {"workload": wl.name, "experts": E, "tokens_per_step": wl.tokens_per_step()}
+
+
 def run_ours(args):
     dist = int(os.environ.get("WORLD_SIZE", "1")) > 1
     rank = int(os.environ.get("RANK", "0"))
@@ -414,12 +432,10 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         ms = timed_replays(graphs, args.steps, args.warmup, dist)
     clocks = clk.summary()
-    ms_t = torch.tensor([ms], device=dev)
-    if dist:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_step = float(ms_t.item()) / args.steps
+    ms_step = max_over_ranks([ms], dev, dist)[0] / args.steps
     kt = kernel_times(S, wl, args.steps, args.warmup)
     e2e_ms, h2d, d2h = e2e_steps(wl, args.steps, args.warmup)
+    e2e_ms = max_over_ranks([e2e_ms], dev, dist)[0]
     acct = [wl.accounting(args.warmup + i) for i in range(min(args.steps, N_BATCHES))]
     ab = float(np.mean([a["bytes"] for a in acct]))
     pk = peaks()
@@ -448,11 +464,11 @@ def run_ours(args):
         roof["traffic_source"] = "ncu dram bytes per touched expert (smaller case) x touched experts per launch"
     tps = wl.tokens_per_step()
     if wl.unit == "GB/s":
-        value = n * ab / (ms_step * 1e-3) / 1e9
-        e2e_val = n * ab / (e2e_ms / args.steps * 1e-3) / 1e9
+        value = whole_job_rate(n, ab, ms_step) / 1e9
+        e2e_val = whole_job_rate(n, ab, e2e_ms / args.steps) / 1e9
     else:
-        value = n * tps / (ms_step * 1e-3)
-        e2e_val = n * tps / (e2e_ms / args.steps * 1e-3)
+        value = whole_job_rate(n, tps, ms_step)
+        e2e_val = whole_job_rate(n, tps, e2e_ms / args.steps)
     out = {
         "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -460,7 +476,7 @@ def run_ours(args):
         "dtype": "bf16 x bf16 (STQ1_0 patterns x activations) and e2m1 x e4m3 (MXFP4 x MXFP8) "
                  "tensor-core products, fp32 accumulate",
         "data": "synthetic (seeded generators; random weights on the format grids)",
-        "config": {"workload": wl.name, "experts": E, "tokens_per_step": tps, "hbm_bytes_per_step": ab,
+        "config": {**base_config(wl), "hbm_bytes_per_step": ab,
                    "touched_experts_per_layer": getattr(wl, "_acct", {}).get((args.warmup) % N_BATCHES),
                    "tflop_per_step": acct[0]["flops"] / 1e12,
                    "l2": "inputs larger than L2: per-step weights exceed L2, batches rotate over 8",
@@ -587,7 +603,7 @@ def run_reference(args):
     value = statistics.mean(vals)
     out = {"impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": wl.name},
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": base_config(wl),
            "cpu_baseline": {"value": value, "unit": wl.unit, "cores": cb["cores"], "kind": "oracle",
                             "sample": cb["sample"]},
            "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
