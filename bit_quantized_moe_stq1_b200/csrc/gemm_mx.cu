@@ -346,13 +346,13 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
             if (col >= I.cnt) break;
             const float g = gate ? __uint_as_float(v[j]) : other[lane * 9 + j];
             const float u = gate ? other[lane * 9 + j] : __uint_as_float(v[8 + j]);
-            const float h = silu_f32(g) * u;
+            const float h = g / (1.0f + __expf(-g)) * u;  // silu(g) * u
             const bool bad = !isfinite(h);
-            float a = bad ? 0.f : fabsf(h);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            // amax over the 32 features of this column: the bits of a non-negative float
+            // order like the float, so one integer max reduction suffices
+            const uint32_t amax_bits = __reduce_max_sync(0xffffffffu, bad ? 0u : (__float_as_uint(h) & 0x7FFFFFFFu));
             const bool anybad = __any_sync(0xffffffffu, bad);
-            const int ex = anybad ? 255 : mx_scale_exponent(a, 0x600000u, 8);
+            const int ex = anybad ? 255 : mx_scale_exponent(__uint_as_float(amax_bits), 0x600000u, 8);
             const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2_float(127 - ex));
             const size_t pos = size_t(I.pos0 + col);
             p.hq[pos * p.R + f] = uint8_t(code);
