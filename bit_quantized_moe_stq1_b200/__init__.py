@@ -60,6 +60,7 @@ SIGNATURES = {
                                   _vp, _vp, _sz, _vp]),
     "moe_get_device_error": (_i32, [_vp, _vp]),
     "stq_set_timing": (_i32, [_vp]),
+    "stq_wait_selftest": (_i32, [_vp, _vp]),
     "stq_rmsnorm_bf16": (_i32, [_vp, _i64, _i64, ctypes.c_float, _vp, _vp]),
 }
 
@@ -210,6 +211,11 @@ def rmsnorm_bf16(x, eps=1e-6, y=None, stream=None):
     _check(lib.stq_rmsnorm_bf16(_ptr(x), x.shape[0], x.shape[1], float(eps), _ptr(y), _stream(stream)),
            "stq_rmsnorm_bf16")
     return y
+
+
+def wait_selftest(err, stream=None):
+    """Run the bounded-wait self-test (about two seconds); *err then holds STQ_ERR_TIMEOUT."""
+    _check(lib.stq_wait_selftest(_ptr(err), _stream(stream)), "stq_wait_selftest")
 
 
 def read_error(err, stream=None):

@@ -383,6 +383,18 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
   }
 }
 
+// A barrier nothing arrives at, waited on through the kernels' bounded wait.
+__global__ void wait_selftest_kernel(int32_t* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) tc::mbar_wait(&bar, 0, err);
+  __syncthreads();
+}
+
 // N tiles of every touched expert: (expert, first token of the tile); one CTA.
 __global__ void __launch_bounds__(1024) mx_plan_kernel(const int32_t* __restrict__ counts, int E, int nt,
                                                        int2* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
@@ -559,4 +571,10 @@ extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales,
   p.max_items = int(items);
   StqTimed tm(STQ_K_GEMM, s);
   return launch_nt<false>(nt, ma, ma, mb, p, s);
+}
+
+extern "C" stq_status stq_wait_selftest(int32_t* err, stq_stream_t stream) {
+  STQ_HOST_CHECK(err != nullptr, STQ_ERR_INVALID_ARG);
+  wait_selftest_kernel<<<1, 32, 0, stq_cuda_stream(stream)>>>(err);
+  return stq_launch_status();
 }

@@ -266,6 +266,13 @@ stq_status stq_rmsnorm_bf16(const uint16_t* x, int64_t T, int64_t H, float eps,
 /* Instrumentation (no counterpart on the pages).                             */
 /* ------------------------------------------------------------------------- */
 
+/* Self-test of the bounded waits: one CTA waits, through the same bounded mbarrier
+ * wait the tensor-core kernels use, on a barrier that nothing arrives at.  After the
+ * limit (about two seconds of GPU clock) the wait gives up, STQ_ERR_TIMEOUT is recorded
+ * in *err (device int32, caller-owned; first error wins) and the kernel returns, so the
+ * context stays usable.  Asynchronous on `stream`. */
+stq_status stq_wait_selftest(int32_t* err, stq_stream_t stream);
+
 /* Kernel kinds reported by the timing hook. */
 enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM,

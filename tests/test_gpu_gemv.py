@@ -64,3 +64,17 @@ def test_stq1_gemv_special_cases(S):
     z = S.stq1_pack(torch.zeros((16, 256), device=DEV))
     assert torch.all(S.stq1_gemv(z, 16, 256, x[:, :256].contiguous()) == 0)
     assert S.stq1_gemv(pk, rows, K, x[:0]).numel() == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(S):
+    """A wait that nothing satisfies runs out (about two seconds), records STQ_ERR_TIMEOUT
+    and returns; the context then runs a GEMV as before."""
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    S.wait_selftest(err)
+    assert S.read_error(err) == -8
+    w = W.stq_grid_weights(32, 256, DEV, 0, "wait")
+    x = W.bf16_normal((1, 256), 1.0, DEV, 0, "waitx")
+    packed = S.stq1_pack(w)
+    y = S.stq1_gemv(packed, 32, 256, x).cpu().double().numpy()
+    yr, sr = M.stq1_gemv(packed.cpu().numpy(), 32, 256, x.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+    assert np.all(np.abs(y - yr) <= 1e-3 * sr + 1e-5)
