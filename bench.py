@@ -47,10 +47,7 @@ NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense
 # capture of the same kernel build on a smaller case (named profile under profiles/); a
 # launch's traffic grows with its touched experts, so the full launch's traffic is this
 # figure times its touched experts.  An entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_EXPERT = {
-    # profiles/w4a8_gemm_decode_mx_64experts.md: 63 touched, 858,358,528 B read + 4,408,832 B written
-    "gate_up_mx": (858_358_528 + 4_408_832) / 63,
-}
+MEASURED_TRAFFIC_PER_EXPERT = {}
 
 
 def peaks():

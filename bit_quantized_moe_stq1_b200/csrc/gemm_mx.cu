@@ -210,17 +210,24 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
     int last_round[C::kStages];
 #pragma unroll
     for (int s = 0; s < C::kStages; ++s) last_round[s] = -1;
+    // When nk is a multiple of the ring (2 kPf steps), the last steps of an item read the
+    // next item's first scale factors into the ring, so an item boundary costs no wait.
+    const bool cross = nk % (2 * kPf) == 0;
     bool ok = true;
+    uint32_t ra[kPf][4], rb[kPf][4];
     for (int it = 0; ok; ++it) {
       const Item I = get_item<NT>(p, blockIdx.x + it * G, MT, C::kRowsPerTile);
       if (!I.valid) break;
+      Item In{};
+      if (cross) In = get_item<NT>(p, blockIdx.x + (it + 1) * G, MT, C::kRowsPerTile);
       const int kt0 = ((pid - it * nk) % 2 + 2) % 2;  // first k-step of this item for this producer
-      uint32_t ra[kPf][4], rb[kPf][4];
+      if (!cross || it == 0) {
 #pragma unroll
-      for (int d = 0; d < kPf; ++d) {
-        if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt0 + 2 * d, nk, lane);
-        else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt0 + 2 * d, nk, lane);
-        load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt0 + 2 * d, nk, lane);
+        for (int d = 0; d < kPf; ++d) {
+          if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt0 + 2 * d, nk, lane);
+          else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt0 + 2 * d, nk, lane);
+          load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt0 + 2 * d, nk, lane);
+        }
       }
       for (int k0 = kt0; k0 < nk && ok; k0 += 2 * kPf) {
 #pragma unroll
@@ -249,9 +256,13 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
             tc::tma_load_2d(st + C::kOffB, &tmB, kt * kKT, I.brow, &full[s]);
           }
           last_round[s] = r;
-          if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt + 2 * kPf, nk, lane);
-          else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt + 2 * kPf, nk, lane);
-          load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt + 2 * kPf, nk, lane);
+          const int kn = kt + 2 * kPf;
+          const Item& J = (cross && kn >= nk) ? In : I;  // In.valid is false past the last item
+          const int kj = (cross && kn >= nk) ? kn - nk : kn;
+          const int nkj = J.valid ? nk : 0;               // an invalid item reads zeros
+          if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, J.arow, k32, kj, nkj, lane);
+          else load_sf(ra[d], p.sa, J.arow, 128, 0x7fffffff, k32, kj, nkj, lane);
+          load_sf(rb[d], p.sb, J.brow, NT, p.Ptot, k32, kj, nkj, lane);
         }
       }
     }
