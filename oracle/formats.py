@@ -323,6 +323,72 @@ def stq1_codes_from_float(w):
     return code.astype(np.int64), dbits
 
 
+STQ_LS_ROUNDS = 3
+
+
+def stq1_codes_ls(w, importance=None, rounds=STQ_LS_ROUNDS):
+    """Least-squares STQ1_0 encoder ("Hy4-preview-GGUF", section 3, "Our encoder"):
+    the byte format is unchanged, two decisions differ from the upstream rule.
+
+    Per 256-block of a row, with importance v_k >= 0 per column (None: all 1):
+      start from the upstream scale d = amax |w|; then, `rounds` times,
+      1. per group of four, the zero goes to the lane j minimising the incremental
+         cost v_j * (w_j^2 - (|w_j| - d)^2) (first lane on ties), with the current d;
+      2. d = sum(v * sel * w) / sum(v * sel^2) over the block, sel = sign(w) on the
+         three kept lanes and 0 on the zero lane (0 when the denominator is 0).
+    Reading: "alternating for 3 rounds" is taken as three (placement, scale) rounds
+    after the upstream start; the stored d is the last scale rounded to FP16, the
+    codes are the last placement with the kept lanes' signs.  All arithmetic is
+    float64, each cost evaluated as v * (w*w - (|w|-d)*(|w|-d)) in that order.
+    Returns (codes [rows, K/256, 64] int64, d bits [rows, K/256] uint16)."""
+    w = np.asarray(w, dtype=np.float32).astype(np.float64)
+    rows, K = w.shape
+    if K % STQ_BLOCK:
+        raise ValueError("K must be a multiple of 256")
+    if not np.all(np.isfinite(w)):
+        raise NonFiniteError("non-finite weight")
+    v = np.ones(K) if importance is None else np.asarray(importance, dtype=np.float32).astype(np.float64)
+    if v.shape != (K,) or not np.all(np.isfinite(v)) or np.any(v < 0):
+        raise ValueError("importance must be K finite non-negative values")
+    nb = K // STQ_BLOCK
+    x = w.reshape(rows, nb, 64, 4)
+    vg = np.broadcast_to(v.reshape(nb, 64, 4), x.shape)
+    ax = np.abs(x)
+    d = np.max(ax.reshape(rows, nb, STQ_BLOCK), axis=2)
+    if np.any(d > 65504.0):
+        raise NonFiniteError("block amax above the FP16 range")
+    z = np.zeros(x.shape[:3], dtype=np.int64)
+    for _ in range(rounds):
+        e = ax - d[:, :, None, None]
+        cost = vg * (x * x - e * e)
+        z = np.argmin(cost, axis=3)                         # first minimum
+        keep = np.ones(x.shape, dtype=bool)
+        np.put_along_axis(keep, z[..., None], False, axis=3)
+        num = np.sum(np.where(keep, vg * ax, 0.0), axis=(2, 3))
+        den = np.sum(np.where(keep, vg, 0.0), axis=(2, 3))
+        d = np.where(den > 0, num / np.where(den > 0, den, 1.0), 0.0)
+    dbits = fp16_encode_rne(d)
+    neg = np.signbit(x).astype(np.int64)
+    sbits = np.take_along_axis(neg, _NZ_LANES[z], axis=3)
+    code = 8 * z + sbits[..., 0] + 2 * sbits[..., 1] + 4 * sbits[..., 2]
+    code = np.where((fp16_decode(dbits) == 0)[:, :, None], 0, code)
+    return code.astype(np.int64), dbits
+
+
+def stq1_pack_ls(w, importance=None):
+    """float32 weights [rows, K] -> STQ1_0 bytes with the least-squares encoder."""
+    code, dbits = stq1_codes_ls(w, importance)
+    return stq1_layout(code, dbits)
+
+
+def stq1_weighted_ssd(w, packed, importance=None):
+    """sum_k v_k (w_k - w_hat_k)^2 of a packed matrix against its float source."""
+    w = np.asarray(w, dtype=np.float32).astype(np.float64)
+    rows, K = w.shape
+    v = np.ones(K) if importance is None else np.asarray(importance, dtype=np.float32).astype(np.float64)
+    return float(np.sum(v[None, :] * (w - stq1_unpack(packed, rows, K)) ** 2))
+
+
 def stq1_layout(code, dbits):
     """Codes [rows, K/256, 64] and d bits [rows, K/256] -> packed bytes."""
     rows, nb = dbits.shape

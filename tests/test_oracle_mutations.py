@@ -100,3 +100,46 @@ def test_rms_norm_mistakes_are_caught(monkeypatch, mistake):
 
     monkeypatch.setattr(M, "rms_norm", wrong)
     _fails(TM.test_rms_norm_closed_forms)
+
+
+@pytest.mark.parametrize("mistake", ["argmax", "unweighted_scale", "magnitude_zero"])
+def test_ls_encoder_mistakes_are_caught(monkeypatch, mistake):
+    import test_oracle_encoder as TE
+    orig_argmin, orig_sum = np.argmin, np.sum
+
+    def codes(w, importance=None, rounds=F.STQ_LS_ROUNDS):
+        w = np.asarray(w, dtype=np.float32).astype(np.float64)
+        rows, K = w.shape
+        v = np.ones(K) if importance is None else np.asarray(importance, np.float32).astype(np.float64)
+        nb = K // 256
+        x = w.reshape(rows, nb, 64, 4)
+        vg = np.broadcast_to(v.reshape(nb, 64, 4), x.shape)
+        ax = np.abs(x)
+        d = np.max(ax.reshape(rows, nb, 256), axis=2)
+        for _ in range(rounds):
+            e = ax - d[:, :, None, None]
+            cost = vg * (x * x - e * e)
+            if mistake == "argmax":
+                z = np.argmax(cost, axis=3)
+            elif mistake == "magnitude_zero":
+                z = np.argmin(ax, axis=3)
+            else:
+                z = np.argmin(cost, axis=3)
+            keep = np.ones(x.shape, dtype=bool)
+            np.put_along_axis(keep, z[..., None], False, axis=3)
+            wt = np.ones_like(vg) if mistake == "unweighted_scale" else vg
+            num = np.sum(np.where(keep, wt * ax, 0.0), axis=(2, 3))
+            den = np.sum(np.where(keep, wt, 0.0), axis=(2, 3))
+            d = np.where(den > 0, num / np.where(den > 0, den, 1.0), 0.0)
+        dbits = F.fp16_encode_rne(d)
+        neg = np.signbit(x).astype(np.int64)
+        sb = np.take_along_axis(neg, F._NZ_LANES[z], axis=3)
+        code = 8 * z + sb[..., 0] + 2 * sb[..., 1] + 4 * sb[..., 2]
+        code = np.where((F.fp16_decode(dbits) == 0)[:, :, None], 0, code)
+        return code.astype(np.int64), dbits
+
+    monkeypatch.setattr(F, "stq1_codes_ls", codes)
+    with pytest.raises(AssertionError):
+        TE.test_importance_moves_the_zero_hand_example()
+        TE.test_importance_weights_the_scale_hand_example()
+        TE.test_uniform_importance_is_argmin_and_mean_of_kept()
