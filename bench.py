@@ -114,6 +114,8 @@ class Workload:
     unit = "tokens/s"
     metric = "MoE-layer tokens/s"
     bound = "hbm"
+    dtype = ("bf16 x bf16 (STQ1_0 patterns x activations) and e2m1 x e4m3 (MXFP4 x MXFP8) "
+             "tensor-core products, fp32 accumulate")
 
     def tokens_per_step(self):
         return self.T
@@ -181,6 +183,34 @@ class W4A8Gemm(Workload):
 
     def h2d_d2h(self):
         return self.T * H * 2, self.T * I * 4
+
+
+class StqPackLs(Workload):
+    """The least-squares STQ1_0 encoder over one 2048 x 6144 float32 expert matrix with
+    per-column importance weights exp(N(0,1)); 8 rotating matrices (400 MB > L2)."""
+
+    name = "stq_pack_ls"
+    unit = "GB/s"
+    dtype = "f32 weights in, f64 decisions, u8 out"
+    metric = "STQ1_0 least-squares encoder GB/s (2048x6144 float32 in, packed out)"
+
+    def __init__(self, S, dev):
+        self.S, self.dev, self.T = S, dev, 1
+        self.Wf = [W.float_normal((I, H), 0.02, dev, 0, "pls", b) for b in range(N_BATCHES)]
+        self.x = self.Wf   # the step's input (end-to-end timing copies it from the host)
+        self.v = torch.exp(W.float_normal((H,), 1.0, dev, 0, "plsv")).contiguous()
+        self.out = torch.empty(STQ_MAT, dtype=torch.uint8, device=dev)
+        self.bytes = I * H * 4 + H * 4 + STQ_MAT
+
+    def step(self, i, x=None, y=None):
+        return self.S.stq1_pack_ls(self.Wf[i % N_BATCHES] if x is None else x, self.v,
+                                   out=self.out if y is None else y)
+
+    def accounting(self, i):
+        return dict(bytes=self.bytes, flops=0, per_kind={"pack_ls": dict(bytes=self.bytes)})
+
+    def h2d_d2h(self):
+        return I * H * 4, STQ_MAT
 
 
 class MoeLayers(Workload):
@@ -303,6 +333,8 @@ def make_workload(name, S, dev, experts=256):
         return StqMatvec(S, dev)
     if name == "w4a8_gemm":
         return W4A8Gemm(S, dev)
+    if name == "stq_pack_ls":
+        return StqPackLs(S, dev)
     if name == "decode_mx":
         # one MXFP4 layer of the stacked workload (a small case for profiler captures)
         return MoeLayers(S, dev, name, 32, ("mx",), True, True, True, experts)
@@ -310,7 +342,7 @@ def make_workload(name, S, dev, experts=256):
     return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual, experts)
 
 
-WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "stacked_decode", "decode_mx"]
+WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "stacked_decode", "decode_mx", "stq_pack_ls"]
 
 
 # ----------------------------------------------------------------------------- measurement
@@ -470,8 +502,7 @@ def run_ours(args):
         "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 x bf16 (STQ1_0 patterns x activations) and e2m1 x e4m3 (MXFP4 x MXFP8) "
-                 "tensor-core products, fp32 accumulate",
+        "dtype": wl.dtype,
         "data": "synthetic (seeded generators; random weights on the format grids)",
         "config": {**base_config(wl), "hbm_bytes_per_step": ab,
                    "touched_experts_per_layer": getattr(wl, "_acct", {}).get((args.warmup) % N_BATCHES),
@@ -509,6 +540,13 @@ def _oracle_units(wl, dev):
         t0 = time.perf_counter()
         M.stq1_gemv(Wb, I, H, xb)
         return time.perf_counter() - t0, 1.0, "one full matvec (unpack + float64 matvec)"
+    if wl.name == "stq_pack_ls":
+        rows = 128
+        wf = wl.Wf[0][:rows].cpu().numpy()
+        v = wl.v.cpu().numpy()
+        t0 = time.perf_counter()
+        F.stq1_pack_ls(wf, v)
+        return (time.perf_counter() - t0) * (I / rows), 1.0, f"{rows} of the {I} rows, scaled to the matrix"
     if wl.name == "w4a8_gemm":
         c, sc = wl.Wt[0]
         xb = wl.x[0][:16].view(torch.int16).cpu().numpy().view(np.uint16)

@@ -45,6 +45,7 @@ SIGNATURES = {
     "stq_read_error": (_i32, [_vp, _vp]),
     "stq1_pack": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "stq1_unpack": (_i32, [_vp, _i64, _i64, _vp, _vp]),
+    "stq1_pack_ls": (_i32, [_vp, _vp, _i64, _i64, _vp, _vp, _vp]),
     "mxfp4_pack": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "mxfp4_unpack": (_i32, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "mxfp8_quantize_bf16": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
@@ -66,7 +67,8 @@ SIGNATURES = {
 
 
 KERNEL_KINDS = ["router_logits", "router_topk", "permute", "quant_x", "gate_up", "down", "combine", "gemv", "gemm",
-                "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down", "rmsnorm"]
+                "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down", "rmsnorm",
+                "pack_ls"]
 
 
 class StqTiming(ctypes.Structure):
@@ -160,6 +162,21 @@ def stq1_pack(w, out=None, err=None, stream=None):
     if out is None:
         out = torch.empty(stq1_packed_bytes(rows, K), dtype=torch.uint8, device=w.device)
     _check(lib.stq1_pack(_ptr(w), rows, K, _ptr(out), _ptr(err), _stream(stream)), "stq1_pack")
+    return out
+
+
+def stq1_pack_ls(w, importance=None, out=None, err=None, stream=None):
+    """float32 [rows, K] -> STQ1_0 bytes by the least-squares encoder; importance:
+    float32 [K] column weights (None = all 1)."""
+    _dev(w)
+    assert w.dtype == torch.float32 and w.dim() == 2
+    rows, K = w.shape
+    if importance is not None:
+        assert importance.dtype == torch.float32 and importance.shape == (K,) and importance.is_contiguous()
+    if out is None:
+        out = torch.empty(stq1_packed_bytes(rows, K), dtype=torch.uint8, device=w.device)
+    imp = _ptr(importance) if importance is not None else None
+    _check(lib.stq1_pack_ls(_ptr(w), imp, rows, K, _ptr(out), _ptr(err), _stream(stream)), "stq1_pack_ls")
     return out
 
 

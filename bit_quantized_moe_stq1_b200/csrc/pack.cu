@@ -84,6 +84,118 @@ __global__ void stq1_pack_kernel(const float* __restrict__ w, int64_t rows, int6
   reinterpret_cast<uint32_t*>(ob + 544)[lane] = words[4];
 }
 
+// ----------------------------------------------------------------------------- STQ1_0, least squares
+
+// Incremental cost of zeroing a lane, v * (x*x - (|x| - d)^2), in FP64 in that order
+// (explicit roundings: no fused multiply-adds, so every decision is reproducible).
+__device__ __forceinline__ double ls_cost(float x, float v, double d) {
+  const double ax = fabs(double(x));
+  const double e = __dsub_rn(ax, d);
+  return __dmul_rn(double(v), __dsub_rn(__dmul_rn(double(x), double(x)), __dmul_rn(e, e)));
+}
+
+// Lane of least cost in a group (first on ties).
+__device__ __forceinline__ uint32_t ls_zero_lane(float4 x, float4 v, double d) {
+  const double c[4] = {ls_cost(x.x, v.x, d), ls_cost(x.y, v.y, d), ls_cost(x.z, v.z, d), ls_cost(x.w, v.w, d)};
+  uint32_t z = 0;
+#pragma unroll
+  for (int l = 1; l < 4; ++l)
+    if (c[l] < c[z]) z = uint32_t(l);
+  return z;
+}
+
+// Least-squares encoder ("Hy4-preview-GGUF", section 3, "Our encoder"): from the upstream
+// scale d = amax, three rounds of (zero placement by least incremental cost at the
+// current d, then d = sum(v |x|) / sum(v) over the kept lanes).  One warp per tile-block
+// as stq1_pack_kernel.  Decisions: lane (row r = lane & 15, half = lane >> 4) owns 32
+// groups of row r; the row's sums are FP64, its two halves added by one shuffle.
+// Codes: lane (g, t) places its groups again with the scale of the last round's
+// placement (the same decision, same arithmetic) and writes the layout.
+__global__ void stq1_pack_ls_kernel(const float* __restrict__ w, const float* __restrict__ imp, int64_t rows,
+                                    int64_t K, uint8_t* __restrict__ out, int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nb = K / 256;
+  if (warp >= (rows / 16) * nb) return;
+  const int64_t tile = warp / nb, b = warp % nb;
+  const float* base = w + tile * 16 * K + b * 256;
+  const float4 one4 = make_float4(1.f, 1.f, 1.f, 1.f);
+  const float4* ib = imp != nullptr ? reinterpret_cast<const float4*>(imp + b * 256) : nullptr;
+
+  const int r = lane & 15, half = lane >> 4;
+  const float4* p = reinterpret_cast<const float4*>(base + r * K + half * 128);
+  float amax = 0.f;
+  bool bad = false, badv = false;
+  for (int i = 0; i < 32; ++i) {
+    const float4 x = p[i];
+    const float4 v = ib != nullptr ? ib[half * 32 + i] : one4;
+    bad |= !isfinite(x.x) || !isfinite(x.y) || !isfinite(x.z) || !isfinite(x.w);
+    badv |= !(v.x >= 0.f && v.y >= 0.f && v.z >= 0.f && v.w >= 0.f) || !isfinite(v.x) || !isfinite(v.y) ||
+            !isfinite(v.z) || !isfinite(v.w);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
+  bad = __any_sync(0xffffffffu, bad || amax > 65504.f);
+  badv = __any_sync(0xffffffffu, badv);
+  if (lane == 0) {
+    if (bad) stq_set_error(err, STQ_ERR_NONFINITE);
+    if (badv) stq_set_error(err, STQ_ERR_INVALID_ARG);
+  }
+  double d = double(amax), d_place = d;
+  for (int round = 0; round < 3; ++round) {
+    d_place = d;
+    double num = 0.0, den = 0.0;
+    for (int i = 0; i < 32; ++i) {
+      const float4 x = p[i];
+      const float4 v = ib != nullptr ? ib[half * 32 + i] : one4;
+      const uint32_t z = ls_zero_lane(x, v, d_place);
+      const float xs[4] = {x.x, x.y, x.z, x.w}, vs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int l = 0; l < 4; ++l)
+        if (uint32_t(l) != z) {
+          num = __dadd_rn(num, __dmul_rn(double(vs[l]), fabs(double(xs[l]))));
+          den = __dadd_rn(den, double(vs[l]));
+        }
+    }
+    num = __dadd_rn(num, __shfl_xor_sync(0xffffffffu, num, 16));
+    den = __dadd_rn(den, __shfl_xor_sync(0xffffffffu, den, 16));
+    d = den > 0.0 ? __ddiv_rn(num, den) : 0.0;
+  }
+  const uint32_t dbits = __half_as_ushort(__double2half(d));  // lanes r and r + 16 hold row r's scale
+
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t d_lo = __shfl_sync(0xffffffffu, dbits, g);
+  const uint32_t d_hi = __shfl_sync(0xffffffffu, dbits, g + 8);
+  const double dp_lo = __shfl_sync(0xffffffffu, d_place, g);
+  const double dp_hi = __shfl_sync(0xffffffffu, d_place, g + 8);
+  uint32_t words[5] = {0u, 0u, 0u, 0u, 0u};
+  for (int s = 0; s < 16; ++s) {
+    const float4 v = ib != nullptr ? ib[16 * t + s] : one4;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = g + 8 * h;
+      const float4 x = *reinterpret_cast<const float4*>(base + row * K + 4 * (16 * t + s));
+      const uint32_t z = ls_zero_lane(x, v, h ? dp_hi : dp_lo);
+      const uint32_t neg[4] = {__float_as_uint(x.x) >> 31, __float_as_uint(x.y) >> 31, __float_as_uint(x.z) >> 31,
+                               __float_as_uint(x.w) >> 31};
+      uint32_t sb = 0, n = 0;
+#pragma unroll
+      for (int l = 0; l < 4; ++l)
+        if (uint32_t(l) != z) { sb |= neg[l] << n; ++n; }
+      uint32_t code = 8u * z + sb;
+      if ((h ? d_hi : d_lo) == 0u) code = 0u;
+      const int i = 2 * s + h, sh = 5 * i, w0 = sh >> 5, off = sh & 31;
+      words[w0] |= code << off;
+      if (off > 27) words[w0 + 1] |= code >> (32 - off);
+    }
+  }
+  uint8_t* ob = out + warp * kTileBlockBytes;
+  const uint32_t dpair = dbits | (__shfl_sync(0xffffffffu, dbits, (lane + 8) & 31) << 16);
+  if (lane < 8) reinterpret_cast<uint32_t*>(ob)[lane] = dpair;
+  reinterpret_cast<uint4*>(ob + 32)[lane] = make_uint4(words[0], words[1], words[2], words[3]);
+  reinterpret_cast<uint32_t*>(ob + 544)[lane] = words[4];
+}
+
 __global__ void stq1_unpack_kernel(const uint8_t* __restrict__ in, int64_t rows, int64_t K, float* __restrict__ w) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -262,6 +374,24 @@ extern "C" stq_status stq1_pack(const float* w, int64_t rows, int64_t K, uint8_t
   const int64_t warps = (rows / 16) * (K / 256);
   if (warps == 0) return STQ_OK;
   stq1_pack_kernel<<<unsigned(ceil_div<int64_t>(warps, 4)), 128, 0, stq_cuda_stream(stream)>>>(w, rows, K, out, err);
+  return stq_launch_status();
+}
+
+extern "C" stq_status stq1_pack_ls(const float* w, const float* importance, int64_t rows, int64_t K, uint8_t* out,
+                                   int32_t* err, stq_stream_t stream) {
+  STQ_HOST_CHECK(rows >= 0 && K >= 0, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(rows % 16 == 0 && K % 256 == 0, STQ_ERR_SHAPE);
+  if (rows == 0 || K == 0) return STQ_OK;  // nothing to read or write: pointers may be NULL
+  STQ_HOST_CHECK(w && out, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(stq_aligned16(w) && stq_aligned16(out) && (importance == nullptr || stq_aligned16(importance)),
+                 STQ_ERR_ALIGN);
+  const int64_t warps = (rows / 16) * (K / 256);
+  if (warps == 0) return STQ_OK;
+  {
+    StqTimed tm(STQ_K_PACK_LS, stq_cuda_stream(stream));
+    stq1_pack_ls_kernel<<<unsigned(ceil_div<int64_t>(warps, 4)), 128, 0, stq_cuda_stream(stream)>>>(
+        w, importance, rows, K, out, err);
+  }
   return stq_launch_status();
 }
 

@@ -93,6 +93,21 @@ stq_status stq_read_error(int32_t* err, stq_stream_t stream);
 stq_status stq1_pack(const float* w, int64_t rows, int64_t K, uint8_t* out,
                      int32_t* err, stq_stream_t stream);
 
+/* The same bytes from the least-squares encoder ("Hy4-preview-GGUF", section 3, "Our
+ * encoder"): per 256-block of a row, starting from d = max |w|, three rounds of
+ *   1. per group, the zero on the lane j of least v_j * (w_j^2 - (|w_j| - d)^2) (first
+ *      lane on ties), the other lanes keeping sign(w);
+ *   2. d = sum(v |w|) / sum(v) over the kept lanes (0 if that sum of v is 0);
+ * then d is stored as fp16_rne (d == 0: all codes 0).  v = importance[k] per column k
+ * (float32 [K], >= 0, e.g. an importance matrix's column weights; NULL = all 1).  The
+ * costs and sums are FP64 with explicit roundings, the scale rounded directly from FP64
+ * to FP16.  A NaN/Inf weight or a block amax > 65504 sets STQ_ERR_NONFINITE, a negative
+ * or non-finite importance STQ_ERR_INVALID_ARG, in *err (may be NULL).  Pointers are
+ * device pointers, 16-byte aligned; rows % 16 == 0, K % 256 == 0; rows == 0 or K == 0
+ * is a no-op (pointers may then be NULL). */
+stq_status stq1_pack_ls(const float* w, const float* importance, int64_t rows, int64_t K,
+                        uint8_t* out, int32_t* err, stq_stream_t stream);
+
 /* STQ1_0 bytes -> float32 [rows, K]: +-d on non-zero lanes (sign applied to d),
  * +0 on the zero lane.  Bit-exact. */
 stq_status stq1_unpack(const uint8_t* in, int64_t rows, int64_t K, float* w,
@@ -277,10 +292,11 @@ stq_status stq_wait_selftest(int32_t* err, stq_stream_t stream);
 enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM,
        STQ_K_GATE_UP_MX, STQ_K_DOWN_MX, STQ_K_PLAN, STQ_K_SHARED_GATE_UP, STQ_K_SHARED_DOWN,
-       STQ_K_RMSNORM, STQ_K_COUNT };
+       STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
- * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm and stq_rmsnorm_bf16 is bracketed by
+ * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm, stq_rmsnorm_bf16 and stq1_pack_ls is
+ * bracketed by
  * event records of events[2n] / events[2n+1] on the call's stream (inside stream
  * capture as external event-record nodes of the graph), kinds[n] is set to its
  * STQ_K_* kind and n = count++ (until capacity pairs are used).  events:

@@ -128,3 +128,36 @@ def test_mxfp8_quant_activation_workload(S):
     assert np.array_equal(c[:512].cpu().numpy(), rc) and np.array_equal(s[:512].cpu().numpy(), rs)
     rc2, rs2 = F.mxfp8_quantize(F.bf16_decode(xb[-7:]))
     assert np.array_equal(c[-7:].cpu().numpy(), rc2) and np.array_equal(s[-7:].cpu().numpy(), rs2)
+
+
+def _imp(K, tag):
+    return torch.exp(W.float_normal((K,), 1.0, DEV, 0, "imp", tag)).contiguous()
+
+
+@pytest.mark.parametrize("rows,K,dist,imp", [(16, 256, "normal", False), (32, 768, "normal", True),
+                                             (48, 512, "laplace", True), (16, 6144, "outlier", True),
+                                             (2048, 6144, "normal", True)])
+def test_stq1_pack_ls_bitexact(S, rows, K, dist, imp):
+    """The least-squares encoder's bytes equal the oracle's (FP64 decisions on both sides)."""
+    w = W.float_normal((rows, K), 0.02, DEV, 0, "ls", rows, K, dist)
+    if dist == "laplace":
+        w = w * torch.log(1.0 / W.float_normal((rows, K), 1.0, DEV, 0, "lsu", rows).abs().clamp_min(1e-3))
+    elif dist == "outlier":
+        w[:, ::97] *= 40.0
+    v = _imp(K, (rows, K)) if imp else None
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    got = S.stq1_pack_ls(w.contiguous(), v, err=err).cpu().numpy()
+    assert S.read_error(err) == 0
+    ref = F.stq1_pack_ls(w.cpu().numpy(), None if v is None else v.cpu().numpy())
+    assert np.array_equal(got, ref), int(np.count_nonzero(got != ref))
+
+
+def test_stq1_pack_ls_errors(S):
+    w = W.float_normal((16, 256), 0.02, DEV, 0, "lserr")
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    S.stq1_pack_ls(w, -torch.ones(256, device=DEV), err=err)
+    assert S.read_error(err) == -1
+    w[2, 7] = float("inf")
+    S.stq1_pack_ls(w, err=err)
+    assert S.read_error(err) == -4
+    assert S.stq1_pack_ls(w[:0]).numel() == 0
