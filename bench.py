@@ -314,8 +314,14 @@ class MoeLayers(Workload):
             if L["fmt"] == "stq":
                 gu = t * 2 * STQ_MAT + (2 * BF16_MAT if self.shared else 0) + T * H * 2 + (P + T) * I * 2
                 dn = t * STQ_MAT + (BF16_MAT if self.shared else 0) + (P + T) * I * 2 + (P + T) * H * 4
-                kinds.setdefault("gate_up", []).append(dict(bytes=gu))
-                kinds.setdefault("down", []).append(dict(bytes=dn))
+                kinds.setdefault("gate_up", []).append(dict(bytes=gu, flops=4 * P * I * H, touched=t))
+                kinds.setdefault("down", []).append(dict(bytes=dn, flops=2 * P * I * H, touched=t))
+                # prefill regime (tensor-core GEMM on MXFP8 activations): weights once, x and
+                # h as MXFP8 codes + scales
+                gu = t * 2 * STQ_MAT + P * H * (1 + 1 / 32) + P * I * (1 + 1 / 32)
+                dn = t * STQ_MAT + P * I * (1 + 1 / 32) + P * H * 4
+                kinds.setdefault("gate_up_stq_tc", []).append(dict(bytes=gu, flops=4 * P * I * H, touched=t))
+                kinds.setdefault("down_stq_tc", []).append(dict(bytes=dn, flops=2 * P * I * H, touched=t))
             else:
                 gu = t * 2 * MX_MAT + P * H * (1 + 1 / 32) + P * I * (1 + 1 / 32)
                 dn = t * MX_MAT + P * I * (1 + 1 / 32) + P * H * 4
@@ -342,7 +348,8 @@ def make_workload(name, S, dev, experts=256):
     return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual, experts)
 
 
-WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "stacked_decode", "decode_mx", "stq_pack_ls"]
+WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "prefill_stq", "stacked_decode", "decode_mx",
+                  "stq_pack_ls"]
 
 
 # ----------------------------------------------------------------------------- measurement
@@ -474,7 +481,8 @@ def run_ours(args):
     per = acct[0]["per_kind"].get(dom, {})
     launch_bytes = float(np.mean([a["per_kind"][dom]["bytes"] for a in acct if dom in a["per_kind"]])) if per else None
     launch_flops = float(np.mean([a["per_kind"][dom].get("flops", 0) for a in acct if dom in a["per_kind"]])) if per else 0
-    if wl.bound == "tensor" or dom in ("gate_up_mx", "down_mx") and wl.name == "prefill_w4a8":
+    if wl.bound == "tensor" or (dom in ("gate_up_mx", "down_mx") and wl.name == "prefill_w4a8") or \
+            dom in ("gate_up_stq_tc", "down_stq_tc"):
         peak = pk["bf16"] * NOMINAL_FP8_OVER_BF16
         achieved = launch_flops / (avg_ms * 1e-3) / 1e12 if launch_flops else None
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -487,7 +495,7 @@ def run_ours(args):
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                 "frac": achieved / pk["hbm"] if achieved else None, "peak_source": pk["src"] + " copy bandwidth",
                 "traffic": None, "bytes_per_launch": launch_bytes, "avg_launch_ms": avg_ms}
-    if dom in MEASURED_TRAFFIC_PER_EXPERT and wl.name != "prefill_w4a8" and per.get("touched"):
+    if dom in MEASURED_TRAFFIC_PER_EXPERT and wl.name not in ("prefill_w4a8", "prefill_stq") and per.get("touched"):
         touched = float(np.mean([a["per_kind"][dom]["touched"] for a in acct if dom in a["per_kind"]]))
         roof["traffic"] = MEASURED_TRAFFIC_PER_EXPERT[dom] * touched
         roof["traffic_source"] = "ncu dram bytes per touched expert (smaller case) x touched experts per launch"
@@ -579,7 +587,12 @@ def _oracle_units(wl, dev):
             M.router_topk(xb, wr, K_TOP)
         t_r = time.perf_counter() - t0
         t0 = time.perf_counter()
-        if fmt == "stq":
+        if fmt == "stq" and wl.name == "prefill_stq":
+            # prefill regime: MXFP8 activations and h
+            mats = [F.stq1_unpack(p_, r, c_) for p_, (r, c_) in zip(packed, ((I, H), (I, H), (H, I)))]
+            xc, xs = F.mxfp8_quantize(X)
+            M.expert_ffn_mx(mats[0], mats[1], mats[2], F.mxfp8_dequantize(xc, xs))
+        elif fmt == "stq":
             mats = [F.stq1_unpack(p_, r, c_) for p_, (r, c_) in zip(packed, ((I, H), (I, H), (H, I)))]
             M.expert_ffn_bf16h(mats[0], mats[1], mats[2], X)
         else:

@@ -30,7 +30,7 @@ _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c
 
 class MoeDesc(ctypes.Structure):
     _fields_ = [("T", _i32), ("H", _i32), ("I", _i32), ("E", _i32), ("k", _i32),
-                ("out_fp32", _i32), ("add_residual", _i32)]
+                ("out_fp32", _i32), ("add_residual", _i32), ("regime", _i32)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -68,7 +68,7 @@ SIGNATURES = {
 
 KERNEL_KINDS = ["router_logits", "router_topk", "permute", "quant_x", "gate_up", "down", "combine", "gemv", "gemm",
                 "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down", "rmsnorm",
-                "pack_ls"]
+                "pack_ls", "gate_up_stq_tc", "down_stq_tc"]
 
 
 class StqTiming(ctypes.Structure):
@@ -318,8 +318,11 @@ def moe_permute(topk_ids, E, err=None, stream=None):
     return out
 
 
-def make_desc(T, H, I, E, k, out_fp32=False, add_residual=False):
-    return MoeDesc(T, H, I, E, k, int(bool(out_fp32)), int(bool(add_residual)))
+REGIME_AUTO, REGIME_DECODE, REGIME_PREFILL = 0, 1, 2
+
+
+def make_desc(T, H, I, E, k, out_fp32=False, add_residual=False, regime=REGIME_AUTO):
+    return MoeDesc(T, H, I, E, k, int(bool(out_fp32)), int(bool(add_residual)), int(regime))
 
 
 def moe_workspace_bytes(desc):

@@ -20,11 +20,14 @@
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
-#include "moe_internal.cuh"
-#include "tcgen05.cuh"
+#include "gemm_common.cuh"
 #include "tma.cuh"
 
 namespace {
+
+using gemm::Item;
+using gemm::load_sf;
+using gemm::store_sf;
 
 constexpr int kKT = 128;                          // k per stage
 constexpr int kATile = 128 * 128;                 // smem bytes of one 128 x 128 E2M1 tile (expanded)
@@ -70,34 +73,14 @@ struct Cfg {
 };
 
 struct GemmProblem {
-  int R, K, Ptot;               // weight rows per expert, reduction length, activation rows
+  gemm::Tiling tiles;           // tiles.R = weight rows per expert
+  int K, Ptot;                  // reduction length, activation rows
   const uint8_t* sa;            // weight scales [E*R][K/32] (gate scales for a pair)
   const uint8_t* sa2;           // up-projection scales (gate/up pair)
   const uint8_t* sb;            // activation scales [Ptot][K/32]
-  const int32_t* offsets;       // grouped: [E+1]; nullptr = one dense expert of dense_M tokens
-  const int2* ntiles;           // grouped: (expert, first token) per N tile
-  const int32_t* n_ntiles;      // grouped: number of N tiles (device)
-  int dense_M;
-  int max_items;                // upper bound of the work items (N tiles x M tiles)
-  float* Y;                     // single: [Ptot][R]
-  uint8_t* hq;                  // pair: MXFP8 codes of h [Ptot][R]
-  uint8_t* hs;                  // pair: scales [Ptot][R/32]
+  gemm::EpiOut out;             // out.R = tiles.R
   int32_t* err;
 };
-
-// Scales of stage kt for the four 32-row slices m1 of a 128-row block: lane m0 reads
-// the 4 bytes (4 k-blocks) of rows m0 + 32*m1.  Rows at or past `limit` (absolute)
-// or `nvalid` (relative), and stages past nk, read as zero.
-__device__ __forceinline__ void load_sf(uint32_t (&v)[4], const uint8_t* src, int row0, int nvalid, int limit,
-                                        int k32, int kt, int nk, int lane) {
-#pragma unroll
-  for (int m1 = 0; m1 < 4; ++m1) {
-    const int r = lane + 32 * m1;
-    v[m1] = (kt < nk && r < nvalid && row0 + r < limit)
-                ? __ldg(reinterpret_cast<const uint32_t*>(src + size_t(row0 + r) * k32 + size_t(kt) * 4))
-                : 0u;
-  }
-}
 
 // Pair tile: slices m1 = 0, 1 are gate rows row0 + lane + 32*m1, slices 2, 3 the same
 // rows of the up projection.
@@ -109,44 +92,6 @@ __device__ __forceinline__ void load_sf_pair(uint32_t (&v)[4], const uint8_t* gs
     const int r = row0 + lane + 32 * (m1 & 1);
     v[m1] = kt < nk ? __ldg(reinterpret_cast<const uint32_t*>(src + size_t(r) * k32 + size_t(kt) * 4)) : 0u;
   }
-}
-
-// Store them into the scale-factor atom: row m = m0 + 32*m1 at byte m0*16 + m1*4 + kb.
-__device__ __forceinline__ void store_sf(uint8_t* dst, const uint32_t (&v)[4], int lane) {
-  *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
-}
-
-// One work item = (N tile, M tile); item i covers N tile i / MT and M tile i % MT.
-struct Item {
-  bool valid;
-  int mt, n0, pos0, cnt, arow, brow;
-};
-
-template <int NT>
-__device__ __forceinline__ Item get_item(const GemmProblem& p, int item, int MT, int rows_per_tile) {
-  Item t{};
-  const int nti = item / MT;
-  t.mt = item - nti * MT;
-  int e;
-  if (p.offsets != nullptr) {
-    t.valid = item < p.max_items && nti < *p.n_ntiles;
-    if (!t.valid) return t;
-    const int2 w = p.ntiles[nti];
-    e = w.x;
-    t.n0 = w.y;
-    t.pos0 = p.offsets[e];
-    t.cnt = p.offsets[e + 1] - t.pos0;
-  } else {
-    t.valid = item < p.max_items;
-    if (!t.valid) return t;
-    e = 0;
-    t.n0 = nti * NT;
-    t.pos0 = 0;
-    t.cnt = p.dense_M;
-  }
-  t.arow = e * p.R + t.mt * rows_per_tile;
-  t.brow = t.pos0 + t.n0;
-  return t;
 }
 
 // Persistent: CTA b takes items b, b + gridDim.x, ...  Warp roles: warps 0 and 6 load
@@ -173,7 +118,7 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int MT = p.R / C::kRowsPerTile;
+  const int MT = p.tiles.R / C::kRowsPerTile;
   const int G = gridDim.x;
   const int nk = p.K / kKT;
   const int k32 = p.K / 32;
@@ -216,10 +161,10 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
     bool ok = true;
     uint32_t ra[kPf][4], rb[kPf][4];
     for (int it = 0; ok; ++it) {
-      const Item I = get_item<NT>(p, blockIdx.x + it * G, MT, C::kRowsPerTile);
+      const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, C::kRowsPerTile, NT);
       if (!I.valid) break;
       Item In{};
-      if (cross) In = get_item<NT>(p, blockIdx.x + (it + 1) * G, MT, C::kRowsPerTile);
+      if (cross) In = gemm::get_item(p.tiles, blockIdx.x + (it + 1) * G, MT, C::kRowsPerTile, NT);
       const int kt0 = ((pid - it * nk) % 2 + 2) % 2;  // first k-step of this item for this producer
       if (!cross || it == 0) {
 #pragma unroll
@@ -276,7 +221,7 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int item = blockIdx.x + it * G;
-        if (item >= p.max_items || (p.offsets != nullptr && item / MT >= *p.n_ntiles)) break;
+        if (item >= p.tiles.max_items || (p.tiles.offsets != nullptr && item / MT >= *p.tiles.n_ntiles)) break;
         const int buf = it & 1;
         if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
@@ -311,75 +256,15 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
     for (int it = 0;; ++it) {
-      const Item I = get_item<NT>(p, blockIdx.x + it * G, MT, C::kRowsPerTile);
+      const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, C::kRowsPerTile, NT);
       if (!I.valid) break;
       const int buf = it & 1;
       bool ok = tc::mbar_wait(&tfull[buf], (it >> 1) & 1, p.err);
-      if constexpr (PAIR) {
-        // the four epilogue warps meet at named barriers below, so they agree on ok first
-        uint32_t all;
-        asm volatile(
-            "{\n .reg .pred p, r;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred r, 1, 128, p;\n"
-            " selp.u32 %0, 1, 0, r;\n}"
-            : "=r"(all)
-            : "r"(ok ? 1u : 0u)
-            : "memory");
-        ok = all != 0u;
-      }
+      // the four epilogue warps meet at named barriers, so they agree on ok first
+      if constexpr (PAIR) ok = gemm::all_of_epilogue(ok);
       if (!ok) break;
       tc::fence_after_sync();
-      const uint32_t tl = tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * NT);
-      for (int c0 = 0; c0 < NT; c0 += 16) {
-        if (I.n0 + c0 >= I.cnt) break;
-        uint32_t v[16];
-        tc::tmem_ld_x16(tl + c0, v);
-        tc::tmem_ld_wait();
-        if constexpr (PAIR) {
-          // Warps q and q+2 hold the gate and up values of the same 32 features; the gate
-          // warp takes columns 0-7 of the chunk and the up warp columns 8-15, each handing
-          // the other its half through shared memory.
-          const int pr = q & 1;
-          const bool gate = q < 2;
-          float* mine = ubuf + (2 * pr + (gate ? 0 : 1)) * (32 * 9);
-          const float* other = ubuf + (2 * pr + (gate ? 1 : 0)) * (32 * 9);
-          if (gate) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mine[lane * 9 + j] = __uint_as_float(v[8 + j]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mine[lane * 9 + j] = __uint_as_float(v[j]);
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          const int f = I.mt * 64 + 32 * pr + lane;  // output feature of this lane
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = I.n0 + c0 + (gate ? j : 8 + j);
-            if (col >= I.cnt) break;
-            const float g = gate ? __uint_as_float(v[j]) : other[lane * 9 + j];
-            const float u = gate ? other[lane * 9 + j] : __uint_as_float(v[8 + j]);
-            const float h = g / (1.0f + __expf(-g)) * u;  // silu(g) * u
-            const bool bad = !isfinite(h);
-            // amax over the 32 features of this column: the bits of a non-negative float
-            // order like the float, so one integer max reduction suffices
-            const uint32_t amax_bits = __reduce_max_sync(0xffffffffu, bad ? 0u : (__float_as_uint(h) & 0x7FFFFFFFu));
-            const bool anybad = __any_sync(0xffffffffu, bad);
-            const int ex = anybad ? 255 : mx_scale_exponent(__uint_as_float(amax_bits), 0x600000u, 8);
-            const uint32_t code = anybad ? 0x7Fu : e4m3_code(h, pow2_float(127 - ex));
-            const size_t pos = size_t(I.pos0 + col);
-            p.hq[pos * p.R + f] = uint8_t(code);
-            if (lane == 0) p.hs[pos * (p.R / 32) + (f >> 5)] = uint8_t(ex);
-          }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-        } else {
-          const int f = I.mt * 128 + 32 * q + lane;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int col = I.n0 + c0 + j;
-            if (col >= I.cnt) break;
-            p.Y[size_t(I.pos0 + col) * p.R + f] = __uint_as_float(v[j]);
-          }
-        }
-      }
+      gemm::epilogue_tile<NT, PAIR>(tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * NT), I, p.out, ubuf, q, lane);
       // this warp's reads of the buffer are complete: hand it back to the MMA warp
       tc::fence_before_sync();
       __syncwarp();
@@ -443,17 +328,7 @@ __global__ void __launch_bounds__(1024) mx_plan_kernel(const int32_t* __restrict
 
 
 
-int sm_count() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
-  }
-  return sms;
-}
-
-// Persistent launch over p.max_items work items: at most kCtasPerSm CTAs per SM.
+// Persistent launch over p.tiles.max_items work items: at most kCtasPerSm CTAs per SM.
 template <int NT, bool PAIR>
 stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
                        cudaStream_t s) {
@@ -465,9 +340,8 @@ stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtens
       return STQ_ERR_CUDA;
     configured = true;
   }
-  if (p.max_items <= 0) return STQ_OK;
-  const int cap = C::kCtasPerSm * sm_count();
-  const unsigned grid = unsigned(p.max_items < cap ? p.max_items : cap);
+  if (p.tiles.max_items <= 0) return STQ_OK;
+  const unsigned grid = unsigned(stq_persistent_grid(p.tiles.max_items, C::kCtasPerSm));
   w4a8_gemm_kernel<NT, PAIR><<<grid, kGemmThreads, C::kSmem, s>>>(a, a2, b, p);
   return stq_launch_status();
 }
@@ -489,8 +363,11 @@ int pick_nt(int64_t tokens_per_expert) {
 
 }  // namespace
 
-// Defined in moe.cu: the shared BF16 expert on its own.
-stq_status moe_shared_expert_bf16(const MoeArgs& a, cudaStream_t s);
+stq_status stq_tile_plan_launch(const int32_t* counts, int E, int nt, int2* tiles, int32_t* n_tiles, cudaStream_t s) {
+  StqTimed tm(STQ_K_PLAN, s);
+  mx_plan_kernel<<<1, 1024, 0, s>>>(counts, E, nt, tiles, n_tiles);
+  return stq_launch_status();
+}
 
 stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStream_t s) {
   (void)slots;
@@ -500,11 +377,7 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   if (st != STQ_OK) return st;
   // 2. N tiles of the touched experts
   const int nt = pick_nt(int64_t(P) / (a.E < P ? a.E : P));
-  {
-    StqTimed tm(STQ_K_PLAN, s);
-    mx_plan_kernel<<<1, 1024, 0, s>>>(a.counts, a.E, nt, a.ntiles, a.n_ntiles);
-  }
-  if ((st = stq_launch_status()) != STQ_OK) return st;
+  if ((st = stq_tile_plan_launch(a.counts, a.E, nt, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
   const int max_tiles = P / nt + (a.E < P ? a.E : P);
   // 3. gate/up pair with SwiGLU and MXFP8 h
   CUtensorMap mg, mu, mx, md, mh;
@@ -513,19 +386,20 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
       !tma::map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !tma::map_u8(&mh, a.hq, a.I, P, nt))
     return STQ_ERR_CUDA;
   GemmProblem gp{};
-  gp.R = a.I;
+  gp.tiles.R = a.I;
+  gp.tiles.offsets = a.offsets;
+  gp.tiles.ntiles = a.ntiles;
+  gp.tiles.n_ntiles = a.n_ntiles;
+  gp.tiles.max_items = max_tiles * (a.I / 64);
   gp.K = a.H;
   gp.Ptot = P;
   gp.sa = a.gsc;
   gp.sa2 = a.usc;
   gp.sb = a.xs;
-  gp.offsets = a.offsets;
-  gp.ntiles = a.ntiles;
-  gp.n_ntiles = a.n_ntiles;
-  gp.hq = a.hq;
-  gp.hs = a.hs;
+  gp.out.R = a.I;
+  gp.out.hq = a.hq;
+  gp.out.hs = a.hs;
   gp.err = a.err;
-  gp.max_items = max_tiles * (a.I / 64);
   {
     StqTimed tm(STQ_K_GATE_UP_MX, s);
     st = launch_nt<true>(nt, mg, mu, mx, gp, s);
@@ -534,15 +408,13 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
   // 4. down
   GemmProblem dp = gp;
-  dp.R = a.H;
+  dp.tiles.R = a.H;
+  dp.tiles.max_items = max_tiles * (a.H / 128);
   dp.K = a.I;
   dp.sa = a.dsc;
   dp.sa2 = nullptr;
   dp.sb = a.hs;
-  dp.Y = a.Y;
-  dp.hq = nullptr;
-  dp.hs = nullptr;
-  dp.max_items = max_tiles * (a.H / 128);
+  dp.out = gemm::EpiOut{a.H, a.Y, nullptr, nullptr};
   {
     StqTimed tm(STQ_K_DOWN_MX, s);
     st = launch_nt<false>(nt, md, md, mh, dp, s);
@@ -569,17 +441,17 @@ extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales,
   if (!tma::map_e2m1(&ma, w_codes, uint64_t(K), uint64_t(N)) || !tma::map_u8(&mb, a_codes, uint64_t(K), uint64_t(M), nt))
     return STQ_ERR_CUDA;
   GemmProblem p{};
-  p.R = int(N);
+  p.tiles.R = int(N);
+  p.tiles.dense_M = int(M);
   p.K = int(K);
   p.Ptot = int(M);
   p.sa = w_scales;
   p.sb = a_scales;
-  p.dense_M = int(M);
-  p.Y = y;
+  p.out = gemm::EpiOut{int(N), y, nullptr, nullptr};
   p.err = err;
   const int64_t items = (N / 128) * ((M + nt - 1) / nt);
   STQ_HOST_CHECK(items < (int64_t(1) << 31), STQ_ERR_SHAPE);
-  p.max_items = int(items);
+  p.tiles.max_items = int(items);
   StqTimed tm(STQ_K_GEMM, s);
   return launch_nt<false>(nt, ma, ma, mb, p, s);
 }

@@ -1,0 +1,471 @@
+// Prefill-regime grouped GEMM of STQ1_0 weights x MXFP8 activations on the sm_100a
+// tensor cores.
+//
+// STQ1_0 ("Hy4-preview-GGUF", section 3; "Hy4-preview-FlashMoE-STQ1_0", "How the STQ1_0
+// packing works"): w = d * t with t in {-1, 0, +1}, one zero per four weights, d FP16
+// per 256 weights of a row.  The ternary t is exact in E4M3 (+-1 = 0x38 / 0xB8), so a
+// 256-k block of weights is decoded in shared memory to E4M3 and multiplied with the
+// MXFP8 activations by tcgen05.mma kind::mxf8f6f4 with a unit weight scale (UE8M0 127);
+// the activations keep their UE8M0 scale per 32 k.  d, FP16 with 11 significant bits,
+// fits neither operand format, so each block's product lands in its own TMEM partial
+// buffer and is promoted in FP32: acc += d[row] * partial.
+//
+// Tile: 128 weight rows (M; for gate/up the 64 gate rows of 64 features and the same
+// up rows) x 112 tokens of one expert (N), over all of K, one 256-k block per stage.
+// TMEM (512 columns): partial buffers at 0 and 128, accumulators at 256 and 384 (112
+// columns each), the scale factors at 112..123.
+//
+// Warp roles (448 threads, one CTA per SM, persistent over work items):
+//   warp 0       TMA of the activation tile (two 128-k boxes, 128-byte swizzle) and its
+//                scale factors, re-laid into the scale-factor atoms the MMA reads;
+//   warp 1       TMEM allocation and, from one thread, tcgen05.cp of the scales and the
+//                eight K = 32 MMAs of a stage into the partial buffer of the block;
+//   warps 2-5    promotion: acc += d * partial, TMEM to TMEM through registers;
+//   warps 6-9    epilogue of a finished accumulator (FP32 outputs, or SwiGLU and the
+//                MXFP8 re-quantisation of h);
+//   warps 10-13  decode: each warp turns two 16-row STQ1_0 tile-blocks into E4M3 rows of
+//                the A tile (a shuffle of a 32-entry pattern table per 5-bit code gives
+//                the four bytes of one group).
+// Every hand-off is an mbarrier with a bounded wait (STQ_ERR_TIMEOUT, then exit).
+
+#include "gemm_common.cuh"
+#include "gemv.cuh"
+#include "tma.cuh"
+
+namespace {
+
+using gemm::Item;
+
+constexpr int kNT = 112;                 // tokens per N tile
+constexpr int kSubA = 128 * 128;         // one 128-row x 128-k E4M3 sub-tile (128-byte swizzle)
+constexpr int kSubB = kNT * 128;         // one 112-row x 128-k activation sub-tile
+constexpr int kSf = 512;                 // scale-factor atom: 128 rows x 4 k-blocks of 32
+constexpr int kOffA = 0;                 // two sub-tiles: k 0..127, 128..255 of the block
+constexpr int kOffB = 2 * kSubA;
+constexpr int kOffSfb = kOffB + 2 * kSubB;
+constexpr int kStage = (kOffSfb + 2 * kSf + 1023) / 1024 * 1024;
+constexpr int kStages = 3;
+constexpr int kUBuf = 4 * 32 * 9 * 4;    // gate/up exchange of the epilogue
+constexpr int kSmem = kStages * kStage + kUBuf + kSf /* unit weight scales */ + 1024 /* barriers */ +
+                      1024 /* alignment */;
+constexpr uint32_t kTxB = 2 * kSubB;     // bytes the TMA delivers per stage
+constexpr int kThreads = 448;
+constexpr int kDecodeWarp0 = 10;
+constexpr int kColP = 0;                 // partial buffers: kColP + 128 * i
+constexpr int kColAcc = 256;             // accumulators: kColAcc + 128 * i
+constexpr int kColSfa = 112;
+constexpr int kColSfb = 116;             // two atoms: 116, 120
+constexpr uint32_t kCols = 512;
+static_assert(kSubB % 1024 == 0 && kStage % 1024 == 0, "128-byte swizzle atoms");
+static_assert(kSmem <= 227 * 1024, "shared memory");
+
+struct StqGemm {
+  gemm::Tiling tiles;          // tiles.R = weight rows per expert
+  int K, Ptot;                 // reduction length, activation rows
+  const uint8_t* w0;           // STQ1_0 matrices, expert-major (gate, or down)
+  const uint8_t* w1;           // up projection (gate/up pair)
+  const uint8_t* sb;           // activation scales [Ptot][K/32]
+  gemm::EpiOut out;
+  int32_t* err;
+};
+
+// Pattern table entry of code c: byte l = E4M3 of t at lane l of the group.
+__device__ __forceinline__ uint32_t e4m3_lut_entry(uint32_t c) {
+  const uint32_t z = (c >> 3) & 3u, s = c & 7u;
+  uint32_t e = 0, n = 0;
+#pragma unroll
+  for (uint32_t l = 0; l < 4; ++l) {
+    if (l != z) {
+      e |= (((s >> n) & 1u) ? 0xB8u : 0x38u) << (8 * l);
+      ++n;
+    }
+  }
+  return e;
+}
+
+// A-tile row m (0..127) -> (matrix, row within the expert matrix).
+template <bool PAIR>
+__device__ __forceinline__ const uint8_t* row_matrix(const StqGemm& p, int m, int mt, int& row) {
+  if constexpr (PAIR) {
+    row = mt * 64 + (m & 63);
+    return m < 64 ? p.w0 : p.w1;
+  } else {
+    row = mt * 128 + m;
+    return p.w0;
+  }
+}
+
+// Tile-block (16 rows x 256 k) of block kb holding A-tile rows 16j..16j+15 of item I.
+template <bool PAIR>
+__device__ __forceinline__ const uint8_t* tile_block(const StqGemm& p, const Item& I, int j, int kb) {
+  int row;
+  const uint8_t* w = row_matrix<PAIR>(p, 16 * j, I.mt, row);
+  const int nb = p.K / 256;
+  const size_t mat = size_t(p.tiles.R) * nb * 42;
+  return w + size_t(I.e) * mat + size_t(row >> 4) * nb * stq::kTileBlockBytes + size_t(kb) * stq::kTileBlockBytes;
+}
+
+// FP16 d of A-tile row m in block kb (the d-pair word of row m % 8, half m / 8 % 2).
+template <bool PAIR>
+__device__ __forceinline__ const uint16_t* d_ptr(const StqGemm& p, const Item& I, int m, int kb) {
+  int row;
+  const uint8_t* w = row_matrix<PAIR>(p, m, I.mt, row);
+  const int nb = p.K / 256;
+  const size_t mat = size_t(p.tiles.R) * nb * 42;
+  const uint8_t* tb = w + size_t(I.e) * mat + size_t(row >> 4) * nb * stq::kTileBlockBytes +
+                      size_t(kb) * stq::kTileBlockBytes;
+  return reinterpret_cast<const uint16_t*>(tb + 4 * (row & 7) + 2 * ((row >> 3) & 1));
+}
+
+struct TileWords {
+  uint32_t w[5];
+};
+
+__device__ __forceinline__ void load_tile_words(TileWords& t, const uint8_t* tb, int lane) {
+  const uint4 a = stq::ldg_stream16(tb + 32 + 16 * lane);
+  t.w[0] = a.x;
+  t.w[1] = a.y;
+  t.w[2] = a.z;
+  t.w[3] = a.w;
+  t.w[4] = stq::ldg_stream4(tb + 544 + 4 * lane);
+}
+
+// Groups 4c4..4c4+3 of this lane's row g + 8h as one 16-byte chunk.
+template <int H, int C4>
+__device__ __forceinline__ uint4 decode_chunk(const TileWords& t, uint32_t lut) {
+  uint4 r;
+  r.x = __shfl_sync(stq::kFull, lut, stq::code_at<2 * (4 * C4 + 0) + H>(t.w));
+  r.y = __shfl_sync(stq::kFull, lut, stq::code_at<2 * (4 * C4 + 1) + H>(t.w));
+  r.z = __shfl_sync(stq::kFull, lut, stq::code_at<2 * (4 * C4 + 2) + H>(t.w));
+  r.w = __shfl_sync(stq::kFull, lut, stq::code_at<2 * (4 * C4 + 3) + H>(t.w));
+  return r;
+}
+
+// Write the tile-block of A-tile rows 16j.. into the stage's A sub-tiles.  Lane (g, t)
+// holds rows 16j + g and 16j + g + 8, k = 64t .. 64t + 63 of the block: sub-tile t / 2,
+// 16-byte chunks 4 (t % 2) + c4 of the 128-byte row, stored at chunk (chunk ^ row % 8).
+template <int H, int C4>
+__device__ __forceinline__ void put_chunk(uint8_t* a_stage, const TileWords& t, uint32_t lut, int j, int lane) {
+  const int g = lane >> 2, tq = lane & 3;
+  const int r = 16 * j + g + 8 * H;
+  const int chunk = 4 * (tq & 1) + C4;
+  uint8_t* dst = a_stage + (tq >> 1) * kSubA + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst) = decode_chunk<H, C4>(t, lut);
+}
+
+__device__ __forceinline__ void put_tile_block(uint8_t* a_stage, const TileWords& t, uint32_t lut, int j, int lane) {
+  put_chunk<0, 0>(a_stage, t, lut, j, lane);
+  put_chunk<0, 1>(a_stage, t, lut, j, lane);
+  put_chunk<0, 2>(a_stage, t, lut, j, lane);
+  put_chunk<0, 3>(a_stage, t, lut, j, lane);
+  put_chunk<1, 0>(a_stage, t, lut, j, lane);
+  put_chunk<1, 1>(a_stage, t, lut, j, lane);
+  put_chunk<1, 2>(a_stage, t, lut, j, lane);
+  put_chunk<1, 3>(a_stage, t, lut, j, lane);
+}
+
+}  // namespace
+
+namespace {
+
+// Persistent over work items b, b + gridDim.x, ...; all roles walk the same item list,
+// and a per-CTA block counter g (items x K blocks) drives every ring: stage g % 3, partial
+// buffer g % 2; accumulator buffer = item % 2.
+template <bool PAIR>
+__global__ void __launch_bounds__(kThreads, 1)
+    stq_gemm_kernel(const __grid_constant__ CUtensorMap tmB, StqGemm p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* ubuf = reinterpret_cast<float*>(smem + kStages * kStage);
+  uint8_t* sfa_unit = smem + kStages * kStage + kUBuf;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sfa_unit + kSf);  // [kStages]: TMA bytes + 5 arrivals
+  uint64_t* empty = full + kStages;                              // [kStages]: MMAs of the stage done
+  uint64_t* pfull = empty + kStages;                             // [2]: partial written
+  uint64_t* pempty = pfull + 2;                                  // [2]: partial promoted (4 warps)
+  uint64_t* afull = pempty + 2;                                  // [2]: accumulator complete (4 warps)
+  uint64_t* aempty = afull + 2;                                  // [2]: accumulator drained (4 warps)
+  uint64_t* mdone = aempty + 2;                                  // every MMA of this CTA completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kRows = PAIR ? 64 : 128;  // output features per item
+  const int MT = p.tiles.R / kRows;
+  const int G = gridDim.x;
+  const int nb = p.K / 256;
+
+  // unit weight scales (UE8M0 127 = 2^0) for every row and k-block
+  for (int i = threadIdx.x; i < kSf / 4; i += kThreads) reinterpret_cast<uint32_t*>(sfa_unit)[i] = 0x7F7F7F7Fu;
+  tc::fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 5);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&pfull[b], 1);
+      tc::mbar_init(&pempty[b], 4);
+      tc::mbar_init(&afull[b], 4);
+      tc::mbar_init(&aempty[b], 4);
+    }
+    tc::mbar_init(mdone, 1);
+    tc::fence_barrier_init();
+    tc::prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) tc::tmem_alloc(tmem_holder, kCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- activation loads
+    const int k32 = p.K / 32, nk = p.K / 128;
+    int last_round[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+    bool ok = true;
+    int g = 0;
+    for (int it = 0; ok; ++it) {
+      const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
+      if (!I.valid) break;
+      for (int kb = 0; kb < nb; ++kb, ++g) {
+        const int s = g % kStages, r = g / kStages;
+        uint32_t v0[4], v1[4];
+        gemm::load_sf(v0, p.sb, I.brow, kNT, p.Ptot, k32, 2 * kb, nk, lane);
+        gemm::load_sf(v1, p.sb, I.brow, kNT, p.Ptot, k32, 2 * kb + 1, nk, lane);
+        if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * kStage;
+        gemm::store_sf(st + kOffSfb, v0, lane);
+        gemm::store_sf(st + kOffSfb + kSf, v1, lane);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(&full[s], kTxB);
+          tc::tma_load_2d(st + kOffB, &tmB, kb * 256, I.brow, &full[s]);
+          tc::tma_load_2d(st + kOffB + kSubB, &tmB, kb * 256 + 128, I.brow, &full[s]);
+        }
+        last_round[s] = r;
+      }
+    }
+    // every load this warp issued has landed before the CTA may exit
+    for (int q = 0; q < kStages; ++q)
+      if (last_round[q] >= 0) tc::mbar_wait(&full[q], last_round[q] & 1, p.err);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      tc::cp_sf_32x128b_x4(tmem + kColSfa, tc::smem_desc_sf(tc::smem_u32(sfa_unit)));
+      int g = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int item = blockIdx.x + it * G;
+        if (item >= p.tiles.max_items || (p.tiles.offsets != nullptr && item / MT >= *p.tiles.n_ntiles)) break;
+        for (int kb = 0; kb < nb; ++kb, ++g) {
+          const int s = g % kStages, r = g / kStages, pb = g & 1, pr = g >> 1;
+          if (pr > 0 && !tc::mbar_wait(&pempty[pb], (pr - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          if (!tc::mbar_wait(&full[s], r & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          uint8_t* st = smem + s * kStage;
+          tc::cp_sf_32x128b_x4(tmem + kColSfb, tc::smem_desc_sf(tc::smem_u32(st + kOffSfb)));
+          tc::cp_sf_32x128b_x4(tmem + kColSfb + 4, tc::smem_desc_sf(tc::smem_u32(st + kOffSfb + kSf)));
+          const uint32_t d_col = tmem + uint32_t(kColP + 128 * pb);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int h = kk >> 2, j = kk & 3;
+            const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + kOffA + h * kSubA)) + 2 * j;
+            const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + kOffB + h * kSubB)) + 2 * j;
+            const uint32_t idesc = tc::idesc_mxf8f6f4_ab(kNT, tc::kFmtE4M3, tc::kFmtE4M3, 0u, uint32_t(j));
+            tc::mma_mxf8f6f4(d_col, da, db, idesc, tmem + kColSfa, (tmem + uint32_t(kColSfb + 4 * h)) | (uint32_t(j) << 30),
+                             kk > 0 ? 1u : 0u);
+          }
+          tc::commit(&empty[s]);
+          tc::commit(&pfull[pb]);
+        }
+      }
+      tc::commit(mdone);
+      tc::mbar_wait(mdone, 0, p.err);
+    }
+    __syncwarp();
+  } else if (warp <= 5) {
+    // ---------------------------------------------------------------- promotion
+    const int q = warp & 3;
+    const int m = 32 * q + lane;  // A-tile row = TMEM lane
+    const uint32_t lane_base = tmem + (uint32_t(32 * q) << 16);
+    int g = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
+      if (!I.valid) break;
+      const int abuf = it & 1, ar = it >> 1;
+      if (ar > 0 && !tc::mbar_wait(&aempty[abuf], (ar - 1) & 1, p.err)) break;
+      const uint32_t tacc = lane_base + uint32_t(kColAcc + 128 * abuf);
+      const uint16_t* dp = d_ptr<PAIR>(p, I, m, 0);
+      uint16_t dnext = __ldg(dp);
+      for (int kb = 0; kb < nb; ++kb, ++g) {
+        const int pb = g & 1, pr = g >> 1;
+        const float d = __half2float(__ushort_as_half(dnext));
+        if (kb + 1 < nb) dnext = __ldg(dp + (kb + 1) * (stq::kTileBlockBytes / 2));
+        if (!tc::mbar_wait(&pfull[pb], pr & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t tp = lane_base + uint32_t(kColP + 128 * pb);
+#pragma unroll 1
+        for (int c0 = 0; c0 < kNT; c0 += 16) {
+          uint32_t v[16], a[16];
+          tc::tmem_ld_x16(tp + c0, v);
+          if (kb > 0) {
+            tc::tmem_ld_x16(tacc + c0, a);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(fmaf(d, __uint_as_float(v[j]), __uint_as_float(a[j])));
+          } else {
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(d * __uint_as_float(v[j]));
+          }
+          tc::tmem_st_x16(tacc + c0, a);
+        }
+        // the partial is read and the accumulator written: release the partial buffer
+        tc::tmem_st_wait();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&pempty[pb]);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&afull[abuf]);
+    }
+  } else if (warp <= 9) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    for (int it = 0;; ++it) {
+      const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
+      if (!I.valid) break;
+      const int abuf = it & 1, ar = it >> 1;
+      bool ok = tc::mbar_wait(&afull[abuf], ar & 1, p.err);
+      // the four epilogue warps meet at named barriers, so they agree on ok first
+      if constexpr (PAIR) ok = gemm::all_of_epilogue(ok);
+      if (!ok) break;
+      tc::fence_after_sync();
+      gemm::epilogue_tile<kNT, PAIR>(tmem + (uint32_t(32 * q) << 16) + uint32_t(kColAcc + 128 * abuf), I, p.out,
+                                     ubuf, q, lane);
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&aempty[abuf]);
+    }
+  } else {
+    // ---------------------------------------------------------------- decode
+    const int dw = warp - kDecodeWarp0;  // tile-blocks 2 dw, 2 dw + 1 of the A tile
+    const uint32_t lut = e4m3_lut_entry(uint32_t(lane));
+    Item I = gemm::get_item(p.tiles, blockIdx.x, MT, kRows, kNT);
+    TileWords cur[2] = {}, nxt[2] = {};
+    if (I.valid) {
+      load_tile_words(cur[0], tile_block<PAIR>(p, I, 2 * dw, 0), lane);
+      load_tile_words(cur[1], tile_block<PAIR>(p, I, 2 * dw + 1, 0), lane);
+    }
+    int g = 0;
+    bool ok = true;
+    for (int it = 0; ok && I.valid; ++it) {
+      const Item In = gemm::get_item(p.tiles, blockIdx.x + (it + 1) * G, MT, kRows, kNT);
+      for (int kb = 0; kb < nb; ++kb, ++g) {
+        const int s = g % kStages, r = g / kStages;
+        if (kb + 1 < nb) {
+          load_tile_words(nxt[0], tile_block<PAIR>(p, I, 2 * dw, kb + 1), lane);
+          load_tile_words(nxt[1], tile_block<PAIR>(p, I, 2 * dw + 1, kb + 1), lane);
+        } else if (In.valid) {
+          load_tile_words(nxt[0], tile_block<PAIR>(p, In, 2 * dw, 0), lane);
+          load_tile_words(nxt[1], tile_block<PAIR>(p, In, 2 * dw + 1, 0), lane);
+        }
+        if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t* a_stage = smem + s * kStage + kOffA;
+        put_tile_block(a_stage, cur[0], lut, 2 * dw, lane);
+        put_tile_block(a_stage, cur[1], lut, 2 * dw + 1, lane);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&full[s]);
+        cur[0] = nxt[0];
+        cur[1] = nxt[1];
+      }
+      I = In;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kCols);
+  }
+}
+
+template <bool PAIR>
+stq_status launch_stq_gemm(const CUtensorMap& b, const StqGemm& p, cudaStream_t s) {
+  static int attr_device = -1;  // the >48 KB shared memory opt-in, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return STQ_ERR_CUDA;
+  if (attr_device != dev) {
+    if (cudaFuncSetAttribute(stq_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+        cudaSuccess)
+      return STQ_ERR_CUDA;
+    attr_device = dev;
+  }
+  if (p.tiles.max_items <= 0) return STQ_OK;
+  stq_gemm_kernel<PAIR><<<unsigned(stq_persistent_grid(p.tiles.max_items, 1)), kThreads, kSmem, s>>>(b, p);
+  return stq_launch_status();
+}
+
+}  // namespace
+
+stq_status moe_stq_prefill_experts(const MoeArgs& a, int slots, cudaStream_t s) {
+  const int P = a.P;
+  // 1. activations -> MXFP8 g32 in sorted (expert-grouped) order
+  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.xq, a.xs, s);
+  if (st != STQ_OK) return st;
+  // 2. N tiles of 112 tokens of the touched experts
+  if ((st = stq_tile_plan_launch(a.counts, a.E, kNT, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
+  const int max_tiles = P / kNT + slots;  // sum over experts of ceil(count / 112)
+  CUtensorMap mx, mh;
+  if (!tma::map_u8(&mx, a.xq, uint64_t(a.H), uint64_t(P), kNT) || !tma::map_u8(&mh, a.hq, uint64_t(a.I), uint64_t(P), kNT))
+    return STQ_ERR_CUDA;
+  // 3. gate/up pair, SwiGLU, MXFP8 h
+  StqGemm gp{};
+  gp.tiles.R = a.I;
+  gp.tiles.offsets = a.offsets;
+  gp.tiles.ntiles = a.ntiles;
+  gp.tiles.n_ntiles = a.n_ntiles;
+  gp.tiles.max_items = max_tiles * (a.I / 64);
+  gp.K = a.H;
+  gp.Ptot = P;
+  gp.w0 = a.wg;
+  gp.w1 = a.wu;
+  gp.sb = a.xs;
+  gp.out = gemm::EpiOut{a.I, nullptr, a.hq, a.hs};
+  gp.err = a.err;
+  {
+    StqTimed tm(STQ_K_GATE_UP_STQ_TC, s);
+    st = launch_stq_gemm<true>(mx, gp, s);
+  }
+  if (st != STQ_OK) return st;
+  // 4. down, FP32 expert outputs
+  StqGemm dp = gp;
+  dp.tiles.R = a.H;
+  dp.tiles.max_items = max_tiles * (a.H / 128);
+  dp.K = a.I;
+  dp.w0 = dp.w1 = a.wd;
+  dp.sb = a.hs;
+  dp.out = gemm::EpiOut{a.H, a.Y, nullptr, nullptr};
+  StqTimed tm(STQ_K_DOWN_STQ_TC, s);
+  return launch_stq_gemm<false>(mh, dp, s);
+}

@@ -540,16 +540,16 @@ __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __re
 
 // ----------------------------------------------------------------------------- host side
 
-// CTAs of a persistent GEMV launch: four per SM (the register-limited occupancy), never
+// CTAs of a persistent launch: per_sm per SM (the register-limited occupancy), never
 // more than the work items.
-int stq_persistent_grid(int items) {
+int stq_persistent_grid(int items, int per_sm) {
   static int sms = 0;
   if (sms == 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       sms = 148;
   }
-  const int cap = 4 * sms;
+  const int cap = per_sm * sms;
   return items < 1 ? 1 : (items < cap ? items : cap);
 }
 
@@ -602,7 +602,7 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
 
 static bool desc_ok(const moe_desc* d) {
   return d && d->T >= 0 && d->H > 0 && d->I > 0 && d->E > 0 && d->E <= 1024 && d->k > 0 && d->k <= 32 &&
-         d->k <= d->E;
+         d->k <= d->E && d->regime >= STQ_REGIME_AUTO && d->regime <= STQ_REGIME_PREFILL;
 }
 
 extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
@@ -689,6 +689,10 @@ stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const f
   return stq_launch_status();
 }
 
+// Average routed tokens per expert from which STQ_REGIME_AUTO runs the STQ1_0 experts
+// on the tensor-core GEMM instead of the decode GEMV.
+constexpr int kStqPrefillTokensPerExpert = 32;
+
 extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, const int32_t* topk_ids,
                                          const float* topk_w, const moe_weights* w, void* y, void* workspace,
                                          size_t ws_bytes, stq_stream_t stream) {
@@ -728,7 +732,12 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   a.err = ws.err;
   const int slots = d->E < P ? d->E : P;
 
-  if (w->fmt == STQ_FMT_STQ1_0) {
+  const bool prefill = d->regime == STQ_REGIME_PREFILL ||
+                       (d->regime == STQ_REGIME_AUTO && P >= kStqPrefillTokensPerExpert * slots);
+  if (w->fmt == STQ_FMT_STQ1_0 && prefill) {
+    if ((st = moe_stq_prefill_experts(a, slots, s)) != STQ_OK) return st;
+    if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
+  } else if (w->fmt == STQ_FMT_STQ1_0) {
     a.routed = 1;
     a.n_shared_cta = has_shared ? d->I / 16 : 0;
     a.sched = ws.sched;

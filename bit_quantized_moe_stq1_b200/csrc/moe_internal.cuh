@@ -47,6 +47,20 @@ struct MoeArgs {
 };
 
 MoeWsLayout moe_ws_layout(const moe_desc& d);
+
+// Grid of a persistent launch: min(items, per_sm x SMs), at least 1.
+int stq_persistent_grid(int items, int per_sm = 4);
+
+// N tiles of nt tokens of every expert with tokens: tiles[i] = (expert, first token),
+// *n_tiles = their number (one CTA, E <= 1024).
+stq_status stq_tile_plan_launch(const int32_t* counts, int E, int nt, int2* tiles, int32_t* n_tiles, cudaStream_t s);
+
+// The BF16 shared expert on its own (gate/up, SwiGLU, down into the rows P.. of h and Y).
+stq_status moe_shared_expert_bf16(const MoeArgs& a, cudaStream_t s);
+
+// Routed STQ1_0 experts in the prefill regime (gemm_stq.cu): activations quantised to
+// MXFP8 in sorted pair order, gate/up + SwiGLU into MXFP8 h, down into Y.
+stq_status moe_stq_prefill_experts(const MoeArgs& a, int slots, cudaStream_t s);
 MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L);
 
 // Routed MXFP4 experts (+ the shared BF16 expert): gate/up, SwiGLU, down.

@@ -127,6 +127,18 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 16 consecutive 32-bit columns of this thread's TMEM lane <- r.
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------- descriptors
 
 // K-major operand tile, rows of 128 bytes, 128-byte swizzle, 8-row groups 1024 bytes apart.
@@ -140,11 +152,21 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
   return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(128 >> 4) << 32) | (uint64_t(1) << 46);
 }
 
-// Instruction descriptor of kind::mxf8f6f4 with UE8M0 scales: A = E2M1 (5), B = E4M3 (0),
-// both K-major, M = 128, N = n, scale-factor byte ids a_sf / b_sf.
+// Operand formats of kind::mxf8f6f4.
+constexpr uint32_t kFmtE4M3 = 0;
+constexpr uint32_t kFmtE2M1 = 5;
+
+// Instruction descriptor of kind::mxf8f6f4 with UE8M0 scales: A and B formats, both
+// K-major, M = 128, N = n, scale-factor byte ids a_sf / b_sf.
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4_ab(int n, uint32_t afmt, uint32_t bfmt, uint32_t a_sf,
+                                                         uint32_t b_sf) {
+  return (b_sf << 4) | (afmt << 7) | (bfmt << 10) | (uint32_t(n >> 3) << 17) | (1u << 23) |
+         (uint32_t(128 >> 4) << 24) | (a_sf << 29);
+}
+
+// A = E2M1 weights, B = E4M3 activations.
 __host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int n, uint32_t a_sf, uint32_t b_sf) {
-  return (b_sf << 4) | (5u << 7) | (0u << 10) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(128 >> 4) << 24) |
-         (a_sf << 29);
+  return idesc_mxf8f6f4_ab(n, kFmtE2M1, kFmtE4M3, a_sf, b_sf);
 }
 
 }  // namespace tc

@@ -222,10 +222,22 @@ typedef struct {
   const uint16_t* sh_down;  /* bf16 [H, I]                                       */
 } moe_weights;
 
+/* Kernels for STQ1_0 routed experts (moe_desc.regime; MXFP4 experts have one path).
+ *   STQ_REGIME_AUTO     prefill when T*k >= 32 * min(E, T*k) (32 or more routed tokens
+ *                       per expert on average), else decode;
+ *   STQ_REGIME_DECODE   the decode GEMV: BF16 activations times the ternary patterns,
+ *                       FP32 accumulation, d per 256-block, h rounded to BF16;
+ *   STQ_REGIME_PREFILL  the tensor-core GEMM ("Hy4-preview-SF-WFP4AFP8": activations
+ *                       FP8 E4M3 g32 with UE8M0 scales): x quantised to MXFP8 g32, the
+ *                       patterns as E4M3 +-1/0 with a unit scale (kind::mxf8f6f4), each
+ *                       256-block's FP32 partial times d, h re-quantised to MXFP8 g32. */
+enum { STQ_REGIME_AUTO = 0, STQ_REGIME_DECODE = 1, STQ_REGIME_PREFILL = 2 };
+
 typedef struct {
   int32_t T, H, I, E, k;    /* tokens, hidden, intermediate, experts, top-k     */
   int32_t out_fp32;         /* 1: y is float32 [T, H]; 0: y is bf16 [T, H]      */
   int32_t add_residual;     /* 1: y += x                                         */
+  int32_t regime;           /* STQ_REGIME_* (STQ1_0 experts)                     */
 } moe_desc;
 
 /* Bytes of device workspace moe_expert_forward needs for `d` (256-byte aligned
@@ -234,8 +246,9 @@ size_t moe_workspace_bytes(const moe_desc* d);
 
 /* y[t] = sum_s topk_w[t,s] * FFN_{topk_ids[t,s]}(x[t]) + FFN_shared(x[t]) (+ x[t])
  * with FFN_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x)).  The intermediate h is
- * rounded to bf16 (STQ1_0 and shared expert) or re-quantised to MXFP8 (MXFP4
- * experts, whose input x is quantised to MXFP8 first).  Slots are summed in order
+ * rounded to bf16 (STQ1_0 decode regime and the shared expert) or re-quantised to
+ * MXFP8 (MXFP4 experts and the STQ1_0 prefill regime, whose input x is quantised to
+ * MXFP8 first).  Slots are summed in order
  * s = 0..k-1, without atomics.  Duplicate ids in a token are separate slots; an
  * id outside [0, E) sets STQ_ERR_DEVICE in the workspace error word and its slot
  * contributes 0.  workspace: >= moe_workspace_bytes(d) bytes, 256-B aligned. */
@@ -249,8 +262,9 @@ stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x,
  *   STQ_WS_COUNTS, _OFFSETS, _PERM, _INV, _TLIST, _NTOUCHED: as moe_permute;
  *   STQ_WS_H   bf16 [(P+T), I]: h of routed pairs (sorted order), then shared tokens;
  *   STQ_WS_Y   f32  [(P+T), H]: expert outputs, same row order (unweighted);
- *   STQ_WS_XQ/_XS  MXFP8 of x [T, H] / [T, H/32] (MXFP4 layers);
- *   STQ_WS_HQ/_HS  MXFP8 of h [P, I] / [P, I/32] (MXFP4 layers).
+ *   STQ_WS_XQ/_XS  MXFP8 of x [P, H] / [P, H/32], rows in sorted pair order
+ *                  (MXFP4 layers, STQ1_0 prefill regime);
+ *   STQ_WS_HQ/_HS  MXFP8 of h [P, I] / [P, I/32] (same layers).
  * P = T*k.  Returns (size_t)-1 for an invalid descriptor or region. */
 enum { STQ_WS_COUNTS = 0, STQ_WS_OFFSETS, STQ_WS_PERM, STQ_WS_INV, STQ_WS_TLIST,
        STQ_WS_NTOUCHED, STQ_WS_H, STQ_WS_Y, STQ_WS_XQ, STQ_WS_XS, STQ_WS_HQ, STQ_WS_HS };
@@ -292,7 +306,7 @@ stq_status stq_wait_selftest(int32_t* err, stq_stream_t stream);
 enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM,
        STQ_K_GATE_UP_MX, STQ_K_DOWN_MX, STQ_K_PLAN, STQ_K_SHARED_GATE_UP, STQ_K_SHARED_DOWN,
-       STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_COUNT };
+       STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_GATE_UP_STQ_TC, STQ_K_DOWN_STQ_TC, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
  * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm, stq_rmsnorm_bf16 and stq1_pack_ls is

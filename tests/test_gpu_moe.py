@@ -10,6 +10,7 @@ import torch
 import workloads as W
 from oracle import formats as F
 from oracle import moe as M
+from mx_checks import check_mxfp8_layer
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -111,12 +112,13 @@ def _make_layer(S, T, H, I, E, k, shared, tag):
     return gw, packs, sh, wr, x
 
 
-def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None, x=None):
+def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None, x=None, regime=None):
     gw, packs, sh, wr, x0 = _make_layer(S, T, H, I, E, k, shared, tag)
     x = x0 if x is None else x
     if ids is None:
         ids, tw, _ = S.moe_router_topk(x, wr, k)
-    desc = S.make_desc(T, H, I, E, k, out_fp32=True, add_residual=residual)
+    regime = S.REGIME_DECODE if regime is None else regime
+    desc = S.make_desc(T, H, I, E, k, out_fp32=True, add_residual=residual, regime=regime)
     ws = torch.zeros(S.moe_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
     y = torch.empty((T, H), dtype=torch.float32, device=DEV)
     ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, *(None, None, None),
@@ -130,6 +132,10 @@ def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None,
         perm=S.moe_workspace_view(desc, ws, "perm", torch.int32, (P,)).cpu().numpy(),
         inv=S.moe_workspace_view(desc, ws, "inv", torch.int32, (P,)).cpu().numpy(),
         offsets=S.moe_workspace_view(desc, ws, "offsets", torch.int32, (E + 1,)).cpu().numpy(),
+        xq=S.moe_workspace_view(desc, ws, "xq", torch.uint8, (P, H)).cpu().numpy(),
+        xs=S.moe_workspace_view(desc, ws, "xs", torch.uint8, (P, H // 32)).cpu().numpy(),
+        hq=S.moe_workspace_view(desc, ws, "hq", torch.uint8, (P, I)).cpu().numpy(),
+        hs=S.moe_workspace_view(desc, ws, "hs", torch.uint8, (P, I // 32)).cpu().numpy(),
     )
     return dict(gw=gw, sh=sh, x=x, ids=ids.cpu().numpy(), tw=tw.cpu().double().numpy(), y=y.cpu().double().numpy(),
                 **st)
@@ -193,6 +199,99 @@ def _check_layer(r, T, H, I, E, k, experts=None):
 def test_moe_stq_small_full_check(S, T, H, I, E, k, shared):
     r = _run_layer(S, T, H, I, E, k, shared, ("small", T, H, I, E, k))
     _check_layer(r, T, H, I, E, k)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,shared", [(40, 512, 256, 8, 4, False), (256, 512, 256, 8, 2, True),
+                                               (97, 1024, 512, 2, 2, False)])
+def test_moe_stq_decode_many_tokens_full_check(S, T, H, I, E, k, shared):
+    """Decode kernels with several 8-token chunks per expert (up to 97 tokens)."""
+    r = _run_layer(S, T, H, I, E, k, shared, ("many", T, H, I, E, k))
+    _check_layer(r, T, H, I, E, k)
+
+
+# --------------------------------------------------------------------------- STQ1_0 prefill regime
+
+
+def _stq_weights(r, H, I):
+    gw = r["gw"]
+
+    def weights(e):
+        return (gw[0][e * I:(e + 1) * I].double().cpu().numpy(), gw[1][e * I:(e + 1) * I].double().cpu().numpy(),
+                gw[2][e * H:(e + 1) * H].double().cpu().numpy())
+    return weights
+
+
+def _check_prefill(r, T, H, I, E, k, experts=None):
+    check_mxfp8_layer(r, T, H, I, E, k, _stq_weights(r, H, I), experts)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,shared", [(5, 512, 256, 8, 2, True), (256, 512, 256, 8, 2, True),
+                                               (200, 768, 512, 4, 3, True), (97, 1024, 512, 2, 2, False),
+                                               (300, 256, 256, 3, 1, False)])
+def test_moe_stq_prefill_full_check(S, T, H, I, E, k, shared):
+    """Tensor-core STQ1_0 GEMM: 1 to 300 tokens per expert (several 112-token tiles with
+    ragged tails), K from one 256-block up, gate/up item groups of 64 features."""
+    r = _run_layer(S, T, H, I, E, k, shared, ("pf", T, H, I, E, k), regime=S.REGIME_PREFILL)
+    _check_prefill(r, T, H, I, E, k)
+
+
+@pytest.mark.parametrize("split", [(112, 113, 1), (300, 0, 0), (111, 1, 224)])
+def test_moe_stq_prefill_tile_edges(S, split):
+    """Expert loads at the 112-token tile edges and one expert taking every token."""
+    E, k, H, I = 3, 1, 512, 256
+    T = sum(split)
+    ids = torch.tensor(np.repeat(np.arange(E), split).reshape(T, 1), dtype=torch.int32, device=DEV)
+    tw = torch.ones((T, 1), dtype=torch.float32, device=DEV)
+    r = _run_layer(S, T, H, I, E, k, True, ("edges",) + split, ids=ids, tw=tw, regime=S.REGIME_PREFILL)
+    _check_prefill(r, T, H, I, E, k)
+
+
+def test_moe_stq_prefill_wide_range_activations(S):
+    """Activations spanning 2^-30 .. 2^30 and a zero row through the MXFP8 prefill path."""
+    T, H, I, E, k = 160, 512, 256, 2, 2
+    g = W.generator(DEV, 0, "wide-pf", "mag")
+    mag = torch.exp2(torch.randint(-30, 31, (T, H), generator=g, device=DEV).float())
+    x = (W.bf16_normal((T, H), 1.0, DEV, 0, "wide-pf", "x").float() * mag).to(torch.bfloat16)
+    x[7] = 0
+    ids, tw = W.uniform_routing(T, E, k, DEV, 0, "wide-pf", "ids")
+    r = _run_layer(S, T, H, I, E, k, True, "wide-pf", ids=ids, tw=tw, x=x, regime=S.REGIME_PREFILL)
+    _check_prefill(r, T, H, I, E, k)
+
+
+def test_moe_stq_auto_regime_threshold(S):
+    """STQ_REGIME_AUTO takes the prefill kernels from 32 routed tokens per expert on
+    average: its output equals the forced regime's, bit for bit, on either side."""
+    H, I, E, k = 512, 256, 4, 2
+    for T, pick in ((63, "decode"), (64, "prefill")):
+        ys = {}
+        for name, reg in (("auto", S.REGIME_AUTO), ("decode", S.REGIME_DECODE), ("prefill", S.REGIME_PREFILL)):
+            ys[name] = _run_layer(S, T, H, I, E, k, True, ("auto", T), regime=reg)["y"]
+        assert np.array_equal(ys["auto"], ys[pick])
+        assert not np.array_equal(ys["decode"], ys["prefill"])
+
+
+def test_moe_stq_prefill_config_sampled(S):
+    """Prefill MoE layer, STQ1_0: 256 experts, 6144/2048, 1024 tokens, top-8, shared
+    (32 routed tokens per expert on average: the automatic regime picks the GEMM)."""
+    T, H, I, E, k = 1024, 6144, 2048, 256, 8
+    r = _run_layer(S, T, H, I, E, k, True, "prefill", regime=S.REGIME_AUTO)
+    counts = np.bincount(r["ids"].reshape(-1), minlength=E)
+    touched = np.flatnonzero(counts)
+    busiest = touched[np.argsort(-counts[touched], kind="stable")[:2]]
+    sample = np.unique(np.concatenate([busiest, touched[:: max(1, touched.size // 3)]]))
+    _check_prefill(r, T, H, I, E, k, experts=sample)
+
+
+def test_moe_stq_prefill_bench_shape_sampled(S):
+    """The STQ1_0 prefill workload as timed: 4096 tokens, Zipf(1.1) routing over 256
+    experts, top-8, 6144/2048, no shared expert; busiest, median and lightest experts."""
+    T, H, I, E, k = 4096, 6144, 2048, 256, 8
+    ids, tw = W.zipf_routing(T, E, k, DEV, 0, "stqpre", "z")
+    r = _run_layer(S, T, H, I, E, k, False, "stqpre", ids=ids, tw=tw, regime=S.REGIME_AUTO)
+    counts = np.bincount(r["ids"].reshape(-1), minlength=E)
+    order = np.argsort(counts, kind="stable")
+    sample = [order[-1], order[len(order) // 2], order[np.flatnonzero(counts[order])[0]]]
+    _check_prefill(r, T, H, I, E, k, experts=sample)
 
 
 def test_moe_stq_decode_config_sampled(S):

@@ -7,6 +7,7 @@ import torch
 import workloads as W
 from oracle import formats as F
 from oracle import moe as M
+from mx_checks import check_mxfp8_layer
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -64,9 +65,6 @@ def test_w4a8_gemm_zero_and_empty(S):
 
 # --------------------------------------------------------------------------- MXFP4 MoE layer
 
-SILU_DMAX = 1.1
-
-
 def _mx_layer(S, T, H, I, E, k, shared, tag, routing="router"):
     g = [W.mxfp4_random(E * I, H, DEV, 0, tag, "g"), W.mxfp4_random(E * I, H, DEV, 0, tag, "u"),
          W.mxfp4_random(E * H, I, DEV, 0, tag, "d")]
@@ -104,50 +102,10 @@ def _rows(pair, e, R, K):
 
 
 def _check_mx_layer(r, T, H, I, E, k, experts=None):
-    P = T * k
-    counts, offsets, perm, inv = M.permute(r["ids"], E)
-    assert np.array_equal(r["perm"], perm) and np.array_equal(r["inv"], inv)
-    xb = np_bits(r["x"])
-    # stage 1: activations quantised in sorted pair order, bit-exact
-    rxq, rxs = F.mxfp8_quantize(F.bf16_decode(xb[perm // k]))
-    assert np.array_equal(r["xq"], rxq) and np.array_equal(r["xs"], rxs)
-    A = F.mxfp8_dequantize(rxq, rxs)
-    hdeq = F.mxfp8_dequantize(r["hq"], r["hs"])
-    touched = np.flatnonzero(counts)
-    for e in (touched if experts is None else experts):
-        pos = np.arange(offsets[e], offsets[e + 1])
-        Wg = F.mxfp4_unpack(*_rows(r["g"][0], e, I, H), I, H)
-        Wu = F.mxfp4_unpack(*_rows(r["g"][1], e, I, H), I, H)
-        Wd = F.mxfp4_unpack(*_rows(r["g"][2], e, H, I), H, I)
-        # stage 2: SwiGLU and MXFP8 h, propagated bound plus the E4M3 step of either scale
-        g, sg = M.matvec_with_scale(Wg, A[pos])
-        u, su = M.matvec_with_scale(Wu, A[pos])
-        tg, tu = 1e-3 * sg + 1e-5, 1e-3 * su + 1e-5
-        h = M.swiglu(g, u)
-        prop = SILU_DMAX * tg * (np.abs(u) + tu) + np.abs(M.silu(g)) * tu
-        _, href_s = F.mxfp8_quantize(h.astype(np.float32).astype(np.float64))
-        sc = np.maximum(np.repeat(F.ue8m0_decode(href_s), 32, axis=1), np.repeat(F.ue8m0_decode(r["hs"][pos]), 32, axis=1))
-        bound = prop * (1 + 2.0 ** -4) + 2.0 ** -4 * np.abs(h) + sc * 2.0 ** -9 + 1e-6
-        assert np.all(np.abs(hdeq[pos] - h) <= bound), float(np.max(np.abs(hdeq[pos] - h) / bound))
-        # stage 3: down on the GPU's own h
-        y, sy = M.matvec_with_scale(Wd, hdeq[pos])
-        assert np.all(np.abs(r["Y"][pos] - y) <= 1e-3 * sy + 1e-5), float(np.max(np.abs(r["Y"][pos] - y) / (1e-3 * sy + 1e-5)))
-    if r["sh"] is not None:
-        X = F.bf16_decode(xb)
-        sg_, su_, sd_ = (m.float().double().cpu().numpy() for m in r["sh"])
-        y, sy = M.matvec_with_scale(sd_, r["h"][P:P + T])
-        assert np.all(np.abs(r["Y"][P:P + T] - y) <= 1e-3 * sy + 1e-5)
-    # combine of the GPU's own expert outputs: FP32 sum of k (+1) terms
-    yc = np.zeros((T, H))
-    mag = np.zeros((T, H))
-    for t in range(T):
-        for s in range(k):
-            yc[t] += r["tw"][t, s] * r["Y"][inv[t * k + s]]
-            mag[t] += np.abs(r["tw"][t, s] * r["Y"][inv[t * k + s]])
-        if r["sh"] is not None:
-            yc[t] += r["Y"][P + t]
-            mag[t] += np.abs(r["Y"][P + t])
-    assert np.all(np.abs(r["y"] - yc) <= 1e-6 * mag + 1e-6)
+    def weights(e):
+        return (F.mxfp4_unpack(*_rows(r["g"][0], e, I, H), I, H), F.mxfp4_unpack(*_rows(r["g"][1], e, I, H), I, H),
+                F.mxfp4_unpack(*_rows(r["g"][2], e, H, I), H, I))
+    check_mxfp8_layer(r, T, H, I, E, k, weights, experts)
 
 
 @pytest.mark.parametrize("T,H,I,E,k,shared", [(5, 512, 256, 8, 2, True), (3, 256, 128 * 2, 4, 4, False),

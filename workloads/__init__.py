@@ -49,6 +49,7 @@ WORKLOADS = {
     "w4a8_gemm": Workload("w4a8_gemm", 128, 1, ("mx",), False, False, False, E=1, k=1),
     "decode_stq": Workload("decode_stq", 8, 1, ("stq",), True, True, False),
     "prefill_w4a8": Workload("prefill_w4a8", 4096, 1, ("mx",), False, False, False),
+    "prefill_stq": Workload("prefill_stq", 4096, 1, ("stq",), False, False, False),
     "stacked_decode": Workload("stacked_decode", 32, 8, ("stq", "mx") * 4, True, True, True),
 }
 
