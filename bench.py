@@ -40,6 +40,7 @@ H, I, E, K_TOP = W.HIDDEN, W.INTER, W.EXPERTS, W.TOPK
 STQ_MAT = I * H // 256 * 42                 # 2,064,384 bytes per STQ1_0 expert matrix
 MX_MAT = I * H // 2 + I * H // 32           # 6,684,672 bytes per MXFP4 matrix (codes + scales)
 BF16_MAT = I * H * 2                        # 25,165,824
+MX8_MAT = I * H + I * H // 32               # 12,976,128 per MXFP8 matrix (codes + scales)
 ROUTER_BYTES = E * H * 2                    # 3,145,728
 NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense BF16 tensor rate
 
@@ -216,11 +217,12 @@ class StqPackLs(Workload):
 class MoeLayers(Workload):
     """MoE layers of hidden 6144, 256 experts of intermediate 2048, top-8."""
 
-    def __init__(self, S, dev, name, T, fmts, router, shared, residual, experts=E):
+    def __init__(self, S, dev, name, T, fmts, router, shared, residual, experts=E, shared_fmt="bf16"):
         global E
         E = experts
         self.S, self.dev, self.name, self.T = S, dev, name, T
         self.fmts, self.router, self.shared, self.residual = fmts, router, shared, residual
+        self.shared_fmt = shared_fmt
         self.layers = [self._layer(l, f) for l, f in enumerate(fmts)]
         self.x = [W.bf16_normal((T, H), 1.0, dev, 0, name, "x", b) for b in range(N_BATCHES)]
         if not router:
@@ -260,7 +262,12 @@ class MoeLayers(Workload):
                   W.bf16_normal((H, I), 0.02, self.dev, 0, self.name, l, "sd")]
         wr = W.bf16_normal((E, H), 0.02, self.dev, 0, self.name, l, "router") if self.router else None
         f = S.FMT_STQ1_0 if fmt == "stq" else S.FMT_MXFP4
-        return dict(fmt=fmt, wr=wr, w=S.ExpertWeights(f, *mats, *scales, *sh))
+        if self.shared and self.shared_fmt == "mx8":
+            q = [S.mxfp8_quantize_bf16(m) for m in sh]
+            return dict(fmt=fmt, wr=wr, sh_bf16=sh,
+                        w=S.ExpertWeights(f, *mats, *scales, *(c for c, _ in q), sh_fmt=S.SHARED_MXFP8,
+                                          sh_gate_sc=q[0][1], sh_up_sc=q[1][1], sh_down_sc=q[2][1]))
+        return dict(fmt=fmt, wr=wr, sh_bf16=sh, w=S.ExpertWeights(f, *mats, *scales, *sh))
 
     def step(self, i, x=None, y=None):
         S = self.S
@@ -307,13 +314,21 @@ class MoeLayers(Workload):
         n = self._acct[b]
         T, P = self.T, self.T * K_TOP
         tot, kinds = 0, {}
+        sh8 = self.shared and self.shared_fmt == "mx8"
+        sh_mat = MX8_MAT if sh8 else BF16_MAT
         for L, t in zip(self.layers, n):
             mat = STQ_MAT if L["fmt"] == "stq" else MX_MAT
-            by = t * 3 * mat + (3 * BF16_MAT if self.shared else 0) + (E * H * 2 if self.router else 0) + 2 * T * H * 2
+            by = t * 3 * mat + (3 * sh_mat if self.shared else 0) + (E * H * 2 if self.router else 0) + 2 * T * H * 2
             tot += by
+            if sh8:
+                kinds.setdefault("shared_gate_up", []).append(
+                    dict(bytes=2 * MX8_MAT + T * H * (1 + 1 / 32) + T * I * (1 + 1 / 32), flops=4 * T * I * H))
+                kinds.setdefault("shared_down", []).append(
+                    dict(bytes=MX8_MAT + T * I * (1 + 1 / 32) + T * H * 4, flops=2 * T * I * H))
+            sh_fused = self.shared and not sh8  # BF16 shared tiles inside the STQ1_0 decode kernels
             if L["fmt"] == "stq":
-                gu = t * 2 * STQ_MAT + (2 * BF16_MAT if self.shared else 0) + T * H * 2 + (P + T) * I * 2
-                dn = t * STQ_MAT + (BF16_MAT if self.shared else 0) + (P + T) * I * 2 + (P + T) * H * 4
+                gu = t * 2 * STQ_MAT + (2 * BF16_MAT if sh_fused else 0) + T * H * 2 + (P + T) * I * 2
+                dn = t * STQ_MAT + (BF16_MAT if sh_fused else 0) + (P + T) * I * 2 + (P + T) * H * 4
                 kinds.setdefault("gate_up", []).append(dict(bytes=gu, flops=4 * P * I * H, touched=t))
                 kinds.setdefault("down", []).append(dict(bytes=dn, flops=2 * P * I * H, touched=t))
                 # prefill regime (tensor-core GEMM on MXFP8 activations): weights once, x and
@@ -345,11 +360,11 @@ def make_workload(name, S, dev, experts=256):
         # one MXFP4 layer of the stacked workload (a small case for profiler captures)
         return MoeLayers(S, dev, name, 32, ("mx",), True, True, True, experts)
     wl = W.WORKLOADS[name]
-    return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual, experts)
+    return MoeLayers(S, dev, name, wl.tokens, wl.formats, wl.router, wl.shared, wl.residual, experts, wl.shared_fmt)
 
 
-WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "prefill_stq", "stacked_decode", "decode_mx",
-                  "stq_pack_ls"]
+WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "decode_stq_sh8", "prefill_w4a8", "prefill_stq",
+                  "stacked_decode", "decode_mx", "stq_pack_ls"]
 
 
 # ----------------------------------------------------------------------------- measurement
@@ -579,8 +594,10 @@ def _oracle_units(wl, dev):
             lw = L["w"]
             packed = [(c_[:r].cpu().numpy(), s_[:r].cpu().numpy()) for c_, s_, r in
                       ((lw.gate, lw.gate_sc, I), (lw.up, lw.up_sc, I), (lw.down, lw.down_sc, H))]
-        shared = [m.float().double().cpu().numpy() for m in (L["w"].sh_gate, L["w"].sh_up, L["w"].sh_down)] \
-            if wl.shared else None
+        shared = [m.float().double().cpu().numpy() for m in L["sh_bf16"]] if wl.shared else None
+        if shared is not None and wl.shared_fmt == "mx8":
+            # stored MXFP8 weights (quantised before the timed unit, like the GPU's)
+            shared = [F.mxfp8_dequantize(*F.mxfp8_quantize(m_)) for m_ in shared]
         wr = L["wr"].view(torch.int16).cpu().numpy().view(np.uint16) if wl.router else None
         t0 = time.perf_counter()
         if wr is not None:
@@ -601,7 +618,10 @@ def _oracle_units(wl, dev):
             M.expert_ffn_mx(mats[0], mats[1], mats[2], F.mxfp8_dequantize(xc, xs))
         t_e = time.perf_counter() - t0
         t0 = time.perf_counter()
-        if shared is not None:
+        if shared is not None and wl.shared_fmt == "mx8":
+            xc, xs = F.mxfp8_quantize(X)
+            M.expert_ffn_mx(shared[0], shared[1], shared[2], F.mxfp8_dequantize(xc, xs))
+        elif shared is not None:
             M.expert_ffn_bf16h(shared[0], shared[1], shared[2], X)
         if wl.residual:
             M.rms_norm(X, W.STACK_RMS_EPS)

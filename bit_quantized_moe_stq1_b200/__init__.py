@@ -36,7 +36,8 @@ class MoeDesc(ctypes.Structure):
 class MoeWeights(ctypes.Structure):
     _fields_ = [("fmt", _i32), ("gate", _vp), ("up", _vp), ("down", _vp),
                 ("gate_sc", _vp), ("up_sc", _vp), ("down_sc", _vp),
-                ("sh_gate", _vp), ("sh_up", _vp), ("sh_down", _vp)]
+                ("sh_gate", _vp), ("sh_up", _vp), ("sh_down", _vp),
+                ("sh_fmt", _i32), ("sh_gate_sc", _vp), ("sh_up_sc", _vp), ("sh_down_sc", _vp)]
 
 
 SIGNATURES = {
@@ -342,19 +343,28 @@ def moe_workspace_view(desc, workspace, region, dtype, shape):
     return workspace[off: off + n * esz].view(dtype).view(*shape)
 
 
+SHARED_BF16, SHARED_MXFP8 = 0, 1
+
+
 class ExpertWeights:
-    """Device tensors of one layer's experts (kept alive by this object)."""
+    """Device tensors of one layer's experts (kept alive by this object).  The shared
+    expert is BF16 (sh_fmt SHARED_BF16) or MXFP8 (SHARED_MXFP8: sh_* E4M3 codes and
+    sh_*_sc UE8M0 scales, as mxfp8_quantize_bf16 writes them)."""
 
     def __init__(self, fmt, gate, up, down, gate_sc=None, up_sc=None, down_sc=None,
-                 sh_gate=None, sh_up=None, sh_down=None):
+                 sh_gate=None, sh_up=None, sh_down=None, sh_fmt=SHARED_BF16,
+                 sh_gate_sc=None, sh_up_sc=None, sh_down_sc=None):
         self.fmt, self.gate, self.up, self.down = fmt, gate, up, down
         self.gate_sc, self.up_sc, self.down_sc = gate_sc, up_sc, down_sc
         self.sh_gate, self.sh_up, self.sh_down = sh_gate, sh_up, sh_down
+        self.sh_fmt = sh_fmt
+        self.sh_gate_sc, self.sh_up_sc, self.sh_down_sc = sh_gate_sc, sh_up_sc, sh_down_sc
 
     def struct(self):
         return MoeWeights(self.fmt, _ptr(self.gate), _ptr(self.up), _ptr(self.down),
                           _ptr(self.gate_sc), _ptr(self.up_sc), _ptr(self.down_sc),
-                          _ptr(self.sh_gate), _ptr(self.sh_up), _ptr(self.sh_down))
+                          _ptr(self.sh_gate), _ptr(self.sh_up), _ptr(self.sh_down), int(self.sh_fmt),
+                          _ptr(self.sh_gate_sc), _ptr(self.sh_up_sc), _ptr(self.sh_down_sc))
 
 
 def moe_expert_forward(desc, x, topk_ids, topk_w, weights, y, workspace, stream=None):

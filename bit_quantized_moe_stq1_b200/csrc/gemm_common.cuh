@@ -68,6 +68,13 @@ __device__ __forceinline__ Item get_item(const Tiling& p, int item, int MT, int 
   return t;
 }
 
+// MMA width for an item: its tokens in the N tile, rounded up to the 16-column step of
+// an M = 128 MMA (columns past it are neither computed nor read).
+__device__ __forceinline__ int item_cols(const Item& I, int NT) {
+  const int n = min(NT, I.cnt - I.n0);
+  return (n + 15) & ~15;
+}
+
 // Outputs of the epilogue.
 struct EpiOut {
   int R;          // weight rows per expert (output features)

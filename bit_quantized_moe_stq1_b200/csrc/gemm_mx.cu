@@ -41,7 +41,8 @@ constexpr int smem_budget(int nt) { return ctas_per_sm(nt) == 2 ? 112 * 1024 : 2
 // PAIR = the gate/up pair of one expert: the 128-row A tile holds 64 gate rows (TMEM
 // lanes 0-63) and the same 64 rows of the up projection (lanes 64-127), so one MMA per
 // k-block produces both and the epilogue pairs lane r with lane r + 64.
-template <int NT, bool PAIR>
+// A8: the weights are E4M3 (MXFP8, one byte per weight) instead of E2M1.
+template <int NT, bool PAIR, bool A8 = false>
 struct Cfg {
   static constexpr int kB = NT * 128;
   static constexpr int kOffA = 0;
@@ -66,7 +67,7 @@ struct Cfg {
   static constexpr int kColsUsed = 2 * NT + 8;
   static constexpr uint32_t kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
-  static constexpr uint32_t kTx = kATx + uint32_t(kB);
+  static constexpr uint32_t kTx = (A8 ? uint32_t(kATile) : kATx) + uint32_t(kB);
   static_assert(kStages >= 2, "shared memory budget (one stage per producer at least)");
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "tile N");
   static_assert(kCtasPerSm * kCols <= 512, "TMEM columns");
@@ -103,11 +104,11 @@ __device__ __forceinline__ void load_sf_pair(uint32_t (&v)[4], const uint8_t* gs
 constexpr int kGemmThreads = 224;  // producer, MMA, 4 epilogue warps, second producer
 constexpr int kProducer2 = 6;
 
-template <int NT, bool PAIR>
-__global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
+template <int NT, bool PAIR, bool A8>
+__global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, GemmProblem p) {
-  using C = Cfg<NT, PAIR>;
+  using C = Cfg<NT, PAIR, A8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* ubuf = reinterpret_cast<float*>(smem + C::kStages * C::kStage);
@@ -220,8 +221,9 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
       int g = 0;  // global k-step
       bool ok = true;
       for (int it = 0; ok; ++it) {
-        const int item = blockIdx.x + it * G;
-        if (item >= p.tiles.max_items || (p.tiles.offsets != nullptr && item / MT >= *p.tiles.n_ntiles)) break;
+        const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, C::kRowsPerTile, NT);
+        if (!I.valid) break;
+        const int ncols = gemm::item_cols(I, NT);
         const int buf = it & 1;
         if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
@@ -241,7 +243,8 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR>::kCtasPerSm)
           const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffB));
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t idesc = tc::idesc_mxf8f6f4(NT, uint32_t(kb), uint32_t(kb));
+            const uint32_t idesc = tc::idesc_mxf8f6f4_ab(ncols, A8 ? tc::kFmtE4M3 : tc::kFmtE2M1, tc::kFmtE4M3,
+                                                         uint32_t(kb), uint32_t(kb));
             const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
             tc::mma_mxf8f6f4(acc_col, da + 2 * kb, db + 2 * kb, idesc, (tmem + C::kColSfa) | (uint32_t(kb) << 30),
                              (tmem + C::kColSfb) | (uint32_t(kb) << 30), acc);
@@ -329,31 +332,33 @@ __global__ void __launch_bounds__(1024) mx_plan_kernel(const int32_t* __restrict
 
 
 // Persistent launch over p.tiles.max_items work items: at most kCtasPerSm CTAs per SM.
-template <int NT, bool PAIR>
+template <int NT, bool PAIR, bool A8>
 stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
                        cudaStream_t s) {
-  using C = Cfg<NT, PAIR>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(w4a8_gemm_kernel<NT, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
-        cudaSuccess)
+  using C = Cfg<NT, PAIR, A8>;
+  static int attr_device = -1;  // the >48 KB shared memory opt-in, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return STQ_ERR_CUDA;
+  if (attr_device != dev) {
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<NT, PAIR, A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmem) != cudaSuccess)
       return STQ_ERR_CUDA;
-    configured = true;
+    attr_device = dev;
   }
   if (p.tiles.max_items <= 0) return STQ_OK;
   const unsigned grid = unsigned(stq_persistent_grid(p.tiles.max_items, C::kCtasPerSm));
-  w4a8_gemm_kernel<NT, PAIR><<<grid, kGemmThreads, C::kSmem, s>>>(a, a2, b, p);
+  w4a8_gemm_kernel<NT, PAIR, A8><<<grid, kGemmThreads, C::kSmem, s>>>(a, a2, b, p);
   return stq_launch_status();
 }
 
-template <bool PAIR>
+template <bool PAIR, bool A8 = false>
 stq_status launch_nt(int nt, const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
                      cudaStream_t s) {
   switch (nt) {
-    case 16: return launch_gemm<16, PAIR>(a, a2, b, p, s);
-    case 32: return launch_gemm<32, PAIR>(a, a2, b, p, s);
-    case 64: return launch_gemm<64, PAIR>(a, a2, b, p, s);
-    default: return launch_gemm<128, PAIR>(a, a2, b, p, s);
+    case 16: return launch_gemm<16, PAIR, A8>(a, a2, b, p, s);
+    case 32: return launch_gemm<32, PAIR, A8>(a, a2, b, p, s);
+    case 64: return launch_gemm<64, PAIR, A8>(a, a2, b, p, s);
+    default: return launch_gemm<128, PAIR, A8>(a, a2, b, p, s);
   }
 }
 
@@ -420,6 +425,56 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
     st = launch_nt<false>(nt, md, md, mh, dp, s);
   }
   return st;
+}
+
+// The MXFP8 shared expert ("Hy4-preview-SF-WFP4AFP8", "Quant Diff": shared experts are
+// MXFP8 W8A8 g32): the same GEMM with E4M3 weights, over the T tokens as one dense
+// expert.  Its activations and h take the rows P.. of the MXFP8 workspace regions, its
+// outputs the rows P.. of Y.  N tile from the token count, halved while the gate/up
+// launch would leave SMs idle.
+stq_status moe_shared_expert_mx8(const MoeArgs& a, cudaStream_t s) {
+  const int T = a.T, P = a.P;
+  uint8_t* xq = a.xq + size_t(P) * a.H;
+  uint8_t* xs = a.xs + size_t(P) * (a.H / 32);
+  uint8_t* hq = a.hq + size_t(P) * a.I;
+  uint8_t* hs = a.hs + size_t(P) * (a.I / 32);
+  stq_status st = stq_mxfp8_quantize_launch(a.x, T, a.H, xq, xs, s);
+  if (st != STQ_OK) return st;
+  int nt = pick_nt(T);
+  while (nt > 16 && (a.I / 64) * ((T + nt - 1) / nt) < 148) nt /= 2;
+  const int ntile = (T + nt - 1) / nt;
+  CUtensorMap mg, mu, mx, md, mh;
+  if (!tma::map_u8(&mg, a.sgq, uint64_t(a.H), uint64_t(a.I), 64) ||
+      !tma::map_u8(&mu, a.suq, uint64_t(a.H), uint64_t(a.I), 64) ||
+      !tma::map_u8(&md, a.sdq, uint64_t(a.I), uint64_t(a.H), 128) || !tma::map_u8(&mx, xq, a.H, T, nt) ||
+      !tma::map_u8(&mh, hq, a.I, T, nt))
+    return STQ_ERR_CUDA;
+  GemmProblem gp{};
+  gp.tiles.R = a.I;
+  gp.tiles.dense_M = T;
+  gp.tiles.max_items = ntile * (a.I / 64);
+  gp.K = a.H;
+  gp.Ptot = T;
+  gp.sa = a.sgs;
+  gp.sa2 = a.sus;
+  gp.sb = xs;
+  gp.out = gemm::EpiOut{a.I, nullptr, hq, hs};
+  gp.err = a.err;
+  {
+    StqTimed tm(STQ_K_SHARED_GATE_UP, s);
+    st = launch_nt<true, true>(nt, mg, mu, mx, gp, s);
+  }
+  if (st != STQ_OK) return st;
+  GemmProblem dp = gp;
+  dp.tiles.R = a.H;
+  dp.tiles.max_items = ntile * (a.H / 128);
+  dp.K = a.I;
+  dp.sa = a.sds;
+  dp.sa2 = nullptr;
+  dp.sb = hs;
+  dp.out = gemm::EpiOut{a.H, a.Y + size_t(P) * a.H, nullptr, nullptr};
+  StqTimed tm(STQ_K_SHARED_DOWN, s);
+  return launch_nt<false, true>(nt, md, md, mh, dp, s);
 }
 
 extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales, int64_t N, int64_t K,

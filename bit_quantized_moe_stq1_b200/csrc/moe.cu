@@ -567,10 +567,10 @@ MoeWsLayout moe_ws_layout(const moe_desc& d) {
   L.inv = take(P * 4);
   L.h = take((P + T) * I * 2);
   L.Y = take((P + T) * H * 4);
-  L.xq = take(P * H);
-  L.xs = take(P * (H / 32));
-  L.hq = take(P * I);
-  L.hs = take(P * (I / 32));
+  L.xq = take((P + T) * H);
+  L.xs = take((P + T) * (H / 32));
+  L.hq = take((P + T) * I);
+  L.hs = take((P + T) * (I / 32));
   L.ntiles = take((P / 16 + E + 1) * 8);
   L.n_ntiles = take(4);
   L.sched = take(16);
@@ -701,6 +701,15 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   STQ_HOST_CHECK(w->gate && w->up && w->down, STQ_ERR_INVALID_ARG);
   const bool has_shared = w->sh_gate != nullptr;
   STQ_HOST_CHECK(!has_shared || (w->sh_up && w->sh_down), STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(!has_shared || w->sh_fmt == STQ_SHARED_BF16 || w->sh_fmt == STQ_SHARED_MXFP8, STQ_ERR_INVALID_ARG);
+  const bool shared_bf16 = has_shared && w->sh_fmt == STQ_SHARED_BF16;
+  const bool shared_mx8 = has_shared && w->sh_fmt == STQ_SHARED_MXFP8;
+  if (shared_mx8) {
+    STQ_HOST_CHECK(w->sh_gate_sc && w->sh_up_sc && w->sh_down_sc, STQ_ERR_INVALID_ARG);
+    STQ_HOST_CHECK(((reinterpret_cast<uintptr_t>(w->sh_gate_sc) | reinterpret_cast<uintptr_t>(w->sh_up_sc) |
+                     reinterpret_cast<uintptr_t>(w->sh_down_sc)) & 3u) == 0,
+                   STQ_ERR_ALIGN);
+  }
   STQ_HOST_CHECK(d->H % 256 == 0 && d->I % 256 == 0, STQ_ERR_SHAPE);
   if (w->fmt == STQ_FMT_MXFP4) STQ_HOST_CHECK(w->gate_sc && w->up_sc && w->down_sc, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(y) && stq_aligned16(w->gate) && stq_aligned16(w->up) &&
@@ -723,7 +732,16 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   a.x = x;
   a.wg = w->gate; a.wu = w->up; a.wd = w->down;
   a.gsc = w->gate_sc; a.usc = w->up_sc; a.dsc = w->down_sc;
-  a.sg = w->sh_gate; a.su = w->sh_up; a.sd = w->sh_down;
+  if (shared_bf16) {
+    a.sg = static_cast<const uint16_t*>(w->sh_gate);
+    a.su = static_cast<const uint16_t*>(w->sh_up);
+    a.sd = static_cast<const uint16_t*>(w->sh_down);
+  } else if (shared_mx8) {
+    a.sgq = static_cast<const uint8_t*>(w->sh_gate);
+    a.suq = static_cast<const uint8_t*>(w->sh_up);
+    a.sdq = static_cast<const uint8_t*>(w->sh_down);
+    a.sgs = w->sh_gate_sc; a.sus = w->sh_up_sc; a.sds = w->sh_down_sc;
+  }
   a.counts = ws.counts; a.offsets = ws.offsets; a.perm = ws.perm; a.tlist = ws.tlist; a.ntouched = ws.ntouched;
   a.h = ws.h; a.Y = ws.Y;
   a.xq = ws.xq; a.xs = ws.xs; a.hq = ws.hq; a.hs = ws.hs;
@@ -736,17 +754,18 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
                        (d->regime == STQ_REGIME_AUTO && P >= kStqPrefillTokensPerExpert * slots);
   if (w->fmt == STQ_FMT_STQ1_0 && prefill) {
     if ((st = moe_stq_prefill_experts(a, slots, s)) != STQ_OK) return st;
-    if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
+    if (shared_bf16 && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
   } else if (w->fmt == STQ_FMT_STQ1_0) {
+    // the BF16 shared expert's tiles are the first work items of the two GEMV kernels
     a.routed = 1;
-    a.n_shared_cta = has_shared ? d->I / 16 : 0;
+    a.n_shared_cta = shared_bf16 ? d->I / 16 : 0;
     a.sched = ws.sched;
     {
       StqTimed tm(STQ_K_GATE_UP, s);
       moe_gateup_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->I / 128))), 128, 0, s>>>(a);
     }
     if ((st = stq_launch_status()) != STQ_OK) return st;
-    a.n_shared_cta = has_shared ? d->H / 16 : 0;
+    a.n_shared_cta = shared_bf16 ? d->H / 16 : 0;
     a.sched = ws.sched + 1;
     {
       StqTimed tm(STQ_K_DOWN, s);
@@ -754,9 +773,10 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     }
     if ((st = stq_launch_status()) != STQ_OK) return st;
   } else {
-    st = moe_mx_experts(a, slots, has_shared, s);
+    st = moe_mx_experts(a, slots, shared_bf16, s);
     if (st != STQ_OK) return st;
   }
+  if (shared_mx8 && (st = moe_shared_expert_mx8(a, s)) != STQ_OK) return st;
   return moe_launch_combine(*d, P, ws, topk_w, has_shared, x, y, s);
 }
 

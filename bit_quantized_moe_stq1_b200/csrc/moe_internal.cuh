@@ -18,10 +18,10 @@ struct MoeWs {
   int32_t* inv;
   uint16_t* h;   // [(P+T), I] bf16: routed pairs (sorted order) then shared-expert tokens
   float* Y;      // [(P+T), H] fp32
-  uint8_t* xq;   // [P, H]     MXFP8 codes of x, rows in sorted pair order (MXFP4 experts)
-  uint8_t* xs;   // [P, H/32]
-  uint8_t* hq;   // [P, I]     MXFP8 codes of h (MXFP4 experts)
-  uint8_t* hs;   // [P, I/32]
+  uint8_t* xq;   // [(P+T), H] MXFP8 codes of x: routed pairs in sorted order, then the tokens
+  uint8_t* xs;   // [(P+T), H/32]
+  uint8_t* hq;   // [(P+T), I] MXFP8 codes of h, same rows
+  uint8_t* hs;   // [(P+T), I/32]
   int2* ntiles;  // [P/16 + E] (expert, first token) of each GEMM N tile
   int32_t* n_ntiles;
   int32_t* sched;  // [4] work counters of the persistent GEMV kernels (zeroed by the permute kernel)
@@ -34,6 +34,8 @@ struct MoeArgs {
   const uint8_t *wg, *wu, *wd;     // routed experts (STQ1_0 bytes or MXFP4 codes)
   const uint8_t *gsc, *usc, *dsc;  // MXFP4 scales
   const uint16_t *sg, *su, *sd;    // shared expert, bf16
+  const uint8_t *sgq, *suq, *sdq;  // shared expert, MXFP8 codes
+  const uint8_t *sgs, *sus, *sds;  // and scales
   const int32_t *counts, *offsets, *perm, *tlist, *ntouched;
   uint16_t* h;
   float* Y;
@@ -57,6 +59,10 @@ stq_status stq_tile_plan_launch(const int32_t* counts, int E, int nt, int2* tile
 
 // The BF16 shared expert on its own (gate/up, SwiGLU, down into the rows P.. of h and Y).
 stq_status moe_shared_expert_bf16(const MoeArgs& a, cudaStream_t s);
+
+// The MXFP8 shared expert (gemm_mx.cu): x -> MXFP8 rows P.. of xq/xs, gate/up + SwiGLU
+// into MXFP8 rows P.. of hq/hs, down into rows P.. of Y.
+stq_status moe_shared_expert_mx8(const MoeArgs& a, cudaStream_t s);
 
 // Routed STQ1_0 experts in the prefill regime (gemm_stq.cu): activations quantised to
 // MXFP8 in sorted pair order, gate/up + SwiGLU into MXFP8 h, down into Y.

@@ -209,6 +209,16 @@ stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router,
                                   int32_t T, int32_t H, int32_t E, int32_t k,
                                   int32_t* topk_ids, float* topk_w, stq_stream_t stream);
 
+/* Format of the shared expert (moe_weights.sh_fmt).
+ *   STQ_SHARED_BF16   sh_gate / sh_up / sh_down are bf16 matrices; h is rounded to bf16.
+ *   STQ_SHARED_MXFP8  "Hy4-preview-SF-WFP4AFP8", "Quant Diff": the shared experts'
+ *                     gate/up/down are MXFP8 W8A8 g32.  sh_* are E4M3 codes (one byte
+ *                     per weight, row-major) and sh_*_sc their UE8M0 scales [rows][K/32]
+ *                     (as written by mxfp8_quantize_bf16); x and h are quantised to
+ *                     MXFP8 g32 (the activation rule of mxfp8_quantize_bf16) and the
+ *                     products accumulate in FP32. */
+enum { STQ_SHARED_BF16 = 0, STQ_SHARED_MXFP8 = 1 };
+
 typedef struct {
   int32_t fmt;              /* STQ_FMT_STQ1_0 or STQ_FMT_MXFP4 (routed experts) */
   const uint8_t* gate;      /* E matrices [I, H], expert-major, contiguous      */
@@ -217,9 +227,13 @@ typedef struct {
   const uint8_t* gate_sc;   /* MXFP4 scales, E x [I, H/32]; NULL for STQ1_0      */
   const uint8_t* up_sc;     /* E x [I, H/32]                                     */
   const uint8_t* down_sc;   /* E x [H, I/32]                                     */
-  const uint16_t* sh_gate;  /* shared expert, bf16 [I, H]; NULL = no shared      */
-  const uint16_t* sh_up;    /* bf16 [I, H]                                       */
-  const uint16_t* sh_down;  /* bf16 [H, I]                                       */
+  const void* sh_gate;      /* shared expert [I, H] (sh_fmt); NULL = no shared   */
+  const void* sh_up;        /* [I, H]                                            */
+  const void* sh_down;      /* [H, I]                                            */
+  int32_t sh_fmt;           /* STQ_SHARED_BF16 (0) or STQ_SHARED_MXFP8           */
+  const uint8_t* sh_gate_sc;  /* MXFP8 scales [I, H/32]; NULL for BF16           */
+  const uint8_t* sh_up_sc;    /* [I, H/32]                                       */
+  const uint8_t* sh_down_sc;  /* [H, I/32]                                       */
 } moe_weights;
 
 /* Kernels for STQ1_0 routed experts (moe_desc.regime; MXFP4 experts have one path).
@@ -246,9 +260,9 @@ size_t moe_workspace_bytes(const moe_desc* d);
 
 /* y[t] = sum_s topk_w[t,s] * FFN_{topk_ids[t,s]}(x[t]) + FFN_shared(x[t]) (+ x[t])
  * with FFN_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x)).  The intermediate h is
- * rounded to bf16 (STQ1_0 decode regime and the shared expert) or re-quantised to
- * MXFP8 (MXFP4 experts and the STQ1_0 prefill regime, whose input x is quantised to
- * MXFP8 first).  Slots are summed in order
+ * rounded to bf16 (STQ1_0 decode regime and the BF16 shared expert) or re-quantised
+ * to MXFP8 (MXFP4 experts, the STQ1_0 prefill regime and the MXFP8 shared expert,
+ * whose input x is quantised to MXFP8 first).  Slots are summed in order
  * s = 0..k-1, without atomics.  Duplicate ids in a token are separate slots; an
  * id outside [0, E) sets STQ_ERR_DEVICE in the workspace error word and its slot
  * contributes 0.  workspace: >= moe_workspace_bytes(d) bytes, 256-B aligned. */
@@ -262,9 +276,10 @@ stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x,
  *   STQ_WS_COUNTS, _OFFSETS, _PERM, _INV, _TLIST, _NTOUCHED: as moe_permute;
  *   STQ_WS_H   bf16 [(P+T), I]: h of routed pairs (sorted order), then shared tokens;
  *   STQ_WS_Y   f32  [(P+T), H]: expert outputs, same row order (unweighted);
- *   STQ_WS_XQ/_XS  MXFP8 of x [P, H] / [P, H/32], rows in sorted pair order
- *                  (MXFP4 layers, STQ1_0 prefill regime);
- *   STQ_WS_HQ/_HS  MXFP8 of h [P, I] / [P, I/32] (same layers).
+ *   STQ_WS_XQ/_XS  MXFP8 of x [(P+T), H] / [(P+T), H/32]: routed pairs in sorted
+ *                  order (MXFP4 layers, STQ1_0 prefill regime), then the T tokens
+ *                  (MXFP8 shared expert);
+ *   STQ_WS_HQ/_HS  MXFP8 of h [(P+T), I] / [(P+T), I/32], same row order.
  * P = T*k.  Returns (size_t)-1 for an invalid descriptor or region. */
 enum { STQ_WS_COUNTS = 0, STQ_WS_OFFSETS, STQ_WS_PERM, STQ_WS_INV, STQ_WS_TLIST,
        STQ_WS_NTOUCHED, STQ_WS_H, STQ_WS_Y, STQ_WS_XQ, STQ_WS_XS, STQ_WS_HQ, STQ_WS_HS };

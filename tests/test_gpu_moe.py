@@ -10,7 +10,7 @@ import torch
 import workloads as W
 from oracle import formats as F
 from oracle import moe as M
-from mx_checks import check_mxfp8_layer
+from mx_checks import check_mx8_shared, check_mxfp8_layer
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -112,7 +112,8 @@ def _make_layer(S, T, H, I, E, k, shared, tag):
     return gw, packs, sh, wr, x
 
 
-def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None, x=None, regime=None):
+def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None, x=None, regime=None,
+               shared_fmt="bf16"):
     gw, packs, sh, wr, x0 = _make_layer(S, T, H, I, E, k, shared, tag)
     x = x0 if x is None else x
     if ids is None:
@@ -121,8 +122,15 @@ def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None,
     desc = S.make_desc(T, H, I, E, k, out_fp32=True, add_residual=residual, regime=regime)
     ws = torch.zeros(S.moe_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
     y = torch.empty((T, H), dtype=torch.float32, device=DEV)
-    ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, *(None, None, None),
-                         *(sh if sh else (None, None, None)))
+    sh_mx8 = None
+    if sh and shared_fmt == "mx8":
+        sh_mx8 = [S.mxfp8_quantize_bf16(m) for m in sh]
+        ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, None, None, None, *(c for c, _ in sh_mx8),
+                             sh_fmt=S.SHARED_MXFP8, sh_gate_sc=sh_mx8[0][1], sh_up_sc=sh_mx8[1][1],
+                             sh_down_sc=sh_mx8[2][1])
+    else:
+        ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, *(None, None, None),
+                             *(sh if sh else (None, None, None)))
     S.moe_expert_forward(desc, x, ids, tw, ew, y, ws)
     assert S.moe_get_device_error(ws) == 0
     P = T * k
@@ -132,10 +140,11 @@ def _run_layer(S, T, H, I, E, k, shared, tag, residual=False, ids=None, tw=None,
         perm=S.moe_workspace_view(desc, ws, "perm", torch.int32, (P,)).cpu().numpy(),
         inv=S.moe_workspace_view(desc, ws, "inv", torch.int32, (P,)).cpu().numpy(),
         offsets=S.moe_workspace_view(desc, ws, "offsets", torch.int32, (E + 1,)).cpu().numpy(),
-        xq=S.moe_workspace_view(desc, ws, "xq", torch.uint8, (P, H)).cpu().numpy(),
-        xs=S.moe_workspace_view(desc, ws, "xs", torch.uint8, (P, H // 32)).cpu().numpy(),
-        hq=S.moe_workspace_view(desc, ws, "hq", torch.uint8, (P, I)).cpu().numpy(),
-        hs=S.moe_workspace_view(desc, ws, "hs", torch.uint8, (P, I // 32)).cpu().numpy(),
+        xq=S.moe_workspace_view(desc, ws, "xq", torch.uint8, (P + T, H)).cpu().numpy(),
+        xs=S.moe_workspace_view(desc, ws, "xs", torch.uint8, (P + T, H // 32)).cpu().numpy(),
+        hq=S.moe_workspace_view(desc, ws, "hq", torch.uint8, (P + T, I)).cpu().numpy(),
+        hs=S.moe_workspace_view(desc, ws, "hs", torch.uint8, (P + T, I // 32)).cpu().numpy(),
+        sh_mx8=None if sh_mx8 is None else [(c.cpu().numpy(), s_.cpu().numpy()) for c, s_ in sh_mx8],
     )
     return dict(gw=gw, sh=sh, x=x, ids=ids.cpu().numpy(), tw=tw.cpu().double().numpy(), y=y.cpu().double().numpy(),
                 **st)
@@ -177,7 +186,9 @@ def _check_layer(r, T, H, I, E, k, experts=None):
         Wd = gw[2][e * H:(e + 1) * H].double().cpu().numpy()
         _check_gate_up(Wg, Wu, xd[toks], r["h"][pos])
         _check_down(Wd, r["h"][pos], r["Y"][pos])
-    if r["sh"] is not None:
+    if r["sh_mx8"] is not None:
+        check_mx8_shared(r, T, H, I, P)
+    elif r["sh"] is not None:
         sg, su, sd = (m.float().double().cpu().numpy() for m in r["sh"])
         _check_gate_up(sg, su, xd, r["h"][P:P + T])
         _check_down(sd, r["h"][P:P + T], r["Y"][P:P + T])
@@ -256,6 +267,22 @@ def test_moe_stq_prefill_wide_range_activations(S):
     ids, tw = W.uniform_routing(T, E, k, DEV, 0, "wide-pf", "ids")
     r = _run_layer(S, T, H, I, E, k, True, "wide-pf", ids=ids, tw=tw, x=x, regime=S.REGIME_PREFILL)
     _check_prefill(r, T, H, I, E, k)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,regime", [(5, 512, 256, 8, 2, "decode"), (8, 6144, 2048, 256, 8, "decode"),
+                                               (200, 768, 512, 4, 3, "prefill"), (17, 512, 512, 2, 2, "decode")])
+def test_moe_stq_mxfp8_shared(S, T, H, I, E, k, regime):
+    """STQ1_0 layers with the MXFP8 shared expert, decode and prefill regimes (the
+    decode config's shape included; routed experts sampled there)."""
+    reg = S.REGIME_DECODE if regime == "decode" else S.REGIME_PREFILL
+    r = _run_layer(S, T, H, I, E, k, True, ("sh8", T, H, I, E, k), regime=reg, shared_fmt="mx8")
+    counts = np.bincount(r["ids"].reshape(-1), minlength=E)
+    touched = np.flatnonzero(counts)
+    sample = touched if touched.size <= 8 else touched[:: touched.size // 4]
+    if regime == "decode":
+        _check_layer(r, T, H, I, E, k, experts=sample)
+    else:
+        _check_prefill(r, T, H, I, E, k, experts=sample)
 
 
 def test_moe_stq_auto_regime_threshold(S):

@@ -65,7 +65,7 @@ def test_w4a8_gemm_zero_and_empty(S):
 
 # --------------------------------------------------------------------------- MXFP4 MoE layer
 
-def _mx_layer(S, T, H, I, E, k, shared, tag, routing="router"):
+def _mx_layer(S, T, H, I, E, k, shared, tag, routing="router", shared_fmt="bf16"):
     g = [W.mxfp4_random(E * I, H, DEV, 0, tag, "g"), W.mxfp4_random(E * I, H, DEV, 0, tag, "u"),
          W.mxfp4_random(E * H, I, DEV, 0, tag, "d")]
     sh = None
@@ -81,16 +81,24 @@ def _mx_layer(S, T, H, I, E, k, shared, tag, routing="router"):
     desc = S.make_desc(T, H, I, E, k, out_fp32=True)
     ws = torch.zeros(S.moe_workspace_bytes(desc), dtype=torch.uint8, device=DEV)
     y = torch.empty((T, H), dtype=torch.float32, device=DEV)
-    ew = S.ExpertWeights(S.FMT_MXFP4, g[0][0], g[1][0], g[2][0], g[0][1], g[1][1], g[2][1],
-                         *(sh if sh else (None, None, None)))
+    sh_mx8 = None
+    if sh and shared_fmt == "mx8":
+        sh_mx8 = [S.mxfp8_quantize_bf16(m) for m in sh]
+        ew = S.ExpertWeights(S.FMT_MXFP4, g[0][0], g[1][0], g[2][0], g[0][1], g[1][1], g[2][1],
+                             *(c for c, _ in sh_mx8), sh_fmt=S.SHARED_MXFP8, sh_gate_sc=sh_mx8[0][1],
+                             sh_up_sc=sh_mx8[1][1], sh_down_sc=sh_mx8[2][1])
+    else:
+        ew = S.ExpertWeights(S.FMT_MXFP4, g[0][0], g[1][0], g[2][0], g[0][1], g[1][1], g[2][1],
+                             *(sh if sh else (None, None, None)))
     S.moe_expert_forward(desc, x, ids, tw, ew, y, ws)
     assert S.moe_get_device_error(ws) == 0
     P = T * k
     v = lambda r, dt, shp: S.moe_workspace_view(desc, ws, r, dt, shp).cpu().numpy()
     return dict(g=[(a.cpu().numpy(), b.cpu().numpy()) for a, b in g], sh=sh, x=x, ids=ids.cpu().numpy(),
                 tw=tw.cpu().double().numpy(), y=y.cpu().double().numpy(),
-                xq=v("xq", torch.uint8, (P, H)), xs=v("xs", torch.uint8, (P, H // 32)),
-                hq=v("hq", torch.uint8, (P, I)), hs=v("hs", torch.uint8, (P, I // 32)),
+                xq=v("xq", torch.uint8, (P + T, H)), xs=v("xs", torch.uint8, (P + T, H // 32)),
+                hq=v("hq", torch.uint8, (P + T, I)), hs=v("hs", torch.uint8, (P + T, I // 32)),
+                sh_mx8=None if sh_mx8 is None else [(c.cpu().numpy(), s_.cpu().numpy()) for c, s_ in sh_mx8],
                 h=S.moe_workspace_view(desc, ws, "h", torch.bfloat16, (P + T, I)).float().cpu().double().numpy(),
                 Y=v("Y", torch.float32, (P + T, H)).astype(np.float64),
                 perm=v("perm", torch.int32, (P,)), inv=v("inv", torch.int32, (P,)))
@@ -112,6 +120,13 @@ def _check_mx_layer(r, T, H, I, E, k, experts=None):
                                                (40, 512, 256, 4, 4, False)])
 def test_moe_mx_small_full_check(S, T, H, I, E, k, shared):
     r = _mx_layer(S, T, H, I, E, k, shared, ("mxs", T, H, I, E, k))
+    _check_mx_layer(r, T, H, I, E, k)
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [(5, 512, 256, 8, 2), (40, 512, 256, 4, 4), (300, 768, 512, 8, 2)])
+def test_moe_mx_mxfp8_shared_full_check(S, T, H, I, E, k):
+    """MXFP4 layer with the MXFP8 shared expert (N tiles of 16 to 128 tokens)."""
+    r = _mx_layer(S, T, H, I, E, k, True, ("mxsh8", T, H, I, E, k), shared_fmt="mx8")
     _check_mx_layer(r, T, H, I, E, k)
 
 

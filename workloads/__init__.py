@@ -38,6 +38,7 @@ class Workload:
     router: bool            # BF16 router (else Zipf routing)
     shared: bool            # shared BF16 expert
     residual: bool
+    shared_fmt: str = "bf16"  # shared expert storage: "bf16" or "mx8" (MXFP8 W8A8 g32)
     H: int = HIDDEN
     I: int = INTER
     E: int = EXPERTS
@@ -48,6 +49,7 @@ WORKLOADS = {
     "stq_matvec": Workload("stq_matvec", 1, 1, ("stq",), False, False, False, E=1, k=1),
     "w4a8_gemm": Workload("w4a8_gemm", 128, 1, ("mx",), False, False, False, E=1, k=1),
     "decode_stq": Workload("decode_stq", 8, 1, ("stq",), True, True, False),
+    "decode_stq_sh8": Workload("decode_stq_sh8", 8, 1, ("stq",), True, True, False, shared_fmt="mx8"),
     "prefill_w4a8": Workload("prefill_w4a8", 4096, 1, ("mx",), False, False, False),
     "prefill_stq": Workload("prefill_stq", 4096, 1, ("stq",), False, False, False),
     "stacked_decode": Workload("stacked_decode", 32, 8, ("stq", "mx") * 4, True, True, True),
