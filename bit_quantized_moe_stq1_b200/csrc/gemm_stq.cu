@@ -17,7 +17,8 @@
 //
 // Warp roles (448 threads, one CTA per SM, persistent over work items):
 //   warp 0       TMA of the activation tile (two 128-k boxes, 128-byte swizzle) and its
-//                scale factors, re-laid into the scale-factor atoms the MMA reads;
+//                scale factors (loaded four stages ahead into a register ring), re-laid
+//                into the scale-factor atoms the MMA reads;
 //   warp 1       TMEM allocation and, from one thread, tcgen05.cp of the scales and the
 //                eight K = 32 MMAs of a stage into the partial buffer of the block;
 //   warps 2-5    promotion: acc += d * partial, TMEM to TMEM through registers;
@@ -51,6 +52,7 @@ constexpr int kSmem = kStages * kStage + kUBuf + kSf /* unit weight scales */ + 
 constexpr uint32_t kTxB = 2 * kSubB;     // bytes the TMA delivers per stage
 constexpr int kThreads = 448;
 constexpr int kDecodeWarp0 = 10;
+constexpr int kDecodeWarps = 4;
 constexpr int kColP = 0;                 // partial buffers: kColP + 128 * i
 constexpr int kColAcc = 256;             // accumulators: kColAcc + 128 * i
 constexpr int kColSfa = 112;
@@ -143,25 +145,39 @@ __device__ __forceinline__ uint4 decode_chunk(const TileWords& t, uint32_t lut) 
 
 // Write the tile-block of A-tile rows 16j.. into the stage's A sub-tiles.  Lane (g, t)
 // holds rows 16j + g and 16j + g + 8, k = 64t .. 64t + 63 of the block: sub-tile t / 2,
-// 16-byte chunks 4 (t % 2) + c4 of the 128-byte row, stored at chunk (chunk ^ row % 8).
+// 16-byte chunks 4 (t % 2) + c of the 128-byte row, stored at chunk (chunk ^ row % 8).
+// Lanes t and t + 2 would hit the same banks (the sub-tiles are 16 KB apart), so lanes
+// t >= 2 rotate their 160-bit code stream by 80 bits: their c-th store then holds chunk
+// c ^ 2, and the eight lanes of each store phase cover eight distinct 16-byte bank groups.
 template <int H, int C4>
-__device__ __forceinline__ void put_chunk(uint8_t* a_stage, const TileWords& t, uint32_t lut, int j, int lane) {
-  const int g = lane >> 2, tq = lane & 3;
-  const int r = 16 * j + g + 8 * H;
-  const int chunk = 4 * (tq & 1) + C4;
-  uint8_t* dst = a_stage + (tq >> 1) * kSubA + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
-  *reinterpret_cast<uint4*>(dst) = decode_chunk<H, C4>(t, lut);
+__device__ __forceinline__ void put_chunk(uint8_t* row_base, const TileWords& t, uint32_t lut, int cbase, int sw,
+                                          int g) {
+  const int chunk = cbase + (C4 ^ sw);
+  *reinterpret_cast<uint4*>(row_base + H * 1024 + ((chunk ^ g) << 4)) = decode_chunk<H, C4>(t, lut);
 }
 
-__device__ __forceinline__ void put_tile_block(uint8_t* a_stage, const TileWords& t, uint32_t lut, int j, int lane) {
-  put_chunk<0, 0>(a_stage, t, lut, j, lane);
-  put_chunk<0, 1>(a_stage, t, lut, j, lane);
-  put_chunk<0, 2>(a_stage, t, lut, j, lane);
-  put_chunk<0, 3>(a_stage, t, lut, j, lane);
-  put_chunk<1, 0>(a_stage, t, lut, j, lane);
-  put_chunk<1, 1>(a_stage, t, lut, j, lane);
-  put_chunk<1, 2>(a_stage, t, lut, j, lane);
-  put_chunk<1, 3>(a_stage, t, lut, j, lane);
+__device__ __forceinline__ void put_tile_block(uint8_t* a_stage, const TileWords& in, uint32_t lut, int j, int lane) {
+  const int g = lane >> 2, tq = lane & 3;
+  const bool up = tq >= 2;
+  TileWords t;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    // bits [32k + 80, 32k + 112) mod 160 of the stream
+    const uint32_t rot = __funnelshift_r(in.w[(k + 2) % 5], in.w[(k + 3) % 5], 16);
+    t.w[k] = up ? rot : in.w[k];
+  }
+  const int sw = up ? 2 : 0;
+  const int cbase = 4 * (tq & 1);
+  // rows 16j + g (H = 0) and 16j + g + 8 (H = 1: one 1024-byte 8-row group further)
+  uint8_t* row_base = a_stage + (up ? kSubA : 0) + (2 * j) * 1024 + g * 128;
+  put_chunk<0, 0>(row_base, t, lut, cbase, sw, g);
+  put_chunk<0, 1>(row_base, t, lut, cbase, sw, g);
+  put_chunk<0, 2>(row_base, t, lut, cbase, sw, g);
+  put_chunk<0, 3>(row_base, t, lut, cbase, sw, g);
+  put_chunk<1, 0>(row_base, t, lut, cbase, sw, g);
+  put_chunk<1, 1>(row_base, t, lut, cbase, sw, g);
+  put_chunk<1, 2>(row_base, t, lut, cbase, sw, g);
+  put_chunk<1, 3>(row_base, t, lut, cbase, sw, g);
 }
 
 }  // namespace
@@ -178,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* ubuf = reinterpret_cast<float*>(smem + kStages * kStage);
   uint8_t* sfa_unit = smem + kStages * kStage + kUBuf;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sfa_unit + kSf);  // [kStages]: TMA bytes + 5 arrivals
+  uint64_t* full = reinterpret_cast<uint64_t*>(sfa_unit + kSf);  // [kStages]: TMA bytes + 3 arrivals
   uint64_t* empty = full + kStages;                              // [kStages]: MMAs of the stage done
   uint64_t* pfull = empty + kStages;                             // [2]: partial written
   uint64_t* pempty = pfull + 2;                                  // [2]: partial promoted (4 warps)
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 5);
+      tc::mbar_init(&full[s], 1 + kDecodeWarps);
       tc::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -219,27 +235,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------------- activation loads
+    // The scale factors of a stage are global loads that the warp must re-lay before the
+    // stage can start; a register ring holds them kLook stages ahead (a second cursor
+    // walks the same item/block sequence), so their latency overlaps earlier stages.
+    constexpr int kLook = 4;
     const int k32 = p.K / 32, nk = p.K / 128;
     int last_round[kStages];
 #pragma unroll
     for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+    Item J = gemm::get_item(p.tiles, blockIdx.x, MT, kRows, kNT);
+    int itJ = 0, kbJ = 0;
+    uint32_t ring[kLook][2][4];
+    auto load_next = [&](uint32_t (&v)[2][4]) {
+      const int nkj = J.valid ? nk : 0;  // past the last item: zeros, no loads
+      gemm::load_sf(v[0], p.sb, J.brow, kNT, p.Ptot, k32, 2 * kbJ, nkj, lane);
+      gemm::load_sf(v[1], p.sb, J.brow, kNT, p.Ptot, k32, 2 * kbJ + 1, nkj, lane);
+      if (J.valid && ++kbJ == nb) {
+        kbJ = 0;
+        ++itJ;
+        J = gemm::get_item(p.tiles, blockIdx.x + itJ * G, MT, kRows, kNT);
+      }
+    };
+#pragma unroll
+    for (int d = 0; d < kLook; ++d) load_next(ring[d]);
+    Item I = gemm::get_item(p.tiles, blockIdx.x, MT, kRows, kNT);
+    int it = 0, kb = 0, g = 0;
     bool ok = true;
-    int g = 0;
-    for (int it = 0; ok; ++it) {
-      const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
-      if (!I.valid) break;
-      for (int kb = 0; kb < nb; ++kb, ++g) {
+    while (ok && I.valid) {
+#pragma unroll
+      for (int d = 0; d < kLook; ++d) {
+        if (!ok || !I.valid) break;
         const int s = g % kStages, r = g / kStages;
-        uint32_t v0[4], v1[4];
-        gemm::load_sf(v0, p.sb, I.brow, kNT, p.Ptot, k32, 2 * kb, nk, lane);
-        gemm::load_sf(v1, p.sb, I.brow, kNT, p.Ptot, k32, 2 * kb + 1, nk, lane);
         if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
           ok = false;
           break;
         }
         uint8_t* st = smem + s * kStage;
-        gemm::store_sf(st + kOffSfb, v0, lane);
-        gemm::store_sf(st + kOffSfb + kSf, v1, lane);
+        gemm::store_sf(st + kOffSfb, ring[d][0], lane);
+        gemm::store_sf(st + kOffSfb + kSf, ring[d][1], lane);
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -248,6 +281,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc::tma_load_2d(st + kOffB + kSubB, &tmB, kb * 256 + 128, I.brow, &full[s]);
         }
         last_round[s] = r;
+        load_next(ring[d]);  // the stage kLook steps ahead
+        ++g;
+        if (++kb == nb) {
+          kb = 0;
+          ++it;
+          I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
+        }
       }
     }
     // every load this warp issued has landed before the CTA may exit
@@ -260,8 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
-        const int item = blockIdx.x + it * G;
-        if (item >= p.tiles.max_items || (p.tiles.offsets != nullptr && item / MT >= *p.tiles.n_ntiles)) break;
+        const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
+        if (!I.valid) break;
+        const uint32_t idesc_n = uint32_t(gemm::item_cols(I, kNT));
         for (int kb = 0; kb < nb; ++kb, ++g) {
           const int s = g % kStages, r = g / kStages, pb = g & 1, pr = g >> 1;
           if (pr > 0 && !tc::mbar_wait(&pempty[pb], (pr - 1) & 1, p.err)) {
@@ -282,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int h = kk >> 2, j = kk & 3;
             const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + kOffA + h * kSubA)) + 2 * j;
             const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + kOffB + h * kSubB)) + 2 * j;
-            const uint32_t idesc = tc::idesc_mxf8f6f4_ab(kNT, tc::kFmtE4M3, tc::kFmtE4M3, 0u, uint32_t(j));
+            const uint32_t idesc = tc::idesc_mxf8f6f4_ab(int(idesc_n), tc::kFmtE4M3, tc::kFmtE4M3, 0u, uint32_t(j));
             tc::mma_mxf8f6f4(d_col, da, db, idesc, tmem + kColSfa, (tmem + uint32_t(kColSfb + 4 * h)) | (uint32_t(j) << 30),
                              kk > 0 ? 1u : 0u);
           }
@@ -307,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int abuf = it & 1, ar = it >> 1;
       if (ar > 0 && !tc::mbar_wait(&aempty[abuf], (ar - 1) & 1, p.err)) break;
       const uint32_t tacc = lane_base + uint32_t(kColAcc + 128 * abuf);
+      const int ncols = gemm::item_cols(I, kNT);  // columns the MMAs wrote
       const uint16_t* dp = d_ptr<PAIR>(p, I, m, 0);
       uint16_t dnext = __ldg(dp);
       for (int kb = 0; kb < nb; ++kb, ++g) {
@@ -320,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_after_sync();
         const uint32_t tp = lane_base + uint32_t(kColP + 128 * pb);
 #pragma unroll 1
-        for (int c0 = 0; c0 < kNT; c0 += 16) {
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
           uint32_t v[16], a[16];
           tc::tmem_ld_x16(tp + c0, v);
           if (kb > 0) {
@@ -365,13 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- decode
-    const int dw = warp - kDecodeWarp0;  // tile-blocks 2 dw, 2 dw + 1 of the A tile
+    constexpr int kTb = 8 / kDecodeWarps;  // tile-blocks per decoder warp
+    const int j0 = (warp - kDecodeWarp0) * kTb;
     const uint32_t lut = e4m3_lut_entry(uint32_t(lane));
     Item I = gemm::get_item(p.tiles, blockIdx.x, MT, kRows, kNT);
-    TileWords cur[2] = {}, nxt[2] = {};
+    TileWords cur[kTb] = {}, nxt[kTb] = {};
     if (I.valid) {
-      load_tile_words(cur[0], tile_block<PAIR>(p, I, 2 * dw, 0), lane);
-      load_tile_words(cur[1], tile_block<PAIR>(p, I, 2 * dw + 1, 0), lane);
+#pragma unroll
+      for (int i = 0; i < kTb; ++i) load_tile_words(cur[i], tile_block<PAIR>(p, I, j0 + i, 0), lane);
     }
     int g = 0;
     bool ok = true;
@@ -380,24 +423,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < nb; ++kb, ++g) {
         const int s = g % kStages, r = g / kStages;
         if (kb + 1 < nb) {
-          load_tile_words(nxt[0], tile_block<PAIR>(p, I, 2 * dw, kb + 1), lane);
-          load_tile_words(nxt[1], tile_block<PAIR>(p, I, 2 * dw + 1, kb + 1), lane);
+#pragma unroll
+          for (int i = 0; i < kTb; ++i) load_tile_words(nxt[i], tile_block<PAIR>(p, I, j0 + i, kb + 1), lane);
         } else if (In.valid) {
-          load_tile_words(nxt[0], tile_block<PAIR>(p, In, 2 * dw, 0), lane);
-          load_tile_words(nxt[1], tile_block<PAIR>(p, In, 2 * dw + 1, 0), lane);
+#pragma unroll
+          for (int i = 0; i < kTb; ++i) load_tile_words(nxt[i], tile_block<PAIR>(p, In, j0 + i, 0), lane);
         }
         if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
           ok = false;
           break;
         }
         uint8_t* a_stage = smem + s * kStage + kOffA;
-        put_tile_block(a_stage, cur[0], lut, 2 * dw, lane);
-        put_tile_block(a_stage, cur[1], lut, 2 * dw + 1, lane);
+#pragma unroll
+        for (int i = 0; i < kTb; ++i) put_tile_block(a_stage, cur[i], lut, j0 + i, lane);
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&full[s]);
-        cur[0] = nxt[0];
-        cur[1] = nxt[1];
+#pragma unroll
+        for (int i = 0; i < kTb; ++i) cur[i] = nxt[i];
       }
       I = In;
     }
