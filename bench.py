@@ -49,6 +49,9 @@ NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense
 # launch's traffic grows with its touched experts, so the full launch's traffic is this
 # figure times its touched experts.  An entry is removed when its kernel changes.
 MEASURED_TRAFFIC_PER_EXPERT = {}
+# DRAM bytes (read + write) of one full-size launch, from an ncu capture of the same workload
+# and kernel build; an entry is removed when its kernel changes.
+MEASURED_TRAFFIC_PER_LAUNCH = {("prefill_stq", "gate_up_stq_tc"): 1.608519e9 + 64.757248e6}
 
 
 def peaks():
@@ -514,6 +517,9 @@ def run_ours(args):
         touched = float(np.mean([a["per_kind"][dom]["touched"] for a in acct if dom in a["per_kind"]]))
         roof["traffic"] = MEASURED_TRAFFIC_PER_EXPERT[dom] * touched
         roof["traffic_source"] = "ncu dram bytes per touched expert (smaller case) x touched experts per launch"
+    if (wl.name, dom) in MEASURED_TRAFFIC_PER_LAUNCH:
+        roof["traffic"] = MEASURED_TRAFFIC_PER_LAUNCH[(wl.name, dom)]
+        roof["traffic_source"] = "ncu dram bytes of one full-size launch of this kernel"
     tps = wl.tokens_per_step()
     if wl.unit == "GB/s":
         value = whole_job_rate(n, ab, ms_step) / 1e9
