@@ -71,7 +71,7 @@ enum {
 const char* stq_status_string(stq_status s);
 
 /* ABI version of this header (bumped on any signature or layout change). */
-#define STQMOE_ABI_VERSION 1
+#define STQMOE_ABI_VERSION 2
 int32_t stq_abi_version(void);
 
 /* Synchronise `stream`, return the error word's value and reset it to 0.

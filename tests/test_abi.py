@@ -49,7 +49,7 @@ def test_binding_loads_and_host_side_calls(built):
 
     import bit_quantized_moe_stq1_b200 as S
 
-    assert S.lib.stq_abi_version() == 1
+    assert S.lib.stq_abi_version() == 2
     assert S.status_string(-2) == "STQ_ERR_SHAPE"
     for name in declared_functions():
         assert name in S.SIGNATURES, name
@@ -63,3 +63,103 @@ def test_binding_loads_and_host_side_calls(built):
     assert S.lib.stq1_gemv(ctypes.c_void_p(16), 16, 100, ctypes.c_void_p(16), 1, ctypes.c_void_p(16), None) == -2
     assert S.lib.stq1_gemv(ctypes.c_void_p(8), 16, 256, ctypes.c_void_p(16), 1, ctypes.c_void_p(16), None) == -3
     assert S.lib.mxfp8_quantize_bf16(ctypes.c_void_p(16), 4, 48, ctypes.c_void_p(16), ctypes.c_void_p(16), None) == -2
+
+
+C_LAYOUT = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "stqmoe.h"
+#define F(T, m) printf("%s.%s %zu %zu\n", #T, #m, offsetof(T, m), sizeof(((T*)0)->m))
+int main(void) {
+  printf("moe_desc %zu\nmoe_weights %zu\n", sizeof(moe_desc), sizeof(moe_weights));
+  F(moe_desc, T); F(moe_desc, H); F(moe_desc, I); F(moe_desc, E); F(moe_desc, k);
+  F(moe_desc, out_fp32); F(moe_desc, add_residual); F(moe_desc, regime);
+  F(moe_weights, fmt); F(moe_weights, gate); F(moe_weights, up); F(moe_weights, down);
+  F(moe_weights, gate_sc); F(moe_weights, up_sc); F(moe_weights, down_sc);
+  F(moe_weights, sh_gate); F(moe_weights, sh_up); F(moe_weights, sh_down); F(moe_weights, sh_fmt);
+  F(moe_weights, sh_gate_sc); F(moe_weights, sh_up_sc); F(moe_weights, sh_down_sc);
+  return 0;
+}
+"""
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The binding's ctypes structs have the C header's sizes and field offsets."""
+    import bit_quantized_moe_stq1_b200 as S
+
+    src = tmp_path / "layout.c"
+    src.write_text(C_LAYOUT)
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    lines = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    sizes = dict(l.split() for l in lines[:2])
+    assert int(sizes["moe_desc"]) == ctypes_size(S.MoeDesc)
+    assert int(sizes["moe_weights"]) == ctypes_size(S.MoeWeights)
+    for line in lines[2:]:
+        if not line:
+            continue
+        name, off, size = line.split()
+        struct, field = name.split(".")
+        cls = S.MoeDesc if struct == "moe_desc" else S.MoeWeights
+        desc = getattr(cls, field)
+        assert (desc.offset, desc.size) == (int(off), int(size)), name
+
+
+def ctypes_size(cls):
+    import ctypes
+    return ctypes.sizeof(cls)
+
+
+def test_moe_host_validation(built):
+    """Argument checks of moe_expert_forward and moe_workspace_bytes return before any launch:
+    regime and shared-expert format out of range, MXFP8 shared expert without scales or with
+    misaligned scales, workspace too small (fake, never dereferenced device pointers)."""
+    import ctypes
+
+    import bit_quantized_moe_stq1_b200 as S
+
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    y = P(1 << 21)
+    ws = P(1 << 22)
+
+    def call(desc, w, ws_bytes=1 << 40):
+        return S.lib.moe_expert_forward(ctypes.byref(desc), fake, fake, fake, ctypes.byref(w), y, ws, ws_bytes, None)
+
+    good = S.make_desc(4, 512, 256, 8, 2)
+    assert S.moe_workspace_bytes(good) > 0
+    bad_regime = S.make_desc(4, 512, 256, 8, 2, regime=3)
+    assert S.moe_workspace_bytes(bad_regime) == 0
+    w_stq = S.MoeWeights(S.FMT_STQ1_0, fake, fake, fake, None, None, None, None, None, None, 0, None, None, None)
+    assert call(bad_regime, w_stq) == -1  # STQ_ERR_INVALID_ARG
+    w_bad_fmt = S.MoeWeights(S.FMT_STQ1_0, fake, fake, fake, None, None, None, fake, fake, fake, 7, None, None, None)
+    assert call(good, w_bad_fmt) == -1
+    w_no_sc = S.MoeWeights(S.FMT_STQ1_0, fake, fake, fake, None, None, None, fake, fake, fake, S.SHARED_MXFP8,
+                           None, None, None)
+    assert call(good, w_no_sc) == -1
+    w_misaligned = S.MoeWeights(S.FMT_STQ1_0, fake, fake, fake, None, None, None, fake, fake, fake,
+                                S.SHARED_MXFP8, P((1 << 20) + 2), fake, fake)
+    assert call(good, w_misaligned) == -3  # STQ_ERR_ALIGN
+    w_mx8 = S.MoeWeights(S.FMT_STQ1_0, fake, fake, fake, None, None, None, fake, fake, fake, S.SHARED_MXFP8,
+                         fake, fake, fake)
+    assert call(good, w_mx8, ws_bytes=S.moe_workspace_bytes(good) - 1) == -7  # STQ_ERR_WORKSPACE
+
+
+def test_workspace_mxfp8_regions_hold_pairs_and_tokens(built):
+    """The MXFP8 regions of x and h have rows for the T*k routed pairs and the T tokens of
+    the shared expert, in the order the header states."""
+    import ctypes
+
+    import bit_quantized_moe_stq1_b200 as S
+
+    T, H, I, E, k = 37, 768, 512, 16, 4
+    d = S.make_desc(T, H, I, E, k)
+    P = T * k
+    off = {r: S.lib.moe_workspace_offset(ctypes.byref(d), i) for i, r in enumerate(S.WS_REGIONS)}
+    total = S.moe_workspace_bytes(d)
+    ends = sorted(off.values()) + [total]
+    room = {r: ends[ends.index(o) + 1] - o for r, o in off.items()}
+    assert room["xq"] >= (P + T) * H and room["xs"] >= (P + T) * H // 32
+    assert room["hq"] >= (P + T) * I and room["hs"] >= (P + T) * I // 32
+    assert room["h"] >= (P + T) * I * 2 and room["Y"] >= (P + T) * H * 4
+    assert all(o % 256 == 0 for o in off.values())
