@@ -34,9 +34,12 @@ constexpr int kATile = 128 * 128;                 // smem bytes of one 128 x 128
 constexpr uint32_t kATx = 128 * 128 / 2;          // bytes the TMA delivers for it
 constexpr int kSf = 512;                          // one scale-factor atom: 128 rows x 4 k-blocks
 // Two CTAs share an SM (half the shared memory each) unless the two accumulator buffers
-// of the 128-wide N tile need more than half of the SM's 512 TMEM columns.
+// of a wider N tile need more than half of the SM's 512 TMEM columns.  The 240-wide tile
+// (prefill) takes 4 stages of 48 KB.
 constexpr int ctas_per_sm(int nt) { return nt <= 64 ? 2 : 1; }
-constexpr int smem_budget(int nt) { return ctas_per_sm(nt) == 2 ? 112 * 1024 : 200 * 1024; }
+constexpr int smem_budget(int nt) {
+  return ctas_per_sm(nt) == 2 ? 112 * 1024 : nt > 128 ? 226 * 1024 : 200 * 1024;
+}
 
 // PAIR = the gate/up pair of one expert: the 128-row A tile holds 64 gate rows (TMEM
 // lanes 0-63) and the same 64 rows of the up projection (lanes 64-127), so one MMA per
@@ -45,11 +48,12 @@ constexpr int smem_budget(int nt) { return ctas_per_sm(nt) == 2 ? 112 * 1024 : 2
 template <int NT, bool PAIR, bool A8 = false>
 struct Cfg {
   static constexpr int kB = NT * 128;
+  static constexpr int kSfbAtoms = NT > 128 ? 2 : 1;   // activation scale factors: 128 rows per atom
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kATile;
   static constexpr int kOffSfa = kOffB + kB;
   static constexpr int kOffSfb = kOffSfa + kSf;
-  static constexpr int kStageRaw = kOffSfb + kSf;
+  static constexpr int kStageRaw = kOffSfb + kSfbAtoms * kSf;
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
   static constexpr int kCtasPerSm = ctas_per_sm(NT);
   static constexpr int kUBuf = PAIR ? 4 * 32 * 9 * 4 : 0;   // gate/up exchange of the epilogue (pitch 9 words)
@@ -60,16 +64,19 @@ struct Cfg {
   static constexpr int stages_of(int) { return kStages / 2; }
   static constexpr int kSmem = kStages * kStage + kUBuf + 1024 /* barriers */ + 1024 /* alignment */;
   static constexpr int kRowsPerTile = PAIR ? 64 : 128;   // output features per CTA
-  // TMEM: accumulator buffers at columns 0 and NT (tile i uses buffer i & 1), then the
-  // scale factors of the current k-block.
-  static constexpr int kColSfa = 2 * NT;
-  static constexpr int kColSfb = 2 * NT + 4;
-  static constexpr int kColsUsed = 2 * NT + 8;
+  // TMEM: accumulator buffers at columns 0 and kAccStride (tile i uses buffer i & 1), and
+  // the scale factors of the current k-block (after both buffers, or between them for the
+  // 240-wide tile: 240..243 weights, 244..251 the two activation atoms).
+  static constexpr int kAccStride = NT > 128 ? 256 : NT;
+  static constexpr int kColSfa = NT > 128 ? NT : 2 * NT;
+  static constexpr int kColSfb = kColSfa + 4;
+  static constexpr int kColsUsed = NT > 128 ? 256 + NT : 2 * NT + 4 + 4 * kSfbAtoms;
   static constexpr uint32_t kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
   static constexpr uint32_t kTx = (A8 ? uint32_t(kATile) : kATx) + uint32_t(kB);
   static_assert(kStages >= 2, "shared memory budget (one stage per producer at least)");
-  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "tile N");
+  static_assert(NT % 16 == 0 && NT >= 16 && (NT <= 128 || NT == 240), "tile N");
+  static_assert(NT <= 128 || kColSfb + 8 <= 256, "scale factors between the accumulators");
   static_assert(kCtasPerSm * kCols <= 512, "TMEM columns");
 };
 
@@ -160,7 +167,8 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
     // next item's first scale factors into the ring, so an item boundary costs no wait.
     const bool cross = nk % (2 * kPf) == 0;
     bool ok = true;
-    uint32_t ra[kPf][4], rb[kPf][4];
+    constexpr int kAt = C::kSfbAtoms;
+    uint32_t ra[kPf][4], rb[kPf][kAt][4];
     for (int it = 0; ok; ++it) {
       const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, C::kRowsPerTile, NT);
       if (!I.valid) break;
@@ -172,7 +180,9 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
         for (int d = 0; d < kPf; ++d) {
           if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, I.arow, k32, kt0 + 2 * d, nk, lane);
           else load_sf(ra[d], p.sa, I.arow, 128, 0x7fffffff, k32, kt0 + 2 * d, nk, lane);
-          load_sf(rb[d], p.sb, I.brow, NT, p.Ptot, k32, kt0 + 2 * d, nk, lane);
+#pragma unroll
+          for (int at = 0; at < kAt; ++at)
+            load_sf(rb[d][at], p.sb, I.brow + 128 * at, NT - 128 * at, p.Ptot, k32, kt0 + 2 * d, nk, lane);
         }
       }
       for (int k0 = kt0; k0 < nk && ok; k0 += 2 * kPf) {
@@ -188,7 +198,8 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
           }
           uint8_t* st = smem + s * C::kStage;
           store_sf(st + C::kOffSfa, ra[d], lane);
-          store_sf(st + C::kOffSfb, rb[d], lane);
+#pragma unroll
+          for (int at = 0; at < kAt; ++at) store_sf(st + C::kOffSfb + at * kSf, rb[d][at], lane);
           tc::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -208,7 +219,9 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
           const int nkj = J.valid ? nk : 0;               // an invalid item reads zeros
           if (PAIR) load_sf_pair(ra[d], p.sa, p.sa2, J.arow, k32, kj, nkj, lane);
           else load_sf(ra[d], p.sa, J.arow, 128, 0x7fffffff, k32, kj, nkj, lane);
-          load_sf(rb[d], p.sb, J.brow, NT, p.Ptot, k32, kj, nkj, lane);
+#pragma unroll
+          for (int at = 0; at < kAt; ++at)
+            load_sf(rb[d][at], p.sb, J.brow + 128 * at, NT - 128 * at, p.Ptot, k32, kj, nkj, lane);
         }
       }
     }
@@ -227,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
         const int buf = it & 1;
         if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) break;
         tc::fence_after_sync();
-        const uint32_t acc_col = tmem + uint32_t(buf * NT);
+        const uint32_t acc_col = tmem + uint32_t(buf * C::kAccStride);
         for (int kt = 0; kt < nk; ++kt, ++g) {
           const int j = g >> 1, np = C::stages_of(g & 1);
           const int s = 2 * (j % np) + (g & 1), r = j / np;
@@ -238,7 +251,9 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
           tc::fence_after_sync();
           uint8_t* st = smem + s * C::kStage;
           tc::cp_sf_32x128b_x4(tmem + C::kColSfa, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfa)));
-          tc::cp_sf_32x128b_x4(tmem + C::kColSfb, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfb)));
+#pragma unroll
+          for (int at = 0; at < C::kSfbAtoms; ++at)
+            tc::cp_sf_32x128b_x4(tmem + C::kColSfb + 4 * at, tc::smem_desc_sf(tc::smem_u32(st + C::kOffSfb + at * kSf)));
           const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffA));
           const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + C::kOffB));
 #pragma unroll
@@ -267,7 +282,8 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
       if constexpr (PAIR) ok = gemm::all_of_epilogue(ok);
       if (!ok) break;
       tc::fence_after_sync();
-      gemm::epilogue_tile<NT, PAIR>(tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * NT), I, p.out, ubuf, q, lane);
+      gemm::epilogue_tile<NT, PAIR>(tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * C::kAccStride), I, p.out, ubuf,
+                                    q, lane);
       // this warp's reads of the buffer are complete: hand it back to the MMA warp
       tc::fence_before_sync();
       __syncwarp();
@@ -358,13 +374,18 @@ stq_status launch_nt(int nt, const CUtensorMap& a, const CUtensorMap& a2, const 
     case 16: return launch_gemm<16, PAIR, A8>(a, a2, b, p, s);
     case 32: return launch_gemm<32, PAIR, A8>(a, a2, b, p, s);
     case 64: return launch_gemm<64, PAIR, A8>(a, a2, b, p, s);
+    case 240: return launch_gemm<240, PAIR, A8>(a, a2, b, p, s);
     default: return launch_gemm<128, PAIR, A8>(a, a2, b, p, s);
   }
 }
 
 int pick_nt(int64_t tokens_per_expert) {
-  return tokens_per_expert <= 16 ? 16 : tokens_per_expert <= 32 ? 32 : tokens_per_expert <= 64 ? 64 : 128;
+  return tokens_per_expert <= 16 ? 16 : tokens_per_expert <= 32 ? 32 : tokens_per_expert <= 64 ? 64
+         : tokens_per_expert < 128 ? 128 : 240;
 }
+
+// The next narrower N tile.
+int narrower_nt(int nt) { return nt > 128 ? 128 : nt / 2; }
 
 }  // namespace
 
@@ -380,15 +401,19 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   // 1. activations -> MXFP8 in sorted (expert-grouped) order
   stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.xq, a.xs, s);
   if (st != STQ_OK) return st;
-  // 2. N tiles of the touched experts
-  const int nt = pick_nt(int64_t(P) / (a.E < P ? a.E : P));
+  // 2. N tiles of the touched experts: the down projection takes the 240-wide tile from
+  // 128 tokens per expert on average, the gate/up pair (whose SwiGLU/MXFP8 epilogue and
+  // item balance measured slower there) at most 128
+  const int slots_ = a.E < P ? a.E : P;
+  const int nt_dn = pick_nt(int64_t(P) / slots_);
+  const int nt = nt_dn > 128 ? 128 : nt_dn;
   if ((st = stq_tile_plan_launch(a.counts, a.E, nt, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
-  const int max_tiles = P / nt + (a.E < P ? a.E : P);
+  const int max_tiles = P / nt + slots_;
   // 3. gate/up pair with SwiGLU and MXFP8 h
   CUtensorMap mg, mu, mx, md, mh;
   if (!tma::map_e2m1(&mg, a.wg, uint64_t(a.H), uint64_t(a.E) * a.I, 64) ||
       !tma::map_e2m1(&mu, a.wu, uint64_t(a.H), uint64_t(a.E) * a.I, 64) || !tma::map_u8(&mx, a.xq, a.H, P, nt) ||
-      !tma::map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !tma::map_u8(&mh, a.hq, a.I, P, nt))
+      !tma::map_e2m1(&md, a.wd, uint64_t(a.I), uint64_t(a.E) * a.H) || !tma::map_u8(&mh, a.hq, a.I, P, nt_dn))
     return STQ_ERR_CUDA;
   GemmProblem gp{};
   gp.tiles.R = a.I;
@@ -411,10 +436,11 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   }
   if (st != STQ_OK) return st;
   if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
-  // 4. down
+  // 4. down (the N-tile plan is redone for its tile width once the gate/up launch is done with it)
+  if (nt_dn != nt && (st = stq_tile_plan_launch(a.counts, a.E, nt_dn, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
   GemmProblem dp = gp;
   dp.tiles.R = a.H;
-  dp.tiles.max_items = max_tiles * (a.H / 128);
+  dp.tiles.max_items = (P / nt_dn + slots_) * (a.H / 128);
   dp.K = a.I;
   dp.sa = a.dsc;
   dp.sa2 = nullptr;
@@ -422,7 +448,7 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   dp.out = gemm::EpiOut{a.H, a.Y, nullptr, nullptr};
   {
     StqTimed tm(STQ_K_DOWN_MX, s);
-    st = launch_nt<false>(nt, md, md, mh, dp, s);
+    st = launch_nt<false>(nt_dn, md, md, mh, dp, s);
   }
   return st;
 }
@@ -441,7 +467,8 @@ stq_status moe_shared_expert_mx8(const MoeArgs& a, cudaStream_t s) {
   stq_status st = stq_mxfp8_quantize_launch(a.x, T, a.H, xq, xs, s);
   if (st != STQ_OK) return st;
   int nt = pick_nt(T);
-  while (nt > 16 && (a.I / 64) * ((T + nt - 1) / nt) < 148) nt /= 2;
+  if (nt > 128) nt = 128;  // the 240-wide tile measured slower for the gate/up pair
+  while (nt > 16 && (a.I / 64) * ((T + nt - 1) / nt) < 148) nt = narrower_nt(nt);
   const int ntile = (T + nt - 1) / nt;
   CUtensorMap mg, mu, mx, md, mh;
   if (!tma::map_u8(&mg, a.sgq, uint64_t(a.H), uint64_t(a.I), 64) ||
@@ -491,7 +518,7 @@ extern "C" stq_status w4a8_gemm(const uint8_t* w_codes, const uint8_t* w_scales,
                  STQ_ERR_ALIGN);
   cudaStream_t s = stq_cuda_stream(stream);
   int nt = pick_nt(M);
-  while (nt > 16 && (N / 128) * ((M + nt - 1) / nt) < 148) nt /= 2;  // fill the SMs
+  while (nt > 16 && (N / 128) * ((M + nt - 1) / nt) < 148) nt = narrower_nt(nt);  // fill the SMs
   CUtensorMap ma, mb;
   if (!tma::map_e2m1(&ma, w_codes, uint64_t(K), uint64_t(N)) || !tma::map_u8(&mb, a_codes, uint64_t(K), uint64_t(M), nt))
     return STQ_ERR_CUDA;

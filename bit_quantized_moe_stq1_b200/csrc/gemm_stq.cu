@@ -361,21 +361,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::fence_after_sync();
         const uint32_t tp = lane_base + uint32_t(kColP + 128 * pb);
+        // 32 columns per TMEM round trip (a 16-column tail when ncols is an odd multiple of 16)
 #pragma unroll 1
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
-          uint32_t v[16], a[16];
-          tc::tmem_ld_x16(tp + c0, v);
-          if (kb > 0) {
-            tc::tmem_ld_x16(tacc + c0, a);
-            tc::tmem_ld_wait();
+        for (int c0 = 0; c0 < ncols; c0 += 32) {
+          if (c0 + 32 <= ncols) {
+            uint32_t v[32], a[32];
+            tc::tmem_ld_x32(tp + c0, v);
+            if (kb > 0) {
+              tc::tmem_ld_x32(tacc + c0, a);
+              tc::tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(fmaf(d, __uint_as_float(v[j]), __uint_as_float(a[j])));
+              for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(fmaf(d, __uint_as_float(v[j]), __uint_as_float(a[j])));
+            } else {
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(d * __uint_as_float(v[j]));
+            }
+            tc::tmem_st_x32(tacc + c0, a);
           } else {
-            tc::tmem_ld_wait();
+            uint32_t v[16], a[16];
+            tc::tmem_ld_x16(tp + c0, v);
+            if (kb > 0) {
+              tc::tmem_ld_x16(tacc + c0, a);
+              tc::tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(d * __uint_as_float(v[j]));
+              for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(fmaf(d, __uint_as_float(v[j]), __uint_as_float(a[j])));
+            } else {
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(d * __uint_as_float(v[j]));
+            }
+            tc::tmem_st_x16(tacc + c0, a);
           }
-          tc::tmem_st_x16(tacc + c0, a);
         }
         // the partial is read and the accumulator written: release the partial buffer
         tc::tmem_st_wait();

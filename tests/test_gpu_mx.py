@@ -117,8 +117,11 @@ def _check_mx_layer(r, T, H, I, E, k, experts=None):
 
 
 @pytest.mark.parametrize("T,H,I,E,k,shared", [(5, 512, 256, 8, 2, True), (3, 256, 128 * 2, 4, 4, False),
-                                               (40, 512, 256, 4, 4, False)])
+                                               (40, 512, 256, 4, 4, False), (1000, 512, 256, 2, 1, True),
+                                               (481, 256, 256, 1, 1, False)])
 def test_moe_mx_small_full_check(S, T, H, I, E, k, shared):
+    """Every N tile width: 16 (decode) up to 240 (128 or more tokens per expert; 481 tokens
+    on one expert give tiles of 240, 240 and 1)."""
     r = _mx_layer(S, T, H, I, E, k, shared, ("mxs", T, H, I, E, k))
     _check_mx_layer(r, T, H, I, E, k)
 
