@@ -17,6 +17,8 @@
 //   down      per touched expert and 256-row tile: Y[pos, H] (FP32); shared -> Y[P+t]
 //   combine   y[t] = sum_s w[t,s] Y[inv[t,s]] (+ Y[P+t]) (+ x[t]) in slot order
 
+#include <mutex>
+
 #include "gemv.cuh"
 #include "moe_internal.cuh"
 
@@ -126,16 +128,6 @@ __global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __rest
 }
 
 // ----------------------------------------------------------------------------- router
-
-__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
-  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc = fmaf(bf16_bits_to_float(aw[i] & 0xFFFFu), bf16_bits_to_float(bw[i] & 0xFFFFu), acc);
-    acc = fmaf(bf16_bits_to_float(aw[i] >> 16), bf16_bits_to_float(bw[i] >> 16), acc);
-  }
-  return acc;
-}
 
 // Router logits, split over K: part[ks][t][e] = sum over the ks-th slice of H of
 // x[t, h] wr[e, h] (bf16 mma.sync, FP32 accumulate).  CTA = 16 experts x one K slice;
@@ -689,6 +681,32 @@ stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const f
   return stq_launch_status();
 }
 
+// A library-owned stream (and fork/join events) per device, created on first use: the
+// MXFP8 shared expert depends on x alone, so it runs beside the routing, permutation and
+// routed experts instead of after them.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+static stq_status side_stream(SideStream** out) {
+  constexpr int kMaxDevices = 64;
+  static SideStream side[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return STQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  SideStream& ss = side[dev];
+  if (ss.stream == nullptr) {
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return STQ_ERR_CUDA;
+  }
+  *out = &ss;
+  return STQ_OK;
+}
+
 // Average routed tokens per expert from which STQ_REGIME_AUTO runs the STQ1_0 experts
 // on the tensor-core GEMM instead of the decode GEMV.
 constexpr int kStqPrefillTokensPerExpert = 32;
@@ -724,8 +742,7 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   cudaStream_t s = stq_cuda_stream(stream);
   const MoeWs ws = moe_ws_pointers(workspace, L);
   const int P = d->T * d->k;
-  stq_status st = moe_launch_permute(topk_ids, P, d->E, ws, s);
-  if (st != STQ_OK) return st;
+  stq_status st = STQ_OK;
 
   MoeArgs a{};
   a.T = d->T; a.H = d->H; a.I = d->I; a.E = d->E; a.k = d->k; a.P = P;
@@ -749,6 +766,18 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   a.sched = ws.sched;
   a.err = ws.err;
   const int slots = d->E < P ? d->E : P;
+
+  // The MXFP8 shared expert on the side stream (its workspace rows P.. and the sticky error
+  // word are all it writes; nothing on the routed path reads them), joined before the combine.
+  SideStream* side = nullptr;
+  if (shared_mx8) {
+    if ((st = side_stream(&side)) != STQ_OK) return st;
+    if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+      return STQ_ERR_CUDA;
+    if ((st = moe_shared_expert_mx8(a, side->stream)) != STQ_OK) return st;
+    if (cudaEventRecord(side->join, side->stream) != cudaSuccess) return STQ_ERR_CUDA;
+  }
+  if ((st = moe_launch_permute(topk_ids, P, d->E, ws, s)) != STQ_OK) return st;
 
   const bool prefill = d->regime == STQ_REGIME_PREFILL ||
                        (d->regime == STQ_REGIME_AUTO && P >= kStqPrefillTokensPerExpert * slots);
@@ -776,7 +805,7 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     st = moe_mx_experts(a, slots, shared_bf16, s);
     if (st != STQ_OK) return st;
   }
-  if (shared_mx8 && (st = moe_shared_expert_mx8(a, s)) != STQ_OK) return st;
+  if (shared_mx8 && cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) return STQ_ERR_CUDA;
   return moe_launch_combine(*d, P, ws, topk_w, has_shared, x, y, s);
 }
 

@@ -216,7 +216,12 @@ stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router,
  *                     per weight, row-major) and sh_*_sc their UE8M0 scales [rows][K/32]
  *                     (as written by mxfp8_quantize_bf16); x and h are quantised to
  *                     MXFP8 g32 (the activation rule of mxfp8_quantize_bf16) and the
- *                     products accumulate in FP32. */
+ *                     products accumulate in FP32.  It depends on x alone, so
+ *                     moe_expert_forward runs it on a library-owned stream of the
+ *                     current device (created with two events on first use, then
+ *                     reused; not device memory), forked from `stream` after the
+ *                     call's argument checks and joined back before the combine; the
+ *                     call stays ordered on `stream` and can be captured into a graph. */
 enum { STQ_SHARED_BF16 = 0, STQ_SHARED_MXFP8 = 1 };
 
 typedef struct {
