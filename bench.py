@@ -51,7 +51,8 @@ NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense
 MEASURED_TRAFFIC_PER_EXPERT = {}
 # DRAM bytes (read + write) of one full-size launch, from an ncu capture of the same workload
 # and kernel build; an entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_LAUNCH = {("prefill_stq", "gate_up_stq_tc"): 1.608519e9 + 64.757248e6}
+MEASURED_TRAFFIC_PER_LAUNCH = {("prefill_stq", "gate_up_stq_tc"): 1.608519e9 + 64.757248e6,
+                               ("prefill_w4a8", "gate_up_mx"): 3.751041e9 + 71.260672e6}
 
 
 def peaks():
