@@ -48,7 +48,7 @@ NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense
 # capture of the same kernel build on a smaller case (named profile under profiles/); a
 # launch's traffic grows with its touched experts, so the full launch's traffic is this
 # figure times its touched experts.  An entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_EXPERT = {}
+MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (2.109465e9 + 6.812928e6) / 157}  # decode_mx, 157 touched
 # DRAM bytes (read + write) of one full-size launch, from an ncu capture of the same workload
 # and kernel build; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC_PER_LAUNCH = {("prefill_stq", "gate_up_stq_tc"): 1.608519e9 + 64.757248e6,

@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
 
 // Routed STQ1_0 down, persistent.  Items: the shared expert's 16-row tiles, then per
 // touched expert 256-row tiles of H (warp = 4 tiles).
-__global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
+__global__ void __launch_bounds__(128, 3) moe_down_stq_kernel(MoeArgs a) {
   __shared__ float red[4][2][4][4][32];
   __shared__ int s_item;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
@@ -632,7 +632,7 @@ stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
   a.sched = a0.sched + 3;
   {
     StqTimed tm(STQ_K_SHARED_DOWN, s);
-    moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta)), 128, 0, s>>>(a);
+    moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta, 3)), 128, 0, s>>>(a);
   }
   return stq_launch_status();
 }
@@ -798,7 +798,7 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     a.sched = ws.sched + 1;
     {
       StqTimed tm(STQ_K_DOWN, s);
-      moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->H / 256))), 128, 0, s>>>(a);
+      moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->H / 256), 3)), 128, 0, s>>>(a);
     }
     if ((st = stq_launch_status()) != STQ_OK) return st;
   } else {

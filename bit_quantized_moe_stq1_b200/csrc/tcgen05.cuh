@@ -153,26 +153,6 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[
       : "memory");
 }
 
-// 8 and 4 consecutive 32-bit columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_x4(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(taddr));
-}
-
-// 8 consecutive 32-bit columns of this thread's TMEM lane <- r.
-__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t* r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
-}
-
 // 16 consecutive 32-bit columns of this thread's TMEM lane <- r.
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -210,9 +190,5 @@ __host__ __device__ constexpr uint32_t idesc_mxf8f6f4_ab(int n, uint32_t afmt, u
          (uint32_t(128 >> 4) << 24) | (a_sf << 29);
 }
 
-// A = E2M1 weights, B = E4M3 activations.
-__host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int n, uint32_t a_sf, uint32_t b_sf) {
-  return idesc_mxf8f6f4_ab(n, kFmtE2M1, kFmtE4M3, a_sf, b_sf);
-}
 
 }  // namespace tc
