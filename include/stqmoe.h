@@ -221,7 +221,11 @@ stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router,
  *                     current device (created with two events on first use, then
  *                     reused; not device memory), forked from `stream` after the
  *                     call's argument checks and joined back before the combine; the
- *                     call stays ordered on `stream` and can be captured into a graph. */
+ *                     call stays ordered on `stream` and can be captured into a graph.
+ *                     Calls on one device share that stream: calls from several host
+ *                     threads serialize their shared-expert work on it, and a call while
+ *                     another thread is capturing such a call into a graph is not
+ *                     supported. */
 enum { STQ_SHARED_BF16 = 0, STQ_SHARED_MXFP8 = 1 };
 
 typedef struct {
