@@ -301,6 +301,10 @@ __global__ void mxfp4_unpack_kernel(const uint8_t* __restrict__ codes, const uin
 // Four lanes per 32-element group, eight elements per lane.
 // Grid (column chunks of 2048 elements, rows; rows beyond 65535 loop): thread = 8
 // consecutive elements, 4 threads = one 32-element group, no 64-bit division per thread.
+// RPB rows per CTA (rows RPB*blockIdx.y .. +RPB, then strided by the grid): every row's
+// source index and activation load are issued before the first row is quantised, so the
+// two dependent load latencies are paid once per RPB rows.
+template <int RPB>
 __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                int64_t K, uint8_t* __restrict__ codes,
                                                                uint8_t* __restrict__ scales,
@@ -308,57 +312,74 @@ __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* _
   const int part = int(threadIdx.x & 3);
   const int64_t col8 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // 8-element chunk of the row
   const bool active = col8 < K / 8;                                     // whole 4-thread groups
-  for (int64_t row = blockIdx.y; row < rows; row += gridDim.y) {
-    const int64_t gi = row * (K / 32) + (col8 >> 2);
-    float v[8];
-    float amax = 0.f;
-    bool bad = false;
-    if (active) {
-      const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
-      const uint4 raw = *reinterpret_cast<const uint4*>(x + src * K + col8 * 8);
-      const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+  for (int64_t r0 = int64_t(blockIdx.y) * RPB; r0 < rows; r0 += int64_t(gridDim.y) * RPB) {
+    uint4 raw[RPB];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[2 * i] = bf16_bits_to_float(rw[i] & 0xFFFFu);
-        v[2 * i + 1] = bf16_bits_to_float(rw[i] >> 16);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        bad |= !isfinite(v[i]);
-        amax = fmaxf(amax, isfinite(v[i]) ? fabsf(v[i]) : 0.f);
+    for (int j = 0; j < RPB; ++j) {
+      raw[j] = make_uint4(0u, 0u, 0u, 0u);
+      const int64_t row = r0 + j;
+      if (active && row < rows) {
+        const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
+        raw[j] = *reinterpret_cast<const uint4*>(x + src * K + col8 * 8);
       }
     }
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const unsigned badmask = __ballot_sync(0xffffffffu, bad);
-    if (!active) continue;
-    const bool gbad = (badmask >> (threadIdx.x & 28)) & 0xFu;
-    int e = mx_scale_exponent(amax, 0x600000u, 8);  // limit 448 = 1.75 * 2^8
-    uint32_t lo = 0u, hi = 0u;
-    if (gbad) {
-      e = 255;
-      lo = hi = 0x7F7F7F7Fu;
-    } else {
-      const float f = pow2_float(127 - e);
 #pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        const __nv_fp8x2_storage_t pr =
-            __nv_cvt_float2_to_fp8x2(make_float2(v[i] * f, v[i + 1] * f), __NV_SATFINITE, __NV_E4M3);
-        uint32_t c0 = pr & 0xFFu, c1 = (pr >> 8) & 0xFFu;
-        // zero results carry the sign of the input
-        if ((c0 & 0x7Fu) == 0u) c0 = (__float_as_uint(v[i]) >> 31) << 7;
-        if ((c1 & 0x7Fu) == 0u) c1 = (__float_as_uint(v[i + 1]) >> 31) << 7;
-        const uint32_t pair = c0 | (c1 << 8);
-        if (i < 4) lo |= pair << (8 * i); else hi |= pair << (8 * (i - 4));
+    for (int j = 0; j < RPB; ++j) {
+      const int64_t row = r0 + j;
+      if (row >= rows) break;  // the same for every thread of the CTA
+      const int64_t gi = row * (K / 32) + (col8 >> 2);
+      float v[8];
+      float amax = 0.f;
+      bool bad = false;
+      if (active) {
+        const uint32_t rw[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[2 * i] = bf16_bits_to_float(rw[i] & 0xFFFFu);
+          v[2 * i + 1] = bf16_bits_to_float(rw[i] >> 16);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          bad |= !isfinite(v[i]);
+          amax = fmaxf(amax, isfinite(v[i]) ? fabsf(v[i]) : 0.f);
+        }
       }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const unsigned badmask = __ballot_sync(0xffffffffu, bad);
+      if (!active) continue;
+      const bool gbad = (badmask >> (threadIdx.x & 28)) & 0xFu;
+      int e = mx_scale_exponent(amax, 0x600000u, 8);  // limit 448 = 1.75 * 2^8
+      uint32_t lo = 0u, hi = 0u;
+      if (gbad) {
+        e = 255;
+        lo = hi = 0x7F7F7F7Fu;
+      } else {
+        const float f = pow2_float(127 - e);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          const __nv_fp8x2_storage_t pr =
+              __nv_cvt_float2_to_fp8x2(make_float2(v[i] * f, v[i + 1] * f), __NV_SATFINITE, __NV_E4M3);
+          uint32_t c0 = pr & 0xFFu, c1 = (pr >> 8) & 0xFFu;
+          // zero results carry the sign of the input
+          if ((c0 & 0x7Fu) == 0u) c0 = (__float_as_uint(v[i]) >> 31) << 7;
+          if ((c1 & 0x7Fu) == 0u) c1 = (__float_as_uint(v[i + 1]) >> 31) << 7;
+          const uint32_t pair = c0 | (c1 << 8);
+          if (i < 4) lo |= pair << (8 * i); else hi |= pair << (8 * (i - 4));
+        }
+      }
+      *reinterpret_cast<uint2*>(codes + gi * 32 + part * 8) = make_uint2(lo, hi);
+      if (part == 0) scales[gi] = uint8_t(e);
     }
-    *reinterpret_cast<uint2*>(codes + gi * 32 + part * 8) = make_uint2(lo, hi);
-    if (part == 0) scales[gi] = uint8_t(e);
   }
 }
 
+// From 4096 rows a CTA takes 8 rows (enough CTAs remain to fill the SMs), below it one.
+constexpr int64_t kQuantMultiRow = 4096;
+
 dim3 quant_grid(int64_t rows, int64_t K) {
-  return dim3(unsigned(ceil_div<int64_t>(K / 8, 256)), unsigned(rows < 65535 ? rows : 65535));
+  const int64_t ry = rows >= kQuantMultiRow ? ceil_div<int64_t>(rows, 8) : rows;
+  return dim3(unsigned(ceil_div<int64_t>(K / 8, 256)), unsigned(ry < 65535 ? ry : 65535));
 }
 
 }  // namespace
@@ -437,7 +458,10 @@ stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K,
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
-  mxfp8_quant_bf16_kernel<<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1);
+  if (rows >= kQuantMultiRow)
+    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1);
+  else
+    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1);
   return stq_launch_status();
 }
 
@@ -446,7 +470,10 @@ stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
-  mxfp8_quant_bf16_kernel<<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k);
+  if (rows >= kQuantMultiRow)
+    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k);
+  else
+    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k);
   return stq_launch_status();
 }
 

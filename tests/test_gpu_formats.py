@@ -130,6 +130,14 @@ def test_mxfp8_quant_activation_workload(S):
     assert np.array_equal(c[-7:].cpu().numpy(), rc2) and np.array_equal(s[-7:].cpu().numpy(), rs2)
 
 
+def test_mxfp8_quant_many_rows_ragged(S):
+    """4099 rows: CTAs of 8 rows with a 3-row tail, every row checked."""
+    x = W.bf16_normal((4099, 512), 1.0, DEV, 0, "act-ragged")
+    c, s = S.mxfp8_quantize_bf16(x)
+    rc, rs = F.mxfp8_quantize(F.bf16_decode(x.view(torch.int16).cpu().numpy().view(np.uint16)))
+    assert np.array_equal(c.cpu().numpy(), rc) and np.array_equal(s.cpu().numpy(), rs)
+
+
 def _imp(K, tag):
     return torch.exp(W.float_normal((K,), 1.0, DEV, 0, "imp", tag)).contiguous()
 
