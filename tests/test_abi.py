@@ -163,3 +163,15 @@ def test_workspace_mxfp8_regions_hold_pairs_and_tokens(built):
     assert room["hq"] >= (P + T) * I and room["hs"] >= (P + T) * I // 32
     assert room["h"] >= (P + T) * I * 2 and room["Y"] >= (P + T) * H * 4
     assert all(o % 256 == 0 for o in off.values())
+
+
+def test_timing_kinds_match_the_header():
+    """The binding names the timing hook's kernel kinds in the header's enum order."""
+    import bit_quantized_moe_stq1_b200 as S
+
+    text = open(os.path.join(ROOT, "include", "stqmoe.h")).read()
+    body = re.search(r"enum\s*\{\s*(STQ_K_ROUTER_LOGITS[^}]*)\}", text).group(1)
+    names = [n.strip().split("=")[0].strip() for n in body.split(",") if n.strip()]
+    assert names[-1] == "STQ_K_COUNT"
+    expect = [n[len("STQ_K_"):].lower() for n in names[:-1]]
+    assert expect == list(S.KERNEL_KINDS)

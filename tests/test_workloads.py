@@ -38,3 +38,15 @@ def test_zipf_routing_distinct_and_skewed():
 def test_workload_table():
     assert W.WORKLOADS["stacked_decode"].formats == ("stq", "mx") * 4
     assert W.HIDDEN == 6144 and W.INTER == 2048 and W.EXPERTS == 256 and W.TOPK == 8
+
+
+def test_bench_unit_bytes():
+    """The bench's algorithmic bytes per matrix: STQ1_0 42 B per 256 weights, MXFP4 a half
+    byte per weight + one scale per 32, MXFP8 a byte per weight + one scale per 32, BF16 2."""
+    import bench
+
+    n = 2048 * 6144
+    assert bench.STQ_MAT == n // 256 * 42 == 2_064_384
+    assert bench.MX_MAT == n // 2 + n // 32 == 6_684_672
+    assert bench.MX8_MAT == n + n // 32 == 12_976_128
+    assert bench.BF16_MAT == 2 * n == 25_165_824
