@@ -63,6 +63,11 @@ SIGNATURES = {
     "moe_get_device_error": (_i32, [_vp, _vp]),
     "stq_set_timing": (_i32, [_vp]),
     "stq_wait_selftest": (_i32, [_vp, _vp]),
+    "stq_slot_bank_create": (_vp, [_i32, _i32]),
+    "stq_slot_bank_destroy": (None, [_vp]),
+    "stq_slot_bank_map": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp]),
+    "stq_slot_bank_resident": (_i32, [_vp, _vp]),
+    "stq_slot_bank_copy": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "stq_rmsnorm_bf16": (_i32, [_vp, _i64, _i64, ctypes.c_float, _vp, _vp]),
 }
 
@@ -382,3 +387,59 @@ def moe_get_device_error(workspace, stream=None):
 
 def status_string(s):
     return lib.stq_status_string(s).decode()
+
+
+class SlotBank:
+    """Host-side expert slot bank (see stq_slot_bank_* in include/stqmoe.h): maps each
+    call's routed ids to slots and lists the experts to copy in."""
+
+    def __init__(self, n_experts, n_slots):
+        self.n_experts, self.n_slots = int(n_experts), int(n_slots)
+        # kept on the instance: module globals may already be gone when a bank is
+        # collected at interpreter exit
+        self._destroy = lib.stq_slot_bank_destroy
+        self._h = lib.stq_slot_bank_create(self.n_experts, self.n_slots)
+        if not self._h:
+            raise StqError(-1, "stq_slot_bank_create")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            self._destroy(h)
+            self._h = None
+
+    def map(self, ids):
+        """ids: host int32 array-like (any shape) -> (slot ids of the same shape, experts to
+        load, their slots), all numpy int32."""
+        import numpy as np
+
+        a = np.ascontiguousarray(np.asarray(ids, dtype=np.int32))
+        slots = np.empty_like(a)
+        le = np.empty(self.n_slots, dtype=np.int32)
+        ls = np.empty(self.n_slots, dtype=np.int32)
+        n = ctypes.c_int32(0)
+        _check(lib.stq_slot_bank_map(self._h, a.ctypes.data, a.size, slots.ctypes.data, le.ctypes.data,
+                                     ls.ctypes.data, ctypes.byref(n)), "stq_slot_bank_map")
+        return slots, le[:n.value].copy(), ls[:n.value].copy()
+
+    def resident(self):
+        import numpy as np
+
+        out = np.empty(self.n_slots, dtype=np.int32)
+        _check(lib.stq_slot_bank_resident(self._h, out.ctypes.data), "stq_slot_bank_resident")
+        return out
+
+    @staticmethod
+    def copy(load_expert, load_slot, src, dst, stream=None):
+        """Copy experts into slots: src / dst are lists of expert-major tensors (host, ideally
+        pinned, and device), one per matrix, each [experts or slots, ...] with equal rows."""
+        import numpy as np
+
+        le = np.ascontiguousarray(load_expert, dtype=np.int32)
+        ls = np.ascontiguousarray(load_slot, dtype=np.int32)
+        n_m = len(src)
+        srcs = (ctypes.c_void_p * n_m)(*[t.data_ptr() for t in src])
+        dsts = (ctypes.c_void_p * n_m)(*[t.data_ptr() for t in dst])
+        sizes = (ctypes.c_size_t * n_m)(*[t[0].numel() * t.element_size() for t in src])
+        _check(lib.stq_slot_bank_copy(le.ctypes.data, ls.ctypes.data, le.size, n_m, srcs, dsts, sizes,
+                                      _stream(stream)), "stq_slot_bank_copy")

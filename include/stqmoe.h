@@ -316,6 +316,45 @@ stq_status stq_rmsnorm_bf16(const uint16_t* x, int64_t T, int64_t H, float eps,
                             uint16_t* y, stq_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
+/* Expert slot bank ("Hy4-preview-FlashMoE-STQ1_0", running with a slot bank:   */
+/* routed experts stay outside HBM and are read on demand into a fixed number   */
+/* of slots; a miss reads its expert in; at least top-k slots).  Host side.     */
+/* ------------------------------------------------------------------------- */
+
+/* Opaque host object: which expert each of n_slots slots holds, and when each slot was last
+ * used.  Replacement (not stated on the pages): the least recently used slot among those
+ * the current call does not need, ties to the lowest slot index. */
+typedef struct stq_slot_bank stq_slot_bank;
+
+/* New empty bank for experts [0, n_experts) in n_slots slots (1 <= n_slots <= n_experts);
+ * NULL on invalid arguments or allocation failure.  Host memory only; not thread-safe. */
+stq_slot_bank* stq_slot_bank_create(int32_t n_experts, int32_t n_slots);
+void stq_slot_bank_destroy(stq_slot_bank* bank);
+
+/* Map the routed expert ids of one call (host int32 [n], e.g. topk_ids of T tokens x k) to
+ * slots: slot_ids (host int32 [n]) gets the slot that holds ids[i] after the call; the
+ * experts that were not resident are listed in first-use order in load_expert / load_slot
+ * (host int32, capacity n_slots), *n_loads of them: the caller copies those experts into
+ * those slots (stq_slot_bank_copy) before running moe_expert_forward with E = n_slots and
+ * the slot ids as topk_ids.  Errors (bank unchanged): STQ_ERR_INVALID_ARG for an id outside
+ * [0, n_experts) or a call touching more distinct experts than there are slots. */
+stq_status stq_slot_bank_map(stq_slot_bank* bank, const int32_t* ids, int64_t n, int32_t* slot_ids,
+                             int32_t* load_expert, int32_t* load_slot, int32_t* n_loads);
+
+/* The expert held by each slot (host int32 [n_slots], -1 = empty). */
+stq_status stq_slot_bank_resident(const stq_slot_bank* bank, int32_t* slot_expert);
+
+/* Copy the listed experts' matrices into their slots: for load i and matrix m,
+ * mat_bytes[m] bytes from src[m] + load_expert[i] * mat_bytes[m] (the full expert-major
+ * array, normally pinned host memory so the copy is asynchronous) to dst[m] +
+ * load_slot[i] * mat_bytes[m] (the slot bank's expert-major device array).  One
+ * cudaMemcpyAsync per load and matrix on `stream`; asynchronous.  STQ_ERR_INVALID_ARG
+ * for null pointers or negative entries, STQ_ERR_CUDA if a copy cannot be enqueued. */
+stq_status stq_slot_bank_copy(const int32_t* load_expert, const int32_t* load_slot, int32_t n_loads,
+                              int32_t n_mats, const void* const* src, void* const* dst,
+                              const size_t* mat_bytes, stq_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
 /* Instrumentation (no counterpart on the pages).                             */
 /* ------------------------------------------------------------------------- */
 
