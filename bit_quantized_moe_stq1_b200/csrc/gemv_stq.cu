@@ -48,7 +48,6 @@ extern "C" stq_status stq1_gemv(const uint8_t* W, int64_t rows, int64_t K, const
   STQ_HOST_CHECK(W && x && y, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(rows % 16 == 0 && K % 256 == 0, STQ_ERR_SHAPE);
   STQ_HOST_CHECK(stq_aligned16(W) && stq_aligned16(x) && stq_aligned16(y), STQ_ERR_ALIGN);
-  if (rows == 0 || n == 0) return STQ_OK;
   if (K == 0) return cudaMemsetAsync(y, 0, size_t(n * rows) * sizeof(float), stq_cuda_stream(stream)) == cudaSuccess
                          ? STQ_OK
                          : STQ_ERR_CUDA;

@@ -593,8 +593,10 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
 }
 
 static bool desc_ok(const moe_desc* d) {
+  // P = T*k below 2^30 (as moe_permute): pair and row indices, P + T included, stay in int32
   return d && d->T >= 0 && d->H > 0 && d->I > 0 && d->E > 0 && d->E <= 1024 && d->k > 0 && d->k <= 32 &&
-         d->k <= d->E && d->regime >= STQ_REGIME_AUTO && d->regime <= STQ_REGIME_PREFILL;
+         d->k <= d->E && int64_t(d->T) * d->k < (int64_t(1) << 30) && d->regime >= STQ_REGIME_AUTO &&
+         d->regime <= STQ_REGIME_PREFILL;
 }
 
 extern "C" size_t moe_workspace_bytes(const moe_desc* d) {

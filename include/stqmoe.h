@@ -184,7 +184,8 @@ stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t 
  * perm [P] = pair at each sorted position, sorted by expert and stably by p;
  * inv [P] = sorted position of each pair (-1 for an id outside [0, E), which
  * also sets STQ_ERR_DEVICE in *err); tlist [E] = touched experts in ascending
- * order, ntouched [1] their number.  Integer, exact.  E <= 1024. */
+ * order, ntouched [1] their number.  Integer, exact.  E <= 1024, T*k < 2^30
+ * (else STQ_ERR_INVALID_ARG). */
 stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                        int32_t* tlist, int32_t* ntouched, int32_t* err,
@@ -257,7 +258,8 @@ typedef struct {
 enum { STQ_REGIME_AUTO = 0, STQ_REGIME_DECODE = 1, STQ_REGIME_PREFILL = 2 };
 
 typedef struct {
-  int32_t T, H, I, E, k;    /* tokens, hidden, intermediate, experts, top-k     */
+  int32_t T, H, I, E, k;    /* tokens, hidden, intermediate, experts, top-k;
+                               T >= 0, E <= 1024, 1 <= k <= min(32, E), T*k < 2^30 */
   int32_t out_fp32;         /* 1: y is float32 [T, H]; 0: y is bf16 [T, H]      */
   int32_t add_residual;     /* 1: y += x                                         */
   int32_t regime;           /* STQ_REGIME_* (STQ1_0 experts)                     */

@@ -58,6 +58,10 @@ def test_binding_loads_and_host_side_calls(built):
     # routed h (bf16) + Y (f32) dominate: (P+T)*I*2 + (P+T)*H*4
     assert ws >= (64 + 8) * 2048 * 2 + (64 + 8) * 6144 * 4
     assert S.moe_workspace_bytes(S.make_desc(8, 6144, 2048, 256, 300)) == 0       # k > E
+    # T*k < 2^30 keeps pair and row indices (P + T) in int32
+    assert S.moe_workspace_bytes(S.make_desc((1 << 27) - 1, 256, 256, 256, 8)) > 0
+    assert S.moe_workspace_bytes(S.make_desc(1 << 27, 256, 256, 256, 8)) == 0
+    assert S.moe_workspace_bytes(S.make_desc((1 << 31) - 1, 256, 256, 256, 32)) == 0
     # host-side validation returns before any device work (null pointers, bad shapes)
     assert S.lib.stq1_pack(None, 16, 256, None, None, None) == -1
     assert S.lib.stq1_gemv(ctypes.c_void_p(16), 16, 100, ctypes.c_void_p(16), 1, ctypes.c_void_p(16), None) == -2
