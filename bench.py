@@ -353,6 +353,78 @@ class MoeLayers(Workload):
                                                       for k, v in kinds.items()})
 
 
+class StreamLayer(MoeLayers):
+    """One STQ1_0 decode layer (8 tokens, BF16 shared expert) whose routed experts sit in
+    pinned host memory and stream on demand into a bank of 96 HBM slots: each step maps its
+    routed ids to slots (least recently used replacement), copies the missing experts in and
+    runs the layer with E = 96 on the slot ids.  Host memory stands in for the SSD sidecar of
+    the 96-slot run ("Hy4-preview-FlashMoE-STQ1_0").  Routing is Zipf with one popularity
+    order for every step, so consecutive steps reuse experts.  The per-step host work (slot
+    mapping, copy list) cannot live in a CUDA graph: steps run eagerly."""
+
+    N_SLOTS = 96
+    POOL = 64  # routing batches, cycled
+
+    def __init__(self, S, dev, experts=E):
+        global E
+        E = experts
+        self.S, self.dev, self.name, self.T = S, dev, "decode_stq_stream", 8
+        self.fmts, self.router, self.shared, self.residual, self.shared_fmt = ("stq",), False, True, False, "bf16"
+        self.n_slots = min(self.N_SLOTS, E)
+        self.host, self.slots = [], []
+        for which, rows, cols in (("g", I, H), ("u", I, H), ("d", H, I)):
+            per = rows * cols // 256 * 42
+            host = torch.empty((E, per), dtype=torch.uint8).pin_memory()
+            for e0 in range(0, E, 16):
+                # same weights as the resident layer's experts (tags of MoeLayers._stq)
+                wf = W.stq_grid_weights(16 * rows, cols, dev, 0, self.name, 0, which, e0)
+                n = min(16, E - e0)
+                host[e0:e0 + n].copy_(S.stq1_pack(wf).view(16, per)[:n])
+                del wf
+            self.host.append(host)
+            self.slots.append(torch.zeros((self.n_slots, per), dtype=torch.uint8, device=dev))
+        sh = [W.bf16_normal((I, H), 0.02, dev, 0, self.name, 0, "sg"),
+              W.bf16_normal((I, H), 0.02, dev, 0, self.name, 0, "su"),
+              W.bf16_normal((H, I), 0.02, dev, 0, self.name, 0, "sd")]
+        self.layers = [dict(fmt="stq", wr=None, sh_bf16=sh,
+                            w=S.ExpertWeights(S.FMT_STQ1_0, *(m.view(-1) for m in self.slots), None, None, None,
+                                              *sh))]
+        self.x = [W.bf16_normal((self.T, H), 1.0, dev, 0, self.name, "x", b) for b in range(N_BATCHES)]
+        ids, tw = W.zipf_routing(self.POOL * self.T, E, K_TOP, "cpu", 0, self.name, "zipf")
+        self.ids_host = [ids[b * self.T:(b + 1) * self.T].numpy().copy() for b in range(self.POOL)]
+        self.tw = [tw[b * self.T:(b + 1) * self.T].to(dev) for b in range(self.POOL)]
+        self.desc = S.make_desc(self.T, H, I, self.n_slots, K_TOP, out_fp32=False, regime=S.REGIME_DECODE)
+        self.ws = torch.zeros(S.moe_workspace_bytes(self.desc), dtype=torch.uint8, device=dev)
+        self.bufs = [torch.empty((self.T, H), dtype=torch.bfloat16, device=dev)]
+        self.sid = torch.empty((self.T, K_TOP), dtype=torch.int32, device=dev)
+        self.bank = S.SlotBank(E, self.n_slots)
+        self.log = []           # (step, experts loaded, distinct experts) per step
+        self.copy_events = None  # list of (start, stop) CUDA events around each step's copies
+
+    def step(self, i, x=None, y=None):
+        S = self.S
+        b = i % self.POOL
+        ids = self.ids_host[b]
+        slot_ids, le, ls = self.bank.map(ids)
+        if self.copy_events is not None:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record()
+        S.SlotBank.copy(le, ls, self.host, self.slots)
+        if self.copy_events is not None:
+            ev[1].record()
+            self.copy_events.append(ev)
+        # pageable source: the runtime has read it when the call returns
+        self.sid.copy_(torch.from_numpy(slot_ids), non_blocking=True)
+        self.log.append((i, int(le.size), int(np.unique(ids).size)))
+        cur = self.x[i % N_BATCHES] if x is None else x
+        out = self.bufs[0] if y is None else y
+        S.moe_expert_forward(self.desc, cur, self.sid, self.tw[b], self.layers[0]["w"], out, self.ws)
+        return out
+
+    def accounting(self, i):
+        raise NotImplementedError("streamed steps are accounted from their own log")
+
+
 def make_workload(name, S, dev, experts=256):
     if name == "stq_matvec":
         return StqMatvec(S, dev)
@@ -360,6 +432,8 @@ def make_workload(name, S, dev, experts=256):
         return W4A8Gemm(S, dev)
     if name == "stq_pack_ls":
         return StqPackLs(S, dev)
+    if name == "decode_stq_stream":
+        return StreamLayer(S, dev, experts)
     if name == "decode_mx":
         # one MXFP4 layer of the stacked workload (a small case for profiler captures)
         return MoeLayers(S, dev, name, 32, ("mx",), True, True, True, experts)
@@ -368,7 +442,7 @@ def make_workload(name, S, dev, experts=256):
 
 
 WORKLOAD_NAMES = ["stq_matvec", "w4a8_gemm", "decode_stq", "decode_stq_sh8", "prefill_w4a8", "prefill_stq",
-                  "stacked_decode", "decode_mx", "stq_pack_ls"]
+                  "stacked_decode", "decode_mx", "stq_pack_ls", "decode_stq_stream"]
 
 
 # ----------------------------------------------------------------------------- measurement
@@ -467,6 +541,106 @@ def base_config(wl):
     return {"workload": wl.name, "experts": E, "tokens_per_step": wl.tokens_per_step()}
 
 
+def run_stream(args, wl, S, dev, dist, n, rank, local):
+    """The streamed layer, timed eagerly: each step (slot mapping on the host, expert copies,
+    the layer) between CUDA events on the launching stream.  A second pass times every kernel
+    and each step's copies; a third runs end to end with x from and y to pinned host memory.
+    The host link's reference is one plain copy, measured in the same run, of one matrix of
+    every expert from pinned host memory to HBM."""
+    for i in range(args.warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+    ref = torch.empty(wl.host[0].shape, dtype=torch.uint8, device=dev)
+    ref.copy_(wl.host[0], non_blocking=True)
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record()
+    ref.copy_(wl.host[0], non_blocking=True)
+    r1.record()
+    torch.cuda.synchronize()
+    link_gbs = wl.host[0].numel() / (r0.elapsed_time(r1) * 1e-3) / 1e9
+    del ref
+    # timed pass
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wl.log = []
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record()
+        for i in range(args.steps):
+            wl.step(args.warmup + i)
+        stop.record()
+        torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    clocks = clk.summary()
+    ms_step = max_over_ranks([start.elapsed_time(stop)], dev, dist)[0] / args.steps
+    log = list(wl.log)
+    # kernel and copy times (a separate pass: the events add work)
+    timer = S.KernelTimer(capacity=16 * args.steps)
+    wl.copy_events, wl.log = [], []
+    with timer:
+        for i in range(args.steps):
+            wl.step(args.warmup + args.steps + i)
+    res = timer.results()
+    copy_ms = [a.elapsed_time(b) for a, b in wl.copy_events]
+    copied = sum(l for _, l, _ in wl.log) * 3 * STQ_MAT
+    wl.copy_events = None
+    kt = {}
+    for kind, ms in res:
+        kt.setdefault(kind, []).append(ms)
+    # end to end: x in from pinned host memory, y out to it, every step
+    hx = [wl.x[b].cpu().pin_memory() for b in range(N_BATCHES)]
+    xs = torch.empty_like(wl.x[0])
+    y_dev = torch.empty_like(wl.bufs[0])
+    hy = torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory()
+    torch.cuda.synchronize()
+    base = args.warmup + 2 * args.steps
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for i in range(args.steps):
+        xs.copy_(hx[(base + i) % N_BATCHES], non_blocking=True)
+        wl.step(base + i, x=xs, y=y_dev)
+        hy.copy_(y_dev, non_blocking=True)
+    s1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([s0.elapsed_time(s1)], dev, dist)[0]
+    loads = float(np.mean([l for _, l, _ in log]))
+    distinct = float(np.mean([d for _, _, d in log]))
+    copy_gbs = copied / (sum(copy_ms) * 1e-3) / 1e9 if copied else None
+    out = {
+        "metric": wl.metric, "value": whole_job_rate(n, wl.T, ms_step), "unit": wl.unit, "n_gpus": n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded generators; random weights on the STQ1_0 grid; Zipf routing)",
+        "config": {**base_config(wl), "slots": wl.n_slots, "experts_loaded_per_step": loads,
+                   "distinct_experts_per_step": distinct, "h2d_weight_bytes_per_step": loads * 3 * STQ_MAT,
+                   "l2": "inputs larger than L2: the bank (96 slots x 6.2 MB) and the copied experts",
+                   "parallelism": f"replicas x{n}",
+                   "timing": "eager steps (host slot mapping, expert copies, the layer), CUDA events"},
+        "roofline": {"bound": "h2d", "kernel": "expert copies (cudaMemcpyAsync, pinned host to HBM)",
+                     "achieved": copy_gbs, "peak": link_gbs, "unit": "GB/s",
+                     "frac": copy_gbs / link_gbs if copy_gbs else None,
+                     "peak_source": f"one plain pinned-host to HBM copy of {wl.host[0].numel() / 1e6:.0f} MB, "
+                                    "measured in this run",
+                     "traffic": None, "copy_ms_per_step": float(np.mean(copy_ms))},
+        "kernels_ms": {k: statistics.mean(v) for k, v in kt.items()},
+        "gpu_launches": len(res),
+        "e2e": {"value": whole_job_rate(n, wl.T, e2e_ms / args.steps), "unit": wl.unit,
+                "h2d_bytes_per_step": xs.numel() * xs.element_size() + wl.sid.numel() * 4 + loads * 3 * STQ_MAT,
+                "d2h_bytes_per_step": hy.numel() * hy.element_size()},
+        "clocks": clocks,
+    }
+    if rank == 0 and not dist and not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(wl, dev)
+    if rank == 0:
+        print(json.dumps(out))
+    if dist:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
 def run_ours(args):
     dist = int(os.environ.get("WORLD_SIZE", "1")) > 1
     rank = int(os.environ.get("RANK", "0"))
@@ -480,6 +654,8 @@ def run_ours(args):
     import bit_quantized_moe_stq1_b200 as S
 
     wl = make_workload(args.workload, S, dev, args.experts)
+    if isinstance(wl, StreamLayer):
+        return run_stream(args, wl, S, dev, dist, n, rank, local)
     for i in range(args.warmup):          # eager warm-up (one-time attribute setup)
         wl.step(i)
     torch.cuda.synchronize()
