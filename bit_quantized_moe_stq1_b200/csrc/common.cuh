@@ -7,6 +7,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/stqmoe.h"
 
 #define STQ_HOST_CHECK(cond, code) \
@@ -22,6 +24,29 @@ static inline stq_status stq_launch_status() {
 }
 
 static inline cudaStream_t stq_cuda_stream(stq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Device ordinals covered by the library's per-device host caches.
+constexpr int kStqMaxDevices = 64;
+
+// Dynamic shared memory above 48 KB needs a per-kernel opt-in, and that attribute belongs
+// to the kernel on one device.  One object per kernel records, per device, the size
+// already allowed, so the driver call runs once per device and size.  Thread-safe.
+struct StqSmemOptIn {
+  std::mutex mu;
+  int allowed[kStqMaxDevices] = {};
+
+  template <typename Kernel>
+  stq_status ensure(Kernel* kernel, int bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStqMaxDevices) return STQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (allowed[dev] >= bytes) return STQ_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return STQ_ERR_CUDA;
+    allowed[dev] = bytes;
+    return STQ_OK;
+  }
+};
 
 // First error wins: only replace a 0 word.
 __device__ __forceinline__ void stq_set_error(int32_t* err, int32_t code) {

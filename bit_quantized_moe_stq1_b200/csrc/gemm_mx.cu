@@ -352,15 +352,9 @@ template <int NT, bool PAIR, bool A8>
 stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmProblem& p,
                        cudaStream_t s) {
   using C = Cfg<NT, PAIR, A8>;
-  static int attr_device = -1;  // the >48 KB shared memory opt-in, once per device
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return STQ_ERR_CUDA;
-  if (attr_device != dev) {
-    if (cudaFuncSetAttribute(w4a8_gemm_kernel<NT, PAIR, A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmem) != cudaSuccess)
-      return STQ_ERR_CUDA;
-    attr_device = dev;
-  }
+  static StqSmemOptIn optin;
+  const stq_status st = optin.ensure(w4a8_gemm_kernel<NT, PAIR, A8>, C::kSmem);
+  if (st != STQ_OK) return st;
   if (p.tiles.max_items <= 0) return STQ_OK;
   const unsigned grid = unsigned(stq_persistent_grid(p.tiles.max_items, C::kCtasPerSm));
   w4a8_gemm_kernel<NT, PAIR, A8><<<grid, kGemmThreads, C::kSmem, s>>>(a, a2, b, p);

@@ -472,15 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <bool PAIR>
 stq_status launch_stq_gemm(const CUtensorMap& b, const StqGemm& p, cudaStream_t s) {
-  static int attr_device = -1;  // the >48 KB shared memory opt-in, once per device
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return STQ_ERR_CUDA;
-  if (attr_device != dev) {
-    if (cudaFuncSetAttribute(stq_gemm_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
-        cudaSuccess)
-      return STQ_ERR_CUDA;
-    attr_device = dev;
-  }
+  static StqSmemOptIn optin;
+  const stq_status st = optin.ensure(stq_gemm_kernel<PAIR>, kSmem);
+  if (st != STQ_OK) return st;
   if (p.tiles.max_items <= 0) return STQ_OK;
   stq_gemm_kernel<PAIR><<<unsigned(stq_persistent_grid(p.tiles.max_items, 1)), kThreads, kSmem, s>>>(b, p);
   return stq_launch_status();

@@ -7,15 +7,21 @@
 // gate/up and down are this library's reading of "run the experts"; the pages give
 // the shapes and formats only.
 //
-// Data flow of moe_expert_forward (one stream, launches in this order):
+// Data flow of moe_expert_forward, launches in this order on the caller's stream:
 //   permute   ids [T,k] -> counts, offsets, perm (pair at each sorted position),
 //             inv (sorted position of each pair), list of touched experts
-//   [MXFP4]   x -> MXFP8 (see gemm_mx.cu)
-//   gate/up   per touched expert and 128-feature tile: g, u (FP32) -> h = silu(g)u
-//             -> h[pos, I] (bf16 for STQ1_0; MXFP8 for MXFP4); the shared expert is
-//             a second set of CTAs (bf16 weights) writing h[P + t, I]
-//   down      per touched expert and 256-row tile: Y[pos, H] (FP32); shared -> Y[P+t]
+//   experts, by format and regime:
+//     STQ1_0, decode regime (this file): gate/up per touched expert and 128-feature
+//             tile, g, u (FP32) -> h = silu(g)u as bf16 h[pos, I]; down per touched
+//             expert and 256-row tile -> Y[pos, H] (FP32).  The BF16 shared expert's
+//             16-row tiles are the first work items of both kernels (h, Y rows P + t).
+//     STQ1_0, prefill regime (gemm_stq.cu) and MXFP4 (gemm_mx.cu): x -> MXFP8 in
+//             sorted pair order, then the tensor-core GEMMs (gate/up with SwiGLU and
+//             the MXFP8 h, then down); the BF16 shared expert as separate launches.
 //   combine   y[t] = sum_s w[t,s] Y[inv[t,s]] (+ Y[P+t]) (+ x[t]) in slot order
+// The MXFP8 shared expert (quantise x, gate/up, down into rows P + t) depends on x
+// alone: it runs on a library-owned side stream, forked after the argument checks and
+// joined before the combine.
 
 #include <mutex>
 
@@ -533,14 +539,16 @@ __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __re
 // ----------------------------------------------------------------------------- host side
 
 // CTAs of a persistent launch: per_sm per SM (the register-limited occupancy), never
-// more than the work items.
+// more than the work items.  The SM count is read once, from the first device that
+// launches (the GPUs of one process are assumed alike).
 int stq_persistent_grid(int items, int per_sm) {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
-  }
+  static const int sms = [] {
+    int dev = 0, n = 0;
+    return cudaGetDevice(&dev) == cudaSuccess &&
+                   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0
+               ? n
+               : 148;
+  }();
   const int cap = per_sm * sms;
   return items < 1 ? 1 : (items < cap ? items : cap);
 }
@@ -609,15 +617,9 @@ extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
 template <int NCH>
 stq_status launch_shared_gateup_wide(const MoeArgs& a, cudaStream_t s) {
   const int smem = kWideWarps * 2 * NCH * 4 * 32 * 4;
-  static int attr_device = -1;  // the >48 KB opt-in, once per device
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return STQ_ERR_CUDA;
-  if (attr_device != dev) {
-    if (cudaFuncSetAttribute(shared_gateup_wide_kernel<NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return STQ_ERR_CUDA;
-    attr_device = dev;
-  }
+  static StqSmemOptIn optin;
+  const stq_status st = optin.ensure(shared_gateup_wide_kernel<NCH>, smem);
+  if (st != STQ_OK) return st;
   StqTimed tm(STQ_K_SHARED_GATE_UP, s);
   shared_gateup_wide_kernel<NCH><<<unsigned(a.I / 16), kWideWarps * 32, smem, s>>>(a);
   return stq_launch_status();
@@ -661,13 +663,9 @@ extern "C" size_t moe_workspace_offset(const moe_desc* d, int32_t region) {
 
 stq_status moe_launch_permute(const int32_t* ids, int P, int E, const MoeWs& ws, cudaStream_t s) {
   const size_t smem = size_t(34) * E * sizeof(int32_t);
-  static int configured_smem = 0;  // dynamic shared memory opt-in (process-wide, set once per size growth)
-  if (int(smem) > configured_smem) {
-    if (cudaFuncSetAttribute(moe_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-      return STQ_ERR_CUDA;
-    configured_smem = int(smem);
-  }
+  static StqSmemOptIn optin;
+  const stq_status st = optin.ensure(moe_permute_kernel, int(smem));
+  if (st != STQ_OK) return st;
   StqTimed tm(STQ_K_PERMUTE, s);
   moe_permute_kernel<<<1, 1024, smem, s>>>(ids, P, E, ws);
   return stq_launch_status();
@@ -692,11 +690,10 @@ struct SideStream {
 };
 
 static stq_status side_stream(SideStream** out) {
-  constexpr int kMaxDevices = 64;
-  static SideStream side[kMaxDevices];
+  static SideStream side[kStqMaxDevices];
   static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return STQ_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStqMaxDevices) return STQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
   SideStream& ss = side[dev];
   if (ss.stream == nullptr) {
@@ -864,7 +861,6 @@ extern "C" stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k,
 // per device with cudaGetSymbolAddress and cached.
 
 constexpr size_t kRouterStaticFloats = size_t(1) << 19;  // 524,288 floats = 2 MiB per GPU
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_router_scratch[kRouterStaticFloats];
 
@@ -872,9 +868,11 @@ namespace {
 
 // Device address of g_router_scratch on the current device (looked up on first use).
 stq_status router_static_scratch(float** out) {
-  static float* addr[kMaxDevices] = {};
+  static float* addr[kStqMaxDevices] = {};
+  static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return STQ_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStqMaxDevices) return STQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_router_scratch) != cudaSuccess || p == nullptr) return STQ_ERR_CUDA;
