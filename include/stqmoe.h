@@ -374,13 +374,13 @@ enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_GATE_UP_STQ_TC, STQ_K_DOWN_STQ_TC, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
- * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm, stq_rmsnorm_bf16 and stq1_pack_ls is
- * bracketed by
- * event records of events[2n] / events[2n+1] on the call's stream (inside stream
- * capture as external event-record nodes of the graph), kinds[n] is set to its
- * STQ_K_* kind and n = count++ (until capacity pairs are used).  events:
- * cudaEvent_t[2*capacity] created with timing.  Process-wide, not thread-safe;
- * NULL uninstalls.  Used by the benchmark to time each kernel on its own stream. */
+ * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm, stq_rmsnorm_bf16 and
+ * stq1_pack_ls is bracketed by event records of events[2n] / events[2n+1] on the
+ * stream it runs on (inside stream capture as external event-record nodes of the
+ * graph), kinds[n] is set to its STQ_K_* kind and n = count++ (until capacity pairs
+ * are used).  events: cudaEvent_t[2*capacity] created with timing.  Process-wide, not
+ * thread-safe; NULL uninstalls.  Used by the benchmark to time each kernel on its own
+ * stream. */
 typedef struct {
   void* const* events;
   int32_t capacity;
