@@ -189,6 +189,39 @@ def test_expert_ffn_stage_consistency():
     assert np.allclose(out["y"], h @ wd.astype(np.float64).T, rtol=1e-13, atol=1e-15)
 
 
+def _ffn_mx_tie_case():
+    """One token through a 32-feature expert whose h is decided by hand.  a = e_0, every
+    gate row 40 e_0 and every up row u e_0 with u = FP32 0x3cd9999a (0.0265625 rounded up),
+    the down projection the identity.  g = 40 and silu(40) = 40 exactly in float64 and in
+    FP32 (exp(-40) vanishes next to 1), so h = 40 u: 1.0625 + 2.98e-8 in float64 but
+    exactly 1.0625 once rounded to FP32, as the GPU's FP32 epilogue holds it.  The
+    smallest power of two 2^k with 1.0625 <= 448 * 2^k is 2^-8 (448 * 2^-9 = 0.875 is too
+    small), so the MXFP8 scale is 2^-8 (UE8M0 119) and h / scale = 272 lies halfway between
+    the E4M3 values 256 (0x78) and 288 (0x79): it rounds to the even 256."""
+    I = H = 32
+    u = np.array([0x3CD9999A], dtype=np.uint32).view(np.float32)[0]
+    A = np.zeros((1, H))
+    A[0, 0] = 1.0
+    Wg = np.zeros((I, H))
+    Wg[:, 0] = 40.0
+    Wu = np.zeros((I, H))
+    Wu[:, 0] = float(u)
+    return Wg, Wu, np.eye(H, I), A
+
+
+def test_expert_ffn_mx_rounds_h_to_f32_before_quantising():
+    """Worked by hand (see _ffn_mx_tie_case): codes 0x78, scale 119, h = y = 1.0.  Without the
+    FP32 rounding of h the tie breaks upward (0x79, 1.125)."""
+    Wg, Wu, Wd, A = _ffn_mx_tie_case()
+    out = M.expert_ffn_mx(Wg, Wu, Wd, A)
+    assert np.all(out["h_codes"] == 0x78) and np.all(out["h_scales"] == 119)
+    assert np.all(out["h"] == 1.0) and np.all(out["y"] == 1.0)
+    # the case has teeth: the same steps without the FP32 rounding give the other code
+    g, _, u, _ = M.expert_gate_up(Wg, Wu, A)
+    hc, hs = F.mxfp8_quantize(M.silu(g) * u)
+    assert np.all(hc == 0x79) and np.all(hs == 119)
+
+
 def test_rms_norm_closed_forms():
     """Constant rows: a / sqrt(a^2 + eps) (eps = 3, a = 1 gives exactly 1/2; eps = 0
     gives sign(a)); a 3-4 row: mean square 12.5, so y = (3, 4) / sqrt(12.5)."""
