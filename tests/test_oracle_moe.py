@@ -189,6 +189,28 @@ def test_expert_ffn_stage_consistency():
     assert np.allclose(out["y"], h @ wd.astype(np.float64).T, rtol=1e-13, atol=1e-15)
 
 
+def test_expert_ffn_bf16h_rounds_h_to_nearest_even_bf16():
+    """Worked by hand: activation e_0, gate rows 64 h*, up rows 1/64, so g >= 37 and
+    silu(g) = g exactly (exp(-g) vanishes next to 1), and h = h* exactly.  h* = 1 + 2^-8 is
+    a BF16 tie that goes down to the even 1.0; 1 + 3 * 2^-8 a tie that goes up to the even
+    1.015625; 1 + 2^-8 + 2^-10 lies above a tie and goes up to 1.0078125.  The down
+    projection (identity rows and one row of ones) must see the rounded h."""
+    H, I = 4, 3
+    hstar = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 + 2.0 ** -8 + 2.0 ** -10])
+    X = np.zeros((1, H))
+    X[0, 0] = 1.0
+    Wg = np.zeros((I, H))
+    Wg[:, 0] = 64.0 * hstar
+    Wu = np.zeros((I, H))
+    Wu[:, 0] = 1.0 / 64.0
+    Wd = np.vstack([np.eye(I), np.ones((1, I))])
+    out = M.expert_ffn_bf16h(Wg, Wu, Wd, X)
+    expect_h = np.array([1.0, 1.015625, 1.0078125])
+    assert np.array_equal(out["h"][0], expect_h)
+    assert np.array_equal(out["h_bits"][0], np.array([0x3F80, 0x3F82, 0x3F81]))
+    assert np.array_equal(out["y"][0], np.append(expect_h, expect_h.sum()))
+
+
 def _ffn_mx_tie_case():
     """One token through a 32-feature expert whose h is decided by hand.  a = e_0, every
     gate row 40 e_0 and every up row u e_0 with u = FP32 0x3cd9999a (0.0265625 rounded up),
