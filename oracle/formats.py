@@ -49,7 +49,8 @@ def fp16_encode_rne(v):
 def bf16_decode(bits):
     """bfloat16 = the top 16 bits of an IEEE binary32 -> float64."""
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
-    return b.view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # signalling-NaN patterns widen to a quiet NaN
+        return b.view(np.float32).astype(np.float64)
 
 
 def bf16_encode_rne(v):
