@@ -43,6 +43,7 @@ class MoeWeights(ctypes.Structure):
 SIGNATURES = {
     "stq_status_string": (ctypes.c_char_p, [_i32]),
     "stq_abi_version": (_i32, []),
+    "stq_kernel_kind_name": (ctypes.c_char_p, [_i32]),
     "stq_read_error": (_i32, [_vp, _vp]),
     "stq1_pack": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "stq1_unpack": (_i32, [_vp, _i64, _i64, _vp, _vp]),

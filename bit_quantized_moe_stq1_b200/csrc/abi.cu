@@ -1,4 +1,6 @@
-// Status strings, version and error-word access of the C ABI.
+// Status strings, version, error-word access and instrumentation of the C ABI.
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_internal.cuh"
 
 extern "C" const char* stq_status_string(stq_status s) {
@@ -39,6 +41,17 @@ extern "C" stq_status moe_get_device_error(void* workspace, stq_stream_t stream)
 
 static stq_timing* g_timing = nullptr;
 
+// Names of the STQ_K_* kernel kinds, in enum order.
+static const char* const kKindNames[] = {"router_logits", "router_topk", "permute", "quant_x", "gate_up", "down",
+                                         "combine", "gemv", "gemm", "gate_up_mx", "down_mx", "plan",
+                                         "shared_gate_up", "shared_down", "rmsnorm", "pack_ls", "gate_up_stq_tc",
+                                         "down_stq_tc"};
+static_assert(sizeof(kKindNames) / sizeof(kKindNames[0]) == STQ_K_COUNT, "one name per kernel kind");
+
+extern "C" const char* stq_kernel_kind_name(int32_t kind) {
+  return kind >= 0 && kind < STQ_K_COUNT ? kKindNames[kind] : "unknown";
+}
+
 extern "C" stq_status stq_set_timing(stq_timing* t) {
   g_timing = t;
   return STQ_OK;
@@ -50,6 +63,8 @@ static cudaError_t record(cudaEvent_t ev, cudaStream_t st, bool capturing) {
 }
 
 StqTimed::StqTimed(int kind, cudaStream_t st) : s(st), slot(-1), capturing(false) {
+  // an NVTX range per launch, named by kind (a no-op unless a profiler is attached)
+  nvtxRangePushA(stq_kernel_kind_name(kind));
   stq_timing* t = g_timing;
   if (t == nullptr || t->count >= t->capacity) return;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -63,4 +78,5 @@ StqTimed::StqTimed(int kind, cudaStream_t st) : s(st), slot(-1), capturing(false
 StqTimed::~StqTimed() {
   if (slot >= 0 && g_timing != nullptr)
     record(static_cast<cudaEvent_t>(g_timing->events[2 * slot + 1]), s, capturing);
+  nvtxRangePop();
 }

@@ -389,6 +389,12 @@ typedef struct {
 } stq_timing;
 stq_status stq_set_timing(stq_timing* t);
 
+/* Name of an STQ_K_* kind ("gate_up", "down_mx", ...; "unknown" outside the enum).  Static
+ * storage.  Every kernel launch of the calls listed above is also wrapped in an NVTX range
+ * of this name (host side, whether or not timing is installed), so a profiler can select
+ * kernels by it (ncu --nvtx --nvtx-include "gate_up/"). */
+const char* stq_kernel_kind_name(int32_t kind);
+
 #ifdef __cplusplus
 }
 #endif

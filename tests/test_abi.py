@@ -179,3 +179,7 @@ def test_timing_kinds_match_the_header():
     assert names[-1] == "STQ_K_COUNT"
     expect = [n[len("STQ_K_"):].lower() for n in names[:-1]]
     assert expect == list(S.KERNEL_KINDS)
+    # the library's own names (also its NVTX range names) agree
+    assert [S.lib.stq_kernel_kind_name(i).decode() for i in range(len(expect))] == expect
+    assert S.lib.stq_kernel_kind_name(len(expect)).decode() == "unknown"
+    assert S.lib.stq_kernel_kind_name(-1).decode() == "unknown"
