@@ -5,6 +5,9 @@ their dtype/shape on the host, and passes raw device pointers and sizes to the C
 ABI declared in include/stqmoe.h.  All arithmetic happens in the CUDA kernels of
 the library; there is no CPU fallback.  If the shared library is missing or
 cannot be loaded, importing this package raises.
+
+STQMOE_CHECKED=1 in the environment loads the checked build (libstqmoe_checked.so,
+`build.py --checked`): same ABI, with device-side re-checks of data-derived indices.
 """
 
 import ctypes
@@ -13,7 +16,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libstqmoe.so")
+CHECKED = os.environ.get("STQMOE_CHECKED", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libstqmoe_checked.so" if CHECKED else "libstqmoe.so")
 
 STQ_OK = 0
 STATUS = {
@@ -44,6 +48,7 @@ SIGNATURES = {
     "stq_status_string": (ctypes.c_char_p, [_i32]),
     "stq_abi_version": (_i32, []),
     "stq_kernel_kind_name": (ctypes.c_char_p, [_i32]),
+    "stq_checked_build": (_i32, []),
     "stq_read_error": (_i32, [_vp, _vp]),
     "stq1_pack": (_i32, [_vp, _i64, _i64, _vp, _vp, _vp]),
     "stq1_unpack": (_i32, [_vp, _i64, _i64, _vp, _vp]),
@@ -115,7 +120,8 @@ class KernelTimer:
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_quantized_moe_stq1_b200/build.py`")
+        how = " --checked" if CHECKED else ""
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_quantized_moe_stq1_b200/build.py{how}`")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

@@ -1,9 +1,10 @@
 """Build libstqmoe.so in-tree from csrc/*.cu for sm_100a.
 
-    python bit_quantized_moe_stq1_b200/build.py
+    python bit_quantized_moe_stq1_b200/build.py [--checked]
 
 Object files go to <repo>/_build/ (not committed); the shared library is written
-next to this file so that it travels with the source tree.
+next to this file so that it travels with the source tree.  --checked builds
+libstqmoe_checked.so (-DSTQ_CHECKED=1) from objects under _build/checked/.
 """
 
 import concurrent.futures
@@ -17,6 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libstqmoe.so")
+CHECKED_LIB = os.path.join(HERE, "libstqmoe_checked.so")
 BUILD = os.path.join(ROOT, "_build")
 
 NVCC_FLAGS = [
@@ -42,32 +44,37 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose=False):
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose=False, checked=False):
+    """Compile csrc/*.cu and link libstqmoe.so; checked=True builds libstqmoe_checked.so
+    (-DSTQ_CHECKED=1: device-side re-checks of data-derived indices) from its own objects."""
+    bdir = os.path.join(BUILD, "checked") if checked else BUILD
+    lib = CHECKED_LIB if checked else LIB
+    flags = NVCC_FLAGS + (["-DSTQ_CHECKED=1"] if checked else [])
+    os.makedirs(bdir, exist_ok=True)
     nvcc = _nvcc()
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
     jobs = []
     objs = []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if _stale(obj, [src] + headers):
-            jobs.append([nvcc] + NVCC_FLAGS + ["-c", src, "-o", obj])
+            jobs.append([nvcc] + flags + ["-c", src, "-o", obj])
     with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as ex:
         for cmd, res in zip(jobs, ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), jobs)):
             if verbose or res.returncode:
                 sys.stderr.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
             if res.returncode:
                 raise RuntimeError("nvcc failed for " + cmd[-3])
-    if jobs or _stale(LIB, objs):
-        cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB] + objs
+    if jobs or _stale(lib, objs):
+        cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", lib] + objs
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode:
             sys.stderr.write(res.stdout + res.stderr)
             raise RuntimeError("link failed")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, checked="--checked" in sys.argv))

@@ -21,6 +21,14 @@ extern "C" const char* stq_status_string(stq_status s) {
 
 extern "C" int32_t stq_abi_version(void) { return STQMOE_ABI_VERSION; }
 
+extern "C" int32_t stq_checked_build(void) {
+#if defined(STQ_CHECKED) && STQ_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 extern "C" stq_status stq_read_error(int32_t* err, stq_stream_t stream) {
   if (err == nullptr) return STQ_ERR_INVALID_ARG;
   cudaStream_t s = stq_cuda_stream(stream);

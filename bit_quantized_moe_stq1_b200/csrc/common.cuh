@@ -53,6 +53,21 @@ __device__ __forceinline__ void stq_set_error(int32_t* err, int32_t code) {
   if (err != nullptr) atomicCAS(err, 0, code);
 }
 
+// Checked build (-DSTQ_CHECKED=1, libstqmoe_checked.so): kernels re-check the indices they
+// take from data (expert ids from the touched list, token indices from the permutation,
+// sorted positions from the inverse map) before using them.  A failed check records
+// STQ_ERR_DEVICE in the error word and the access is skipped; nothing traps.  In the
+// default build STQ_DCHECK is the constant true and its condition is not evaluated.
+#if defined(STQ_CHECKED) && STQ_CHECKED
+__device__ __forceinline__ bool stq_dcheck(bool ok, int32_t* err) {
+  if (!ok) stq_set_error(err, STQ_ERR_DEVICE);
+  return ok;
+}
+#define STQ_DCHECK(cond, err) stq_dcheck((cond), (err))
+#else
+#define STQ_DCHECK(cond, err) true
+#endif
+
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
 
 // float -> bf16 bits, round to nearest even (the library conversion intrinsic).

@@ -393,7 +393,7 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
   (void)slots;
   const int P = a.P;
   // 1. activations -> MXFP8 in sorted (expert-grouped) order
-  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.xq, a.xs, s);
+  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.T, a.err, a.xq, a.xs, s);
   if (st != STQ_OK) return st;
   // 2. N tiles of the touched experts: the down projection takes the 240-wide tile from
   // 128 tokens per expert on average, the gate/up pair (whose SwiGLU/MXFP8 epilogue and

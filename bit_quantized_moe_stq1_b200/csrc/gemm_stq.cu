@@ -485,7 +485,7 @@ stq_status launch_stq_gemm(const CUtensorMap& b, const StqGemm& p, cudaStream_t 
 stq_status moe_stq_prefill_experts(const MoeArgs& a, int slots, cudaStream_t s) {
   const int P = a.P;
   // 1. activations -> MXFP8 g32 in sorted (expert-grouped) order
-  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.xq, a.xs, s);
+  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.T, a.err, a.xq, a.xs, s);
   if (st != STQ_OK) return st;
   // 2. N tiles of 112 tokens of the touched experts
   if ((st = stq_tile_plan_launch(a.counts, a.E, kNT, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;

@@ -427,7 +427,9 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
     const int bid = item - a.n_shared_cta;
     const int slot = bid / per_expert, ct = bid % per_expert;
     const int e = a.tlist[slot];
+    if (!STQ_DCHECK(e >= 0 && e < a.E, a.err)) continue;
     const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+    if (!STQ_DCHECK(pos0 >= 0 && cnt >= 0 && pos0 + cnt <= a.P, a.err)) continue;
     const int f0 = ct * 128 + warp * 32;
     const uint8_t* gb = a.wg + size_t(e) * mat;
     const uint8_t* ub = a.wu + size_t(e) * mat;
@@ -435,7 +437,9 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
                             ub + size_t(f0 / 16) * tstride, ub + size_t(f0 / 16 + 1) * tstride};
     for (int c0 = 0; c0 < cnt; c0 += 8) {
       const int j = c0 + g;
-      const uint16_t* xrow = j < cnt ? a.x + size_t(a.perm[pos0 + j] / a.k) * a.H : nullptr;
+      const int tok = j < cnt ? a.perm[pos0 + j] / a.k : -1;
+      const uint16_t* xrow =
+          (j < cnt && STQ_DCHECK(tok >= 0 && tok < a.T, a.err)) ? a.x + size_t(tok) * a.H : nullptr;
       float acc[4][4] = {};
       stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
 #pragma unroll
@@ -472,7 +476,9 @@ __global__ void __launch_bounds__(128, 3) moe_down_stq_kernel(MoeArgs a) {
     const int bid = item - a.n_shared_cta;
     const int slot = bid / per_expert, ct = bid % per_expert;
     const int e = a.tlist[slot];
+    if (!STQ_DCHECK(e >= 0 && e < a.E, a.err)) continue;
     const int pos0 = a.offsets[e], cnt = a.offsets[e + 1] - pos0;
+    if (!STQ_DCHECK(pos0 >= 0 && cnt >= 0 && pos0 + cnt <= a.P, a.err)) continue;
     const int r0 = ct * 256 + warp * 64;
     const uint8_t* db = a.wd + size_t(e) * mat;
     const uint8_t* tb[4] = {db + size_t(r0 / 16) * tstride, db + size_t(r0 / 16 + 1) * tstride,
@@ -498,7 +504,8 @@ __global__ void __launch_bounds__(128, 3) moe_down_stq_kernel(MoeArgs a) {
 
 __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __restrict__ Y,
                                    const int32_t* __restrict__ inv, const float* __restrict__ topk_w, int has_shared,
-                                   const uint16_t* __restrict__ resid, void* __restrict__ y, int out_fp32) {
+                                   const uint16_t* __restrict__ resid, void* __restrict__ y, int out_fp32,
+                                   int32_t* err) {
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int h4 = H / 4;
   if (idx >= int64_t(T) * h4) return;
@@ -506,7 +513,7 @@ __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __re
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < k; ++s) {
     const int pos = inv[size_t(t) * k + s];
-    if (pos < 0) continue;
+    if (pos < 0 || !STQ_DCHECK(pos < P, err)) continue;
     const float w = topk_w[size_t(t) * k + s];
     const float4 v = reinterpret_cast<const float4*>(Y + size_t(pos) * H)[c];
     acc.x = fmaf(w, v.x, acc.x);
@@ -677,7 +684,8 @@ stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const f
   if (n == 0) return STQ_OK;
   StqTimed tm(STQ_K_COMBINE, s);
   moe_combine_kernel<<<unsigned(ceil_div<int64_t>(n, 256)), 256, 0, s>>>(
-      d.T, d.H, d.k, P, ws.Y, ws.inv, topk_w, has_shared ? 1 : 0, d.add_residual ? x : nullptr, y, d.out_fp32);
+      d.T, d.H, d.k, P, ws.Y, ws.inv, topk_w, has_shared ? 1 : 0, d.add_residual ? x : nullptr, y, d.out_fp32,
+      ws.err);
   return stq_launch_status();
 }
 

@@ -75,6 +75,8 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
 // BF16 -> MXFP8 quantisation launch (pack.cu).
 stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales,
                                      cudaStream_t s);
-// Same, with output row r taken from input row rowmap[r] / k (gather into sorted pair order).
+// Same, with output row r taken from input row rowmap[r] / k (gather into sorted pair order)
+// of src_rows input rows; err: the error word of the checked build's source-row check.
 stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int64_t K, const int32_t* rowmap, int k,
-                                            uint8_t* codes, uint8_t* scales, cudaStream_t s);
+                                            int64_t src_rows, int32_t* err, uint8_t* codes, uint8_t* scales,
+                                            cudaStream_t s);

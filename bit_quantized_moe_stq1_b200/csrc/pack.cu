@@ -308,7 +308,8 @@ template <int RPB>
 __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                int64_t K, uint8_t* __restrict__ codes,
                                                                uint8_t* __restrict__ scales,
-                                                               const int32_t* __restrict__ rowmap, int k) {
+                                                               const int32_t* __restrict__ rowmap, int k,
+                                                               int64_t src_rows, int32_t* err) {
   const int part = int(threadIdx.x & 3);
   const int64_t col8 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // 8-element chunk of the row
   const bool active = col8 < K / 8;                                     // whole 4-thread groups
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* _
       const int64_t row = r0 + j;
       if (active && row < rows) {
         const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
-        raw[j] = *reinterpret_cast<const uint4*>(x + src * K + col8 * 8);
+        if (STQ_DCHECK(src >= 0 && src < src_rows, err)) raw[j] = *reinterpret_cast<const uint4*>(x + src * K + col8 * 8);
       }
     }
 #pragma unroll
@@ -459,21 +460,26 @@ stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K,
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
   if (rows >= kQuantMultiRow)
-    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1);
+    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1, rows,
+                                                                   nullptr);
   else
-    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1);
+    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1, rows,
+                                                                   nullptr);
   return stq_launch_status();
 }
 
 stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int64_t K, const int32_t* rowmap, int k,
-                                            uint8_t* codes, uint8_t* scales, cudaStream_t s) {
+                                            int64_t src_rows, int32_t* err, uint8_t* codes, uint8_t* scales,
+                                            cudaStream_t s) {
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
   if (rows >= kQuantMultiRow)
-    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k);
+    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k, src_rows,
+                                                                   err);
   else
-    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k);
+    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k, src_rows,
+                                                                   err);
   return stq_launch_status();
 }
 

@@ -389,6 +389,13 @@ typedef struct {
 } stq_timing;
 stq_status stq_set_timing(stq_timing* t);
 
+/* 1 for the checked build (libstqmoe_checked.so, compiled with -DSTQ_CHECKED=1), 0 otherwise.
+ * The checked build has the same ABI; its kernels re-check every index they take from data
+ * (expert ids of the touched list, token indices from the permutation, sorted positions from
+ * the inverse map, gathered source rows) and, instead of using a bad one, record
+ * STQ_ERR_DEVICE in the error word and skip the access. */
+int32_t stq_checked_build(void);
+
 /* Name of an STQ_K_* kind ("gate_up", "down_mx", ...; "unknown" outside the enum).  Static
  * storage.  Every kernel launch of the calls listed above is also wrapped in an NVTX range
  * of this name (host side, whether or not timing is installed), so a profiler can select
