@@ -51,12 +51,14 @@ np.savez(sys.argv[2], **out)
 
 
 def test_checked_build_matches_the_default_build(tmp_path):
+    # the default library is the one this process has loaded; only the checked one may
+    # need building here (nvcc is on the box), and building it touches nothing else
     spec = importlib.util.spec_from_file_location("_stq_build", os.path.join(ROOT, "bit_quantized_moe_stq1_b200",
                                                                              "build.py"))
     b = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(b)
-    b.build()
-    b.build(checked=True)
+    if not os.path.exists(b.CHECKED_LIB):
+        b.build(checked=True)
     outs = []
     for checked in (0, 1):
         path = str(tmp_path / f"out{checked}.npz")
