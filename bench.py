@@ -409,7 +409,7 @@ class StreamLayer(MoeLayers):
         if self.copy_events is not None:
             ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             ev[0].record()
-        S.SlotBank.copy(le, ls, self.host, self.slots)
+        self.bank.copy(le, ls, self.host, self.slots)
         if self.copy_events is not None:
             ev[1].record()
             self.copy_events.append(ev)

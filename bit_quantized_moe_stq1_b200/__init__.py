@@ -73,7 +73,7 @@ SIGNATURES = {
     "stq_slot_bank_destroy": (None, [_vp]),
     "stq_slot_bank_map": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp]),
     "stq_slot_bank_resident": (_i32, [_vp, _vp]),
-    "stq_slot_bank_copy": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "stq_slot_bank_copy": (_i32, [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "stq_rmsnorm_bf16": (_i32, [_vp, _i64, _i64, ctypes.c_float, _vp, _vp]),
 }
 
@@ -436,17 +436,26 @@ class SlotBank:
         _check(lib.stq_slot_bank_resident(self._h, out.ctypes.data), "stq_slot_bank_resident")
         return out
 
-    @staticmethod
-    def copy(load_expert, load_slot, src, dst, stream=None):
-        """Copy experts into slots: src / dst are lists of expert-major tensors (host, ideally
-        pinned, and device), one per matrix, each [experts or slots, ...] with equal rows."""
+    def copy(self, load_expert, load_slot, src, dst, stream=None):
+        """Copy experts into slots: src / dst are lists of contiguous expert-major tensors, one
+        per matrix: src[m] [n_experts, ...] (host, ideally pinned), dst[m] [n_slots, ...] on the
+        GPU, with the same bytes per expert."""
         import numpy as np
 
+        if len(src) != len(dst):
+            raise ValueError("one destination per source matrix")
+        for a, b in zip(src, dst):
+            if a.shape[0] != self.n_experts or b.shape[0] != self.n_slots:
+                raise ValueError("source rows must be n_experts and destination rows n_slots")
+            if not (a.is_contiguous() and b.is_contiguous()) or not b.is_cuda:
+                raise ValueError("contiguous sources; contiguous destinations on the GPU")
+            if a[0].numel() * a.element_size() != b[0].numel() * b.element_size():
+                raise ValueError("bytes per expert differ between source and destination")
         le = np.ascontiguousarray(load_expert, dtype=np.int32)
         ls = np.ascontiguousarray(load_slot, dtype=np.int32)
         n_m = len(src)
         srcs = (ctypes.c_void_p * n_m)(*[t.data_ptr() for t in src])
         dsts = (ctypes.c_void_p * n_m)(*[t.data_ptr() for t in dst])
         sizes = (ctypes.c_size_t * n_m)(*[t[0].numel() * t.element_size() for t in src])
-        _check(lib.stq_slot_bank_copy(le.ctypes.data, ls.ctypes.data, le.size, n_m, srcs, dsts, sizes,
+        _check(lib.stq_slot_bank_copy(self._h, le.ctypes.data, ls.ctypes.data, le.size, n_m, srcs, dsts, sizes,
                                       _stream(stream)), "stq_slot_bank_copy")

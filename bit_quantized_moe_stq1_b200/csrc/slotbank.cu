@@ -89,16 +89,21 @@ extern "C" stq_status stq_slot_bank_resident(const stq_slot_bank* b, int32_t* sl
   return STQ_OK;
 }
 
-extern "C" stq_status stq_slot_bank_copy(const int32_t* load_expert, const int32_t* load_slot, int32_t n_loads,
-                                         int32_t n_mats, const void* const* src, void* const* dst,
+extern "C" stq_status stq_slot_bank_copy(const stq_slot_bank* b, const int32_t* load_expert, const int32_t* load_slot,
+                                         int32_t n_loads, int32_t n_mats, const void* const* src, void* const* dst,
                                          const size_t* mat_bytes, stq_stream_t stream) {
-  STQ_HOST_CHECK(n_loads >= 0 && n_mats >= 0, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(b != nullptr && n_loads >= 0 && n_mats >= 0, STQ_ERR_INVALID_ARG);
   if (n_loads == 0 || n_mats == 0) return STQ_OK;
   STQ_HOST_CHECK(load_expert != nullptr && load_slot != nullptr && src != nullptr && dst != nullptr &&
                      mat_bytes != nullptr,
                  STQ_ERR_INVALID_ARG);
   for (int32_t m = 0; m < n_mats; ++m) STQ_HOST_CHECK(src[m] != nullptr && dst[m] != nullptr, STQ_ERR_INVALID_ARG);
-  for (int32_t i = 0; i < n_loads; ++i) STQ_HOST_CHECK(load_expert[i] >= 0 && load_slot[i] >= 0, STQ_ERR_INVALID_ARG);
+  // the arrays hold the bank's n_experts (source) and n_slots (destination) matrices: an
+  // index outside them is refused before any copy is enqueued
+  for (int32_t i = 0; i < n_loads; ++i)
+    STQ_HOST_CHECK(load_expert[i] >= 0 && load_expert[i] < b->n_experts && load_slot[i] >= 0 &&
+                       load_slot[i] < b->n_slots,
+                   STQ_ERR_INVALID_ARG);
   cudaStream_t s = stq_cuda_stream(stream);
   // one copy per matrix and expert
   for (int32_t i = 0; i < n_loads; ++i)

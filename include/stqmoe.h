@@ -348,12 +348,13 @@ stq_status stq_slot_bank_resident(const stq_slot_bank* bank, int32_t* slot_exper
 
 /* Copy the listed experts' matrices into their slots: for load i and matrix m,
  * mat_bytes[m] bytes from src[m] + load_expert[i] * mat_bytes[m] (the full expert-major
- * array, normally pinned host memory so the copy is asynchronous) to dst[m] +
- * load_slot[i] * mat_bytes[m] (the slot bank's expert-major device array).  One
- * cudaMemcpyAsync per load and matrix on `stream`; asynchronous.  STQ_ERR_INVALID_ARG
- * for null pointers or negative entries, STQ_ERR_CUDA if a copy cannot be enqueued. */
-stq_status stq_slot_bank_copy(const int32_t* load_expert, const int32_t* load_slot, int32_t n_loads,
-                              int32_t n_mats, const void* const* src, void* const* dst,
+ * array of the bank's n_experts matrices, normally pinned host memory so the copy is
+ * asynchronous) to dst[m] + load_slot[i] * mat_bytes[m] (the slot array of its n_slots
+ * matrices, device memory).  One cudaMemcpyAsync per load and matrix on `stream`;
+ * asynchronous.  STQ_ERR_INVALID_ARG (nothing enqueued) for null pointers or an expert or
+ * slot index outside the bank's sizes; STQ_ERR_CUDA if a copy cannot be enqueued. */
+stq_status stq_slot_bank_copy(const stq_slot_bank* bank, const int32_t* load_expert, const int32_t* load_slot,
+                              int32_t n_loads, int32_t n_mats, const void* const* src, void* const* dst,
                               const size_t* mat_bytes, stq_stream_t stream);
 
 /* ------------------------------------------------------------------------- */

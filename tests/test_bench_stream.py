@@ -60,7 +60,7 @@ def test_streamed_layer_host_path(monkeypatch, capsys):
         rows, K = w.shape
         return torch.zeros(rows * K // 256 * 42, dtype=torch.uint8)
 
-    def copy(le, ls, src, dst, stream=None):
+    def copy(self, le, ls, src, dst, stream=None):
         for m in range(len(src)):
             for e, s in zip(le.tolist(), ls.tolist()):
                 dst[m][s].copy_(src[m][e])
@@ -84,7 +84,7 @@ def test_streamed_layer_host_path(monkeypatch, capsys):
     monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
     monkeypatch.setattr(S, "stq1_pack", pack)
     monkeypatch.setattr(S, "moe_expert_forward", forward)
-    monkeypatch.setattr(S.SlotBank, "copy", staticmethod(copy))
+    monkeypatch.setattr(S.SlotBank, "copy", copy)
     monkeypatch.setattr(S, "KernelTimer", _Timer)
     monkeypatch.setattr(bench, "ClockSampler", _Clock)
     # the fake pack reads only the shape: skip drawing full-size weights

@@ -108,16 +108,34 @@ def test_create_rejects_bad_sizes(S):
 
 
 def test_copy_argument_checks_need_no_gpu(S):
+    """Every case below fails an argument check, which returns before any CUDA call."""
     lib = S.lib
+    bank = S.SlotBank(32, 4)
+    h = bank._h
     e = (ctypes.c_int32 * 1)(0)
     s = (ctypes.c_int32 * 1)(0)
-    assert lib.stq_slot_bank_copy(e, s, 0, 3, None, None, None, None) == 0          # nothing to copy
-    assert lib.stq_slot_bank_copy(e, s, 1, 1, None, None, None, None) == -1         # null arrays
+    assert lib.stq_slot_bank_copy(h, e, s, 0, 3, None, None, None, None) == 0       # nothing to copy
+    assert lib.stq_slot_bank_copy(None, e, s, 1, 1, None, None, None, None) == -1   # no bank
+    assert lib.stq_slot_bank_copy(h, e, s, 1, 1, None, None, None, None) == -1      # null arrays
     src = (ctypes.c_void_p * 1)(None)
     dst = (ctypes.c_void_p * 1)(None)
     sz = (ctypes.c_size_t * 1)(16)
-    assert lib.stq_slot_bank_copy(e, s, 1, 1, src, dst, sz, None) == -1             # null matrix pointers
-    neg = (ctypes.c_int32 * 1)(-1)
+    assert lib.stq_slot_bank_copy(h, e, s, 1, 1, src, dst, sz, None) == -1          # null matrix pointers
     src2 = (ctypes.c_void_p * 1)(1 << 20)
     dst2 = (ctypes.c_void_p * 1)(1 << 21)
-    assert lib.stq_slot_bank_copy(neg, s, 1, 1, src2, dst2, sz, None) == -1         # negative expert
+    for ex, sl in ((-1, 0), (32, 0), (0, -1), (0, 4)):                              # outside 32 experts, 4 slots
+        ee, ss = (ctypes.c_int32 * 1)(ex), (ctypes.c_int32 * 1)(sl)
+        assert lib.stq_slot_bank_copy(h, ee, ss, 1, 1, src2, dst2, sz, None) == -1, (ex, sl)
+
+
+def test_copy_binding_checks_shapes(S):
+    import torch
+
+    bank = S.SlotBank(8, 2)
+    src = [torch.zeros((8, 64), dtype=torch.uint8)]
+    with pytest.raises(ValueError):
+        bank.copy([0], [0], src, [torch.zeros((3, 64), dtype=torch.uint8)])   # 3 rows for 2 slots
+    with pytest.raises(ValueError):
+        bank.copy([0], [0], src, [])                                           # one destination per matrix
+    with pytest.raises(ValueError):
+        bank.copy([0], [0], src, [torch.zeros((2, 64), dtype=torch.uint8)])   # destination not on the GPU

@@ -45,7 +45,7 @@ def test_moe_stq_slot_bank_streaming(S):
     for c in range(calls):
         ids = ids_all[c * T:(c + 1) * T].contiguous()
         slot_ids, le, ls = bank.map(ids.numpy())
-        S.SlotBank.copy(le, ls, host, bank_w)
+        bank.copy(le, ls, host, bank_w)
         n_loads += le.size
         sid = torch.from_numpy(slot_ids).to(DEV)
         tw = tw_all[c * T:(c + 1) * T].contiguous().to(DEV)
