@@ -51,7 +51,9 @@ NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense
 MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (2.109465e9 + 6.812928e6) / 157}  # decode_mx, 157 touched
 # DRAM bytes (read + write) of one full-size launch, from an ncu capture of the same workload
 # and kernel build; an entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_LAUNCH = {("decode_stq", "gate_up"): 285.818880e6 + 8.129536e6,
+MEASURED_TRAFFIC_PER_LAUNCH = {("stq_matvec", "gemv"): 2.09e6, ("w4a8_gemm", "gemm"): 7.55e6,
+                               ("stq_pack_ls", "pack_ls"): 50.41e6,
+                               ("decode_stq", "gate_up"): 285.818880e6 + 8.129536e6,
                                ("prefill_stq", "gate_up_stq_tc"): 1.608519e9 + 64.757248e6,
                                ("prefill_w4a8", "gate_up_mx"): 3.751041e9 + 71.260672e6}
 
