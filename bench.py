@@ -43,6 +43,10 @@ BF16_MAT = I * H * 2                        # 25,165,824
 MX8_MAT = I * H + I * H // 32               # 12,976,128 per MXFP8 matrix (codes + scales)
 ROUTER_BYTES = E * H * 2                    # 3,145,728
 NOMINAL_FP8_OVER_BF16 = 2.0                 # dense FP8 (kind::mxf8f6f4) / dense BF16 tensor rate
+# A second tensor peak for the block-scaled GEMMs: back-to-back tcgen05 kind::mxf8f6f4 MMAs
+# (M = 128, N >= 128, one CTA per SM, no memory traffic) measured 8,190 MACs per clock per
+# SM on this machine's B200s; at the 1965 MHz maximum SM clock of 148 SMs that is 4.76 PFLOP/s.
+MMA_MICROBENCH_TFLOPS = 2 * 8190 * 148 * 1.965e9 / 1e12
 
 # DRAM bytes (read + write) per touched expert of one decode-size launch, from one ncu
 # capture of the same kernel build on a smaller case (named profile under profiles/); a
@@ -540,8 +544,11 @@ def whole_job_rate(n_ranks, units_per_rank_step, ms_per_step):
     return n_ranks * units_per_rank_step / (ms_per_step * 1e-3)
 
 
-def base_config(wl):
-    return {"workload": wl.name, "experts": E, "tokens_per_step": wl.tokens_per_step()}
+def base_config(name, n):
+    """The workload's configuration: the same dict in both arms (no measured values)."""
+    return {"workload": name, "experts": E, "tokens_per_step": tokens_of(name),
+            "l2": "inputs larger than L2: per-step weights exceed L2, batches rotate over 8",
+            "parallelism": f"replicas x{n}"}
 
 
 def run_stream(args, wl, S, dev, dist, n, rank, local):
@@ -619,11 +626,11 @@ def run_stream(args, wl, S, dev, dist, n, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded generators; random weights on the STQ1_0 grid; Zipf routing)",
-        "config": {**base_config(wl), "slots": wl.n_slots, "experts_loaded_per_step": loads,
+        "config": base_config(wl.name, n),
+        "stream": {"slots": wl.n_slots, "experts_loaded_per_step": loads,
                    "distinct_experts_per_step": distinct, "h2d_weight_bytes_per_step": loads * 3 * STQ_MAT,
-                   "l2": "inputs larger than L2: the bank (96 slots x 6.2 MB) and the copied experts",
-                   "parallelism": f"replicas x{n}",
-                   "timing": "eager steps (host slot mapping, expert copies, the layer), CUDA events"},
+                   "l2": "inputs larger than L2: the bank (96 slots x 6.2 MB) and the copied experts"},
+        "timing": "eager steps (host slot mapping, expert copies, the layer), CUDA events",
         "roofline": {"bound": "h2d", "kernel": "expert copies (cudaMemcpyAsync, pinned host to HBM)",
                      "achieved": copy_gbs, "peak": link_gbs, "unit": "GB/s",
                      "frac": copy_gbs / link_gbs if copy_gbs else None,
@@ -638,7 +645,7 @@ def run_stream(args, wl, S, dev, dist, n, rank, local):
         "clocks": clocks,
     }
     if rank == 0 and not dist and not args.no_cpu:
-        out["cpu_baseline"] = cpu_baseline(wl, dev)
+        out["cpu_baseline"] = cpu_baseline(wl.name)
     if rank == 0:
         print(json.dumps(out))
     if dist:
@@ -646,33 +653,22 @@ def run_stream(args, wl, S, dev, dist, n, rank, local):
         torch.distributed.destroy_process_group()
 
 
-def run_ours(args):
-    dist = int(os.environ.get("WORLD_SIZE", "1")) > 1
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    n = int(os.environ.get("WORLD_SIZE", "1"))
-    if dist:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    import bit_quantized_moe_stq1_b200 as S
-
-    wl = make_workload(args.workload, S, dev, args.experts)
-    if isinstance(wl, StreamLayer):
-        return run_stream(args, wl, S, dev, dist, n, rank, local)
-    for i in range(args.warmup):          # eager warm-up (one-time attribute setup)
+def measure(wl, S, dev, dist, n, local, steps, warmup):
+    """Time one workload: CUDA graph replays of whole steps (max over ranks), per-kernel
+    CUDA events, the end-to-end pass, clocks and the dominant kernel's roofline."""
+    for i in range(warmup):          # eager warm-up (one-time attribute setup)
         wl.step(i)
     torch.cuda.synchronize()
     graphs = capture(wl)
     with ClockSampler(local) as clk:
-        ms = timed_replays(graphs, args.steps, args.warmup, dist)
+        ms = timed_replays(graphs, steps, warmup, dist)
     clocks = clk.summary()
-    ms_step = max_over_ranks([ms], dev, dist)[0] / args.steps
-    kt = kernel_times(S, wl, args.steps, args.warmup)
-    e2e_ms, h2d, d2h = e2e_steps(wl, args.steps, args.warmup)
+    del graphs
+    ms_step = max_over_ranks([ms], dev, dist)[0] / steps
+    kt = kernel_times(S, wl, steps, warmup)
+    e2e_ms, h2d, d2h = e2e_steps(wl, steps, warmup)
     e2e_ms = max_over_ranks([e2e_ms], dev, dist)[0]
-    acct = [wl.accounting(args.warmup + i) for i in range(min(args.steps, N_BATCHES))]
+    acct = [wl.accounting(warmup + i) for i in range(min(steps, N_BATCHES))]
     ab = float(np.mean([a["bytes"] for a in acct]))
     pk = peaks()
     tot = {k: sum(v) for k, v in kt.items()}
@@ -688,6 +684,7 @@ def run_ours(args):
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak if achieved else None,
                 "peak_source": f"{pk['src']} bf16 burst x {NOMINAL_FP8_OVER_BF16} (nominal FP8/BF16 dense ratio)",
+                "frac_of_mma_microbenchmark": achieved / MMA_MICROBENCH_TFLOPS if achieved else None,
                 "traffic": None, "flops_per_launch": launch_flops, "avg_launch_ms": avg_ms,
                 "hbm_gbs": launch_bytes / (avg_ms * 1e-3) / 1e9 if launch_bytes else None}
     else:
@@ -705,164 +702,311 @@ def run_ours(args):
     tps = wl.tokens_per_step()
     if wl.unit == "GB/s":
         value = whole_job_rate(n, ab, ms_step) / 1e9
-        e2e_val = whole_job_rate(n, ab, e2e_ms / args.steps) / 1e9
+        e2e_val = whole_job_rate(n, ab, e2e_ms / steps) / 1e9
     else:
         value = whole_job_rate(n, tps, ms_step)
-        e2e_val = whole_job_rate(n, tps, e2e_ms / args.steps)
-    out = {
-        "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        e2e_val = whole_job_rate(n, tps, e2e_ms / steps)
+    return {
+        "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": n, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
         "dtype": wl.dtype,
         "data": "synthetic (seeded generators; random weights on the format grids)",
-        "config": {**base_config(wl), "hbm_bytes_per_step": ab,
-                   "touched_experts_per_layer": getattr(wl, "_acct", {}).get((args.warmup) % N_BATCHES),
-                   "tflop_per_step": acct[0]["flops"] / 1e12,
-                   "l2": "inputs larger than L2: per-step weights exceed L2, batches rotate over 8",
-                   "parallelism": f"replicas x{n}", "timing": "CUDA graph replays, CUDA events"},
+        "config": base_config(wl.name, n),
+        "accounting": {"hbm_bytes_per_step": ab,
+                       "touched_experts_per_layer": getattr(wl, "_acct", {}).get(warmup % N_BATCHES),
+                       "tflop_per_step": acct[0]["flops"] / 1e12},
+        "timing": "CUDA graph replays, CUDA events",
         "roofline": roof,
         "kernels_ms": {k: statistics.mean(v) for k, v in kt.items()},
-        "gpu_launches": int(sum(len(v) for v in kt.values()) / args.steps * args.steps),
+        "gpu_launches": int(sum(len(v) for v in kt.values())),
         "e2e": {"value": e2e_val, "unit": wl.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,
     }
+
+
+# The other configurations of the target, timed in the default run after the headline
+# (one GPU, one process): the single STQ1_0 matvec, the single-expert W4A8 GEMM, the
+# STQ1_0 decode layer, and the two prefill layers (W4A8 and STQ1_0).
+CONFIG_WORKLOADS = ["stq_matvec", "w4a8_gemm", "decode_stq", "prefill_w4a8", "prefill_stq"]
+
+
+def config_summary(r):
+    roof = r["roofline"]
+    return {"metric": r["metric"], "value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
+            "steps": r["steps"], "warmup": r["warmup"],
+            "roofline": {k: roof.get(k) for k in ("bound", "kernel", "achieved", "peak", "unit", "frac",
+                                                  "frac_of_mma_microbenchmark", "traffic")},
+            "e2e": r["e2e"]["value"], "clocks": r["clocks"], "kernels_ms": r["kernels_ms"]}
+
+
+def run_ours(args):
+    dist = int(os.environ.get("WORLD_SIZE", "1")) > 1
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    if dist:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import bit_quantized_moe_stq1_b200 as S
+
+    wl = make_workload(args.workload, S, dev, args.experts)
+    if isinstance(wl, StreamLayer):
+        return run_stream(args, wl, S, dev, dist, n, rank, local)
+    out = measure(wl, S, dev, dist, n, local, args.steps, args.warmup)
+    del wl
+    torch.cuda.empty_cache()
+    if not dist and args.workload == DEFAULT_WORKLOAD and args.experts == E and not args.no_configs:
+        cfg = {}
+        for name in CONFIG_WORKLOADS:
+            w2 = make_workload(name, S, dev, args.experts)
+            cfg[name] = config_summary(measure(w2, S, dev, dist, n, local, min(args.steps, 20), args.warmup))
+            del w2
+            torch.cuda.empty_cache()
+        out["configs"] = cfg
     if rank == 0 and not dist and not args.no_cpu:
-        out["cpu_baseline"] = cpu_baseline(wl, dev)
+        out["cpu_baseline"] = cpu_baseline(args.workload)
     if rank == 0:
         print(json.dumps(out))
-    del graphs
     if dist:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
 
 
-# ----------------------------------------------------------------------------- oracle timing
+# ----------------------------------------------------------------------------- oracle timing (CPU)
+#
+# The oracle (plain float64 numpy under oracle/) timed on the host's cores, as it stands, on
+# a bounded sample of the same workload.  Its inputs are drawn on the CPU by workloads/ with
+# the workloads' shapes and distributions (the CPU generators give other values than the
+# GPU's); nothing here imports this package or touches the GPU.
+
+MOE_SPECS = {
+    # name: (tokens, formats per layer, router, shared, shared format, residual, prefill regime)
+    "decode_stq": (8, ("stq",), True, True, "bf16", False, False),
+    "decode_stq_sh8": (8, ("stq",), True, True, "mx8", False, False),
+    "decode_mx": (32, ("mx",), True, True, "bf16", True, False),
+    "prefill_w4a8": (4096, ("mx",), False, False, "bf16", False, True),
+    "prefill_stq": (4096, ("stq",), False, False, "bf16", False, True),
+    "stacked_decode": (32, ("stq", "mx") * 4, True, True, "bf16", True, False),
+    "decode_stq_stream": (8, ("stq",), False, True, "bf16", False, False),
+}
+SINGLE_TOKENS = {"stq_matvec": 1, "w4a8_gemm": 128, "stq_pack_ls": 1}
+# bytes per step of the workloads whose metric is GB/s (their algorithmic bytes)
+SINGLE_BYTES = {"stq_matvec": STQ_MAT + H * 2 + I * 4, "stq_pack_ls": I * H * 4 + H * 4 + STQ_MAT}
+ORACLE_POOL_MAX = 16   # packed experts per format drawn once and reused by every sample
 
 
-def _oracle_units(wl, dev):
-    """One bounded unit of oracle work for the workload and its scale to one step:
-    returns (seconds for the unit, units per step, description)."""
-    from oracle import formats as F
-    from oracle import moe as M
+def tokens_of(name):
+    return MOE_SPECS[name][0] if name in MOE_SPECS else SINGLE_TOKENS[name]
 
-    if wl.name == "stq_matvec":
-        Wb = wl.Wt[0].cpu().numpy()
-        xb = wl.x[0].view(torch.int16).cpu().numpy().view(np.uint16)
-        t0 = time.perf_counter()
-        M.stq1_gemv(Wb, I, H, xb)
-        return time.perf_counter() - t0, 1.0, "one full matvec (unpack + float64 matvec)"
-    if wl.name == "stq_pack_ls":
-        rows = 128
-        wf = wl.Wf[0][:rows].cpu().numpy()
-        v = wl.v.cpu().numpy()
-        t0 = time.perf_counter()
-        F.stq1_pack_ls(wf, v)
-        return (time.perf_counter() - t0) * (I / rows), 1.0, f"{rows} of the {I} rows, scaled to the matrix"
-    if wl.name == "w4a8_gemm":
-        c, sc = wl.Wt[0]
-        xb = wl.x[0][:16].view(torch.int16).cpu().numpy().view(np.uint16)
-        c, sc = c.cpu().numpy(), sc.cpu().numpy()
-        t0 = time.perf_counter()
-        ac, asc = F.mxfp8_quantize(F.bf16_decode(xb))
-        M.w4a8_gemm(c, sc, ac, asc, I, H)
-        return time.perf_counter() - t0, wl.T / 16, "16 of the 128 tokens (quantise, unpack, float64 GEMM)"
-    # MoE: one token through one routed expert (+ router and shared expert) per format
-    total, desc = 0.0, []
-    for fmt in sorted({L["fmt"] for L in wl.layers}):
-        l = next(i for i, L in enumerate(wl.layers) if L["fmt"] == fmt)
-        L = wl.layers[l]
-        xb = wl.x[0][:1].view(torch.int16).cpu().numpy().view(np.uint16)
-        X = F.bf16_decode(xb)
-        e = 0
+
+def metric_unit_of(name):
+    cls = {"stq_matvec": StqMatvec, "w4a8_gemm": W4A8Gemm, "stq_pack_ls": StqPackLs}.get(name, Workload)
+    return cls.metric, cls.unit
+
+
+def host_cores():
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def _cpu_bits(shape, std, *tag):
+    return W.bf16_normal(shape, std, "cpu", 0, *tag).view(torch.int16).numpy().view(np.uint16)
+
+
+class OracleSampler:
+    """Times the oracle on one bounded sample per call of step(i) and scales it to one
+    step of the workload; returns (seconds per step, description).
+
+    MoE workloads: per weight format, one layer of the step: router (or the given
+    routing), grouping, the activation quantisation of the MXFP8 paths, the shared expert,
+    the combine and the RMS normalisation, all in full; of the layer's n touched experts, a
+    uniform sample of m (each with all its tokens, its packed matrices unpacked once) runs on
+    m threads, and that time is scaled by n / m; the layer time is scaled to the step's layers
+    of that format.  The m packed experts come from a pool drawn once (same distributions as
+    the workload's experts); numpy's own threading is off, so each thread is one core."""
+
+    def __init__(self, name, cores=None):
+        from oracle import formats as F
+        from oracle import moe as M
+
+        self.F, self.M = F, M
+        self.name = name
+        self.cores = cores or host_cores()
+        self.pool = {}
+        if name in MOE_SPECS:
+            T, fmts, router, shared, sh_fmt, residual, prefill = MOE_SPECS[name]
+            self.m = max(1, min(self.cores, ORACLE_POOL_MAX))
+            for f in sorted(set(fmts)):
+                self.pool[f] = self._threads(lambda j, f=f: self._packed_expert(f, j), range(self.m))
+            self.wr = {f: _cpu_bits((E, H), 0.02, name, "oracle-router", f) for f in set(fmts)} if router else None
+            if shared:
+                sh = [_cpu_bits((I, H), 0.02, name, "oracle-sg"), _cpu_bits((I, H), 0.02, name, "oracle-su"),
+                      _cpu_bits((H, I), 0.02, name, "oracle-sd")]
+                if sh_fmt == "mx8":
+                    # stored MXFP8 codes and scales, quantised once (as the GPU path's weights are)
+                    sh = [F.mxfp8_quantize(F.bf16_decode(b)) for b in sh]
+                self.shared = sh
+        elif name == "stq_matvec":
+            self.packed = F.stq1_pack(W.stq_grid_weights(I, H, "cpu", 0, name, "oracle-w").numpy())
+        elif name == "w4a8_gemm":
+            c, sc = W.mxfp4_random(I, H, "cpu", 0, name, "oracle-w")
+            self.codes, self.scales = c.numpy(), sc.numpy()
+        elif name == "stq_pack_ls":
+            self.rows = 128
+            self.v = torch.exp(W.float_normal((H,), 1.0, "cpu", 0, name, "oracle-v")).numpy()
+
+    def _threads(self, fn, items):
+        import concurrent.futures
+
+        from threadpoolctl import threadpool_limits
+
+        items = list(items)
+        with threadpool_limits(limits=1):
+            with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(self.cores, len(items)))) as ex:
+                return list(ex.map(fn, items))
+
+    def _packed_expert(self, fmt, j):
+        F = self.F
         if fmt == "stq":
-            blks = [W.stq_grid_weights(16 * r, c_, dev, 0, wl.name, l, which, 0)[:r].cpu().numpy()
-                    for which, (r, c_) in (("g", (I, H)), ("u", (I, H)), ("d", (H, I)))]
-            packed = [F.stq1_pack(b_) for b_ in blks]
+            return [F.stq1_pack(W.stq_grid_weights(r, c, "cpu", 0, self.name, "oracle-pool", which, j).numpy())
+                    for which, r, c in (("g", I, H), ("u", I, H), ("d", H, I))]
+        return [tuple(t.numpy() for t in W.mxfp4_random(r, c, "cpu", 0, self.name, "oracle-pool", which, j))
+                for which, r, c in (("g", I, H), ("u", I, H), ("d", H, I))]
+
+    def _expert(self, fmt, j, X, A):
+        """One routed expert on its tokens: unpack its three matrices, gate/up, SwiGLU, h,
+        down (float64)."""
+        F, M = self.F, self.M
+        shapes = ((I, H), (I, H), (H, I))
+        if fmt == "stq":
+            mats = [F.stq1_unpack(p_, r, c) for p_, (r, c) in zip(self.pool[fmt][j], shapes)]
         else:
-            lw = L["w"]
-            packed = [(c_[:r].cpu().numpy(), s_[:r].cpu().numpy()) for c_, s_, r in
-                      ((lw.gate, lw.gate_sc, I), (lw.up, lw.up_sc, I), (lw.down, lw.down_sc, H))]
-        shared = [m.float().double().cpu().numpy() for m in L["sh_bf16"]] if wl.shared else None
-        if shared is not None and wl.shared_fmt == "mx8":
-            # stored MXFP8 weights (quantised before the timed unit, like the GPU's)
-            shared = [F.mxfp8_dequantize(*F.mxfp8_quantize(m_)) for m_ in shared]
-        wr = L["wr"].view(torch.int16).cpu().numpy().view(np.uint16) if wl.router else None
-        t0 = time.perf_counter()
-        if wr is not None:
-            M.router_topk(xb, wr, K_TOP)
-        t_r = time.perf_counter() - t0
-        t0 = time.perf_counter()
-        if fmt == "stq" and wl.name == "prefill_stq":
-            # prefill regime: MXFP8 activations and h
-            mats = [F.stq1_unpack(p_, r, c_) for p_, (r, c_) in zip(packed, ((I, H), (I, H), (H, I)))]
-            xc, xs = F.mxfp8_quantize(X)
-            M.expert_ffn_mx(mats[0], mats[1], mats[2], F.mxfp8_dequantize(xc, xs))
-        elif fmt == "stq":
-            mats = [F.stq1_unpack(p_, r, c_) for p_, (r, c_) in zip(packed, ((I, H), (I, H), (H, I)))]
-            M.expert_ffn_bf16h(mats[0], mats[1], mats[2], X)
-        else:
-            mats = [F.mxfp4_unpack(c_, s_, r, cc) for (c_, s_), (r, cc) in zip(packed, ((I, H), (I, H), (H, I)))]
-            xc, xs = F.mxfp8_quantize(X)
-            M.expert_ffn_mx(mats[0], mats[1], mats[2], F.mxfp8_dequantize(xc, xs))
-        t_e = time.perf_counter() - t0
-        t0 = time.perf_counter()
-        if shared is not None and wl.shared_fmt == "mx8":
-            xc, xs = F.mxfp8_quantize(X)
-            M.expert_ffn_mx(shared[0], shared[1], shared[2], F.mxfp8_dequantize(xc, xs))
-        elif shared is not None:
-            M.expert_ffn_bf16h(shared[0], shared[1], shared[2], X)
-        if wl.residual:
-            M.rms_norm(X, W.STACK_RMS_EPS)
-        t_s = time.perf_counter() - t0
-        nl = sum(1 for L_ in wl.layers if L_["fmt"] == fmt)
-        total += nl * (t_r + K_TOP * t_e + t_s)
-        desc.append(f"{fmt}: 1 token through the router ({t_r:.2f} s), one expert ({t_e:.2f} s) and the shared "
-                    f"expert ({t_s:.2f} s), scaled to {K_TOP} experts x {nl} layers")
-    # per step the workload processes T tokens; the sample above is one token
-    return total, float(wl.T), "; ".join(desc)
+            mats = [F.mxfp4_unpack(c_, s_, r, c) for (c_, s_), (r, c) in zip(self.pool[fmt][j], shapes)]
+        if A is not None:
+            return M.expert_ffn_mx(mats[0], mats[1], mats[2], A)["y"]
+        return M.expert_ffn_bf16h(mats[0], mats[1], mats[2], X)["y"]
+
+    def step(self, i):
+        F, M = self.F, self.M
+        b = i % N_BATCHES
+        if self.name == "stq_matvec":
+            x = _cpu_bits((1, H), 1.0, self.name, "oracle-x", b)
+            t0 = time.perf_counter()
+            M.stq1_gemv(self.packed, I, H, x)
+            return time.perf_counter() - t0, "one full 2048 x 6144 matvec (unpack, float64 product), 1 core"
+        if self.name == "w4a8_gemm":
+            x = _cpu_bits((128, H), 1.0, self.name, "oracle-x", b)
+            with __import__("threadpoolctl").threadpool_limits(limits=self.cores):
+                t0 = time.perf_counter()
+                ac, asc = F.mxfp8_quantize(F.bf16_decode(x))
+                M.w4a8_gemm(self.codes, self.scales, ac, asc, I, H)
+                dt = time.perf_counter() - t0
+            return dt, f"the full GEMM: 128 tokens quantised, weights unpacked, float64 product ({self.cores} cores)"
+        if self.name == "stq_pack_ls":
+            wf = W.float_normal((self.rows, H), 0.02, "cpu", 0, self.name, "oracle-w", b).numpy()
+            t0 = time.perf_counter()
+            F.stq1_pack_ls(wf, self.v)
+            return (time.perf_counter() - t0) * (I / self.rows), f"{self.rows} of the {I} rows, scaled to the matrix"
+        T, fmts, router, shared, sh_fmt, residual, prefill = MOE_SPECS[self.name]
+        P = T * K_TOP
+        total, desc = 0.0, []
+        rng = np.random.default_rng(i)
+        for f in sorted(set(fmts)):
+            nl = sum(1 for g in fmts if g == f)
+            xb = _cpu_bits((T, H), 1.0, self.name, "oracle-x", f, b)
+            if not router:
+                ids_t, tw_t = W.zipf_routing(T, E, K_TOP, "cpu", 0, self.name, "oracle-zipf", b)
+                ids, tw = ids_t.numpy(), tw_t.double().numpy()
+            t0 = time.perf_counter()
+            if router:
+                ids, tw, _ = M.router_topk(xb, self.wr[f], K_TOP)
+            counts, offsets, perm, inv = M.permute(ids, E)
+            X = F.bf16_decode(xb)
+            A = None
+            if f == "mx" or prefill:
+                qc, qs = F.mxfp8_quantize(X)
+                A = F.mxfp8_dequantize(qc, qs)
+            y_sh = 0.0
+            if shared and sh_fmt == "mx8":
+                sh = [F.mxfp8_dequantize(c_, s_) for c_, s_ in self.shared]
+                qc, qs = F.mxfp8_quantize(X)
+                y_sh = M.expert_ffn_mx(sh[0], sh[1], sh[2], F.mxfp8_dequantize(qc, qs))["y"]
+            elif shared:
+                sh = [F.bf16_decode(m_) for m_ in self.shared]
+                y_sh = M.expert_ffn_bf16h(sh[0], sh[1], sh[2], X)["y"]
+            t_fixed = time.perf_counter() - t0
+            touched = np.flatnonzero(counts)
+            pick = np.sort(rng.choice(touched, size=min(self.m, touched.size), replace=False))
+            jobs = [(j, perm[offsets[e]:offsets[e + 1]] // K_TOP) for j, e in enumerate(pick)]
+            t0 = time.perf_counter()
+            ys = self._threads(lambda jt: self._expert(f, jt[0], X[jt[1]], None if A is None else A[jt[1]]), jobs)
+            t_exp = time.perf_counter() - t0
+            # combine (all pairs; the sampled experts' outputs stand in for the rest) and norm
+            Yp = np.zeros((P, H))     # sorted pair order
+            for (j, toks), ye in zip(jobs, ys):
+                Yp[offsets[pick[j]]:offsets[pick[j]] + len(toks)] = ye
+            t0 = time.perf_counter()
+            y, _ = M.combine(Yp[inv], np.abs(Yp[inv]), tw, y_sh if shared else None, None, X if residual else None)
+            if residual:
+                M.rms_norm(y, W.STACK_RMS_EPS)
+            t_fixed += time.perf_counter() - t0
+            per_layer = t_fixed + t_exp * touched.size / pick.size
+            total += nl * per_layer
+            desc.append(f"{f}: {nl} layer(s) x ({t_fixed:.2f} s router/grouping/quant/shared/combine/norm in full + "
+                        f"{t_exp:.2f} s for {pick.size} of {touched.size} touched experts on {pick.size} threads, "
+                        f"x {touched.size / pick.size:.1f})")
+        return total, "; ".join(desc)
+
+    def threads_used(self):
+        if self.name in MOE_SPECS:
+            return self.m
+        return self.cores if self.name == "w4a8_gemm" else 1
 
 
-def cpu_baseline(wl, dev, budget_s=12.0):
-    """The oracle, single-threaded, on a bounded sample of the workload, scaled to the
-    metric's unit.  Small units repeat until budget_s has passed."""
-    from threadpoolctl import threadpool_limits
-
-    with threadpool_limits(limits=1):
-        times, t0 = [], time.perf_counter()
-        while True:
-            dt, per_step, desc = _oracle_units(wl, dev)
-            times.append(dt)
-            if time.perf_counter() - t0 > budget_s or len(times) >= 20 or isinstance(wl, MoeLayers):
-                break
+def cpu_baseline(name, budget_s=12.0, sampler=None):
+    """The oracle on a bounded sample of the workload, scaled to the metric's unit."""
+    smp = sampler or OracleSampler(name)
+    times, t0, desc = [], time.perf_counter(), ""
+    while True:
+        dt, desc = smp.step(len(times))
+        times.append(dt)
+        if time.perf_counter() - t0 > budget_s or len(times) >= 20 or name in MOE_SPECS:
+            break
     dt = statistics.mean(times)
-    if wl.unit == "GB/s":
-        value = wl.bytes / dt / 1e9
-    else:
-        value = wl.tokens_per_step() / (dt * per_step)
-    return {"value": value, "unit": wl.unit, "cores": 1, "kind": "oracle",
-            "sample": f"{desc}; {len(times)} repetitions, mean {dt:.2f} s"}
+    _, unit = metric_unit_of(name)
+    value = SINGLE_BYTES[name] / dt / 1e9 if unit == "GB/s" else tokens_of(name) / dt
+    return {"value": value, "unit": unit, "cores": smp.threads_used(), "kind": "oracle",
+            "sample": f"{desc}; {len(times)} sample(s), mean {dt:.2f} s per step"}
 
 
 def run_reference(args):
+    """The oracle arm: rank 0 alone times the CPU oracle, one bounded sample per step; the
+    other ranks exit without work.  Never imports this package and never touches a GPU."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    dev = torch.device("cuda", 0)
-    import bit_quantized_moe_stq1_b200 as S
-
-    wl = make_workload(args.workload, S, dev, args.experts)
-    vals = []
+    name = args.workload
+    smp = OracleSampler(name)
+    metric, unit = metric_unit_of(name)
+    secs, desc = [], ""
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(wl, dev, budget_s=0.0)   # one bounded unit per step
+        dt, desc = smp.step(i)
         if i >= args.warmup:
-            vals.append(cb["value"])
-    value = statistics.mean(vals)
-    out = {"impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": args.gpus,
-           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": base_config(wl),
-           "cpu_baseline": {"value": value, "unit": wl.unit, "cores": cb["cores"], "kind": "oracle",
-                            "sample": cb["sample"]},
-           "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            secs.append(dt)
+    ms = 1e3 * statistics.mean(secs)
+    value = SINGLE_BYTES[name] / (ms * 1e-3) / 1e9 if unit == "GB/s" else tokens_of(name) / (ms * 1e-3)
+    out = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": base_config(name, args.gpus),
+           "cpu_baseline": {"value": value, "unit": unit, "cores": smp.threads_used(), "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
 
 
@@ -874,6 +1018,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_NAMES)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations timed after the default workload")
     ap.add_argument("--experts", type=int, default=256,
                     help="routed experts per layer (256 = the workloads; fewer only for small profiler captures)")
     args = ap.parse_args()

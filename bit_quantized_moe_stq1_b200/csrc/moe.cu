@@ -689,28 +689,46 @@ stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const f
   return stq_launch_status();
 }
 
-// A library-owned stream (and fork/join events) per device, created on first use: the
-// MXFP8 shared expert depends on x alone, so it runs beside the routing, permutation and
-// routed experts instead of after them.
+// A library-owned stream per device, created on first use: the MXFP8 shared expert
+// depends on x alone, so it runs beside the routing, permutation and routed experts
+// instead of after them.  Calls from several host threads share the stream; `mu` is held
+// from the fork to the join record, so one call's launches on it never interleave with
+// another's.
 struct SideStream {
   cudaStream_t stream = nullptr;
+  std::mutex mu;
+};
+
+// Fork and join events of the calling host thread on one device: a call waits on its own
+// records only, whatever other threads record meanwhile.  Created on first use, kept for
+// the thread's lifetime.
+struct ForkJoin {
   cudaEvent_t fork = nullptr, join = nullptr;
 };
 
-static stq_status side_stream(SideStream** out) {
+static stq_status side_stream(SideStream** out, ForkJoin** fj) {
   static SideStream side[kStqMaxDevices];
-  static std::mutex mu;
+  static std::mutex create_mu;
+  thread_local ForkJoin events[kStqMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStqMaxDevices) return STQ_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  SideStream& ss = side[dev];
-  if (ss.stream == nullptr) {
-    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+  {
+    std::lock_guard<std::mutex> lock(create_mu);
+    if (side[dev].stream == nullptr &&
+        cudaStreamCreateWithFlags(&side[dev].stream, cudaStreamNonBlocking) != cudaSuccess)
       return STQ_ERR_CUDA;
   }
-  *out = &ss;
+  ForkJoin& ev = events[dev];
+  if (ev.fork == nullptr) {
+    if (cudaEventCreateWithFlags(&ev.fork, cudaEventDisableTiming) != cudaSuccess) return STQ_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ev.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventDestroy(ev.fork);
+      ev.fork = nullptr;
+      return STQ_ERR_CUDA;
+    }
+  }
+  *out = &side[dev];
+  *fj = &ev;
   return STQ_OK;
 }
 
@@ -777,12 +795,14 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   // The MXFP8 shared expert on the side stream (its workspace rows P.. and the sticky error
   // word are all it writes; nothing on the routed path reads them), joined before the combine.
   SideStream* side = nullptr;
+  ForkJoin* fj = nullptr;
   if (shared_mx8) {
-    if ((st = side_stream(&side)) != STQ_OK) return st;
-    if (cudaEventRecord(side->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+    if ((st = side_stream(&side, &fj)) != STQ_OK) return st;
+    std::lock_guard<std::mutex> lock(side->mu);
+    if (cudaEventRecord(fj->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, fj->fork, 0) != cudaSuccess)
       return STQ_ERR_CUDA;
     if ((st = moe_shared_expert_mx8(a, side->stream)) != STQ_OK) return st;
-    if (cudaEventRecord(side->join, side->stream) != cudaSuccess) return STQ_ERR_CUDA;
+    if (cudaEventRecord(fj->join, side->stream) != cudaSuccess) return STQ_ERR_CUDA;
   }
   if ((st = moe_launch_permute(topk_ids, P, d->E, ws, s)) != STQ_OK) return st;
 
@@ -812,7 +832,7 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     st = moe_mx_experts(a, slots, shared_bf16, s);
     if (st != STQ_OK) return st;
   }
-  if (shared_mx8 && cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) return STQ_ERR_CUDA;
+  if (shared_mx8 && cudaStreamWaitEvent(s, fj->join, 0) != cudaSuccess) return STQ_ERR_CUDA;
   return moe_launch_combine(*d, P, ws, topk_w, has_shared, x, y, s);
 }
 
@@ -865,32 +885,14 @@ extern "C" stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k,
 // library a scratch buffer: the logits partial sums live in a fixed array compiled
 // into this module, one copy on every GPU that loads the library, kept until the
 // process exits.  Host code may not pass the array's name to a kernel (on the host
-// it is only a stand-in for the symbol), so its device address is looked up once
-// per device with cudaGetSymbolAddress and cached.
+// it is only a stand-in for the symbol), so every call looks up its device address
+// with cudaGetSymbolAddress, with the call's device current.  Looking it up per call
+// (not caching it) keeps the address right after a cudaDeviceReset, which reloads the
+// module at another address in a new context.
 
 constexpr size_t kRouterStaticFloats = size_t(1) << 19;  // 524,288 floats = 2 MiB per GPU
 
 static __device__ __align__(256) float g_router_scratch[kRouterStaticFloats];
-
-namespace {
-
-// Device address of g_router_scratch on the current device (looked up on first use).
-stq_status router_static_scratch(float** out) {
-  static float* addr[kStqMaxDevices] = {};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStqMaxDevices) return STQ_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_router_scratch) != cudaSuccess || p == nullptr) return STQ_ERR_CUDA;
-    addr[dev] = static_cast<float*>(p);
-  }
-  *out = addr[dev];
-  return STQ_OK;
-}
-
-}  // namespace
 
 extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router, int32_t T, int32_t H,
                                              int32_t E, int32_t k, int32_t* topk_ids, float* topk_w,
@@ -901,16 +903,22 @@ extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* 
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
   const int KS = stq_router_ksplit(H);
   STQ_HOST_CHECK(size_t(KS) * size_t(T) * size_t(E) <= kRouterStaticFloats, STQ_ERR_WORKSPACE);
-  float* scratch = nullptr;
-  const stq_status st0 = router_static_scratch(&scratch);
-  if (st0 != STQ_OK) return st0;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_router_scratch) != cudaSuccess || addr == nullptr) return STQ_ERR_CUDA;
+  float* scratch = static_cast<float*>(addr);
   if (T == 0) return STQ_OK;
   cudaStream_t s = stq_cuda_stream(stream);
   // Every entry the top-k step reads is written first by the logits step, so the
   // array needs no clearing between calls.
-  router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 256, 0, s>>>(x, w_router, T, H, E, KS, scratch);
+  {
+    StqTimed tm(STQ_K_ROUTER_LOGITS, s);
+    router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 256, 0, s>>>(x, w_router, T, H, E, KS, scratch);
+  }
   stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
-  router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(scratch, T, E, KS, k, topk_ids, topk_w);
+  {
+    StqTimed tm(STQ_K_ROUTER_TOPK, s);
+    router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(scratch, T, E, KS, k, topk_ids, topk_w);
+  }
   return stq_launch_status();
 }

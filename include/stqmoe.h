@@ -199,9 +199,10 @@ stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
  * The logits' partial sums go to a fixed 2 MiB array inside the library instead,
  * one per GPU that loads the library, held until the process exits.  Limit:
  * stq_router_ksplit(H) * T * E <= 524288 (e.g. T <= 256 for H = 6144, E = 256);
- * larger requests return STQ_ERR_WORKSPACE before any launch.  The array's device
- * address is looked up on the first call on each device (cudaGetSymbolAddress,
- * with that device current): make that first call before any stream capture.
+ * larger requests return STQ_ERR_WORKSPACE before any launch.  Every call looks up
+ * the array's device address on the current device (cudaGetSymbolAddress); the first
+ * call on a device may also load the library's module there, so make that first call
+ * before any stream capture.
  * Every call shares the array and leaves its last contents there (each call
  * writes every entry it reads, so nothing needs clearing); calls whose kernels
  * overlap on the GPU (other streams, other host threads) race on it.  Allocates
@@ -223,8 +224,11 @@ stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router,
  *                     reused; not device memory), forked from `stream` after the
  *                     call's argument checks and joined back before the combine; the
  *                     call stays ordered on `stream` and can be captured into a graph.
- *                     Calls on one device share that stream: calls from several host
- *                     threads serialize their shared-expert work on it, and a call while
+ *                     Calls on one device share that stream: a lock keeps one call's
+ *                     launches on it from interleaving with another's, each host thread
+ *                     forks and joins through its own pair of events (so a call waits
+ *                     for its own shared expert only), and calls from several host
+ *                     threads run their shared experts one after another.  A call while
  *                     another thread is capturing such a call into a graph is not
  *                     supported. */
 enum { STQ_SHARED_BF16 = 0, STQ_SHARED_MXFP8 = 1 };
@@ -375,8 +379,8 @@ enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_GATE_UP_STQ_TC, STQ_K_DOWN_STQ_TC, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
- * moe_router_topk, moe_expert_forward, stq1_gemv, w4a8_gemm, stq_rmsnorm_bf16 and
- * stq1_pack_ls is bracketed by event records of events[2n] / events[2n+1] on the
+ * moe_router_topk, moe_router_topk_static, moe_expert_forward, stq1_gemv, w4a8_gemm,
+ * stq_rmsnorm_bf16 and stq1_pack_ls is bracketed by event records of events[2n] / events[2n+1] on the
  * stream it runs on (inside stream capture as external event-record nodes of the
  * graph), kinds[n] is set to its STQ_K_* kind and n = count++ (until capacity pairs
  * are used).  events: cudaEvent_t[2*capacity] created with timing.  Process-wide, not

@@ -105,7 +105,7 @@ def test_streamed_layer_host_path(monkeypatch, capsys):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert seen["layers"] == 3 + 3 * 6
     assert seen["loads"] > 40                       # the 40-slot bank evicted
-    assert line["config"]["slots"] == 40 and line["config"]["workload"] == "decode_stq_stream"
+    assert line["stream"]["slots"] == 40 and line["config"]["workload"] == "decode_stq_stream"
     assert line["roofline"]["bound"] == "h2d" and line["gpu_launches"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] >= 8 * 6144 * 2
-    assert 0 < line["config"]["experts_loaded_per_step"] <= line["config"]["distinct_experts_per_step"] <= 40
+    assert 0 < line["stream"]["experts_loaded_per_step"] <= line["stream"]["distinct_experts_per_step"] <= 40
