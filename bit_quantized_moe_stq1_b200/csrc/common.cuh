@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 
 #include "../../include/stqmoe.h"
 
@@ -47,6 +48,33 @@ struct StqSmemOptIn {
     return STQ_OK;
   }
 };
+
+// Programmatic dependent launch.  The hot-path kernels are launched with programmatic
+// stream serialisation (stq_launch): a kernel may then start while its predecessor on the
+// stream is still running.  Each one first lets its own successor launch, then waits until
+// the predecessor has completed and its writes are visible, before it touches any global
+// memory.  Launched without the attribute, both instructions do nothing.
+__device__ __forceinline__ void stq_pdl_begin() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Launch with programmatic stream serialisation (see stq_pdl_begin).
+template <typename... KArgs, typename... Args>
+static inline stq_status stq_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    Args&&... args) {
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? STQ_OK : STQ_ERR_CUDA;
+}
 
 // First error wins: only replace a 0 word.
 __device__ __forceinline__ void stq_set_error(int32_t* err, int32_t code) {

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kGemmThreads, Cfg<NT, PAIR, A8>::kCtasPerSm)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+  stq_pdl_begin();   // barriers and TMEM are set up; from here on global memory is read
 
   if (warp == 0 || warp == kProducer2) {
     // ---------------------------------------------------------------- producers
@@ -313,6 +314,7 @@ __global__ void wait_selftest_kernel(int32_t* err) {
 // N tiles of every touched expert: (expert, first token of the tile); one CTA.
 __global__ void __launch_bounds__(1024) mx_plan_kernel(const int32_t* __restrict__ counts, int E, int nt,
                                                        int2* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
+  stq_pdl_begin();
   __shared__ int wsum[32];
   __shared__ int total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -357,8 +359,7 @@ stq_status launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtens
   if (st != STQ_OK) return st;
   if (p.tiles.max_items <= 0) return STQ_OK;
   const unsigned grid = unsigned(stq_persistent_grid(p.tiles.max_items, C::kCtasPerSm));
-  w4a8_gemm_kernel<NT, PAIR, A8><<<grid, kGemmThreads, C::kSmem, s>>>(a, a2, b, p);
-  return stq_launch_status();
+  return stq_launch(w4a8_gemm_kernel<NT, PAIR, A8>, dim3(grid), dim3(kGemmThreads), C::kSmem, s, a, a2, b, p);
 }
 
 template <bool PAIR, bool A8 = false>
@@ -385,20 +386,21 @@ int narrower_nt(int nt) { return nt > 128 ? 128 : nt / 2; }
 
 stq_status stq_tile_plan_launch(const int32_t* counts, int E, int nt, int2* tiles, int32_t* n_tiles, cudaStream_t s) {
   StqTimed tm(STQ_K_PLAN, s);
-  mx_plan_kernel<<<1, 1024, 0, s>>>(counts, E, nt, tiles, n_tiles);
-  return stq_launch_status();
+  return stq_launch(mx_plan_kernel, dim3(1), dim3(1024), 0, s, counts, E, nt, tiles, n_tiles);
 }
 
-stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStream_t s) {
+stq_status moe_mx_experts(const MoeArgs& a, int slots, cudaStream_t s) {
   (void)slots;
   const int P = a.P;
   // 1. activations -> MXFP8 in sorted (expert-grouped) order
-  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.T, a.err, a.xq, a.xs, s);
+  stq_status st = stq_mxfp8_quantize_scatter_launch(a.x, a.T, a.H, a.inv, a.k, P, a.err, a.xq, a.xs, s);
   if (st != STQ_OK) return st;
   // 2. N tiles of the touched experts: the down projection takes the 240-wide tile from
   // 128 tokens per expert on average, the gate/up pair (whose SwiGLU/MXFP8 epilogue and
   // item balance measured slower there) at most 128
   const int slots_ = a.E < P ? a.E : P;
+  // prefill (128 or more routed tokens per expert on average): the CTA-pair GEMM
+  if (int64_t(P) / slots_ >= 128) return moe_mx_experts_pair(a, slots_, s);
   const int nt_dn = pick_nt(int64_t(P) / slots_);
   const int nt = nt_dn > 128 ? 128 : nt_dn;
   if ((st = stq_tile_plan_launch(a.counts, a.E, nt, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
@@ -429,7 +431,6 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStre
     st = launch_nt<true>(nt, mg, mu, mx, gp, s);
   }
   if (st != STQ_OK) return st;
-  if (has_shared && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
   // 4. down (the N-tile plan is redone for its tile width once the gate/up launch is done with it)
   if (nt_dn != nt && (st = stq_tile_plan_launch(a.counts, a.E, nt_dn, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
   GemmProblem dp = gp;

@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+  stq_pdl_begin();   // barriers and TMEM are set up; from here on global memory is read
 
   if (warp == 0) {
     // ---------------------------------------------------------------- activation loads
@@ -476,8 +477,8 @@ stq_status launch_stq_gemm(const CUtensorMap& b, const StqGemm& p, cudaStream_t 
   const stq_status st = optin.ensure(stq_gemm_kernel<PAIR>, kSmem);
   if (st != STQ_OK) return st;
   if (p.tiles.max_items <= 0) return STQ_OK;
-  stq_gemm_kernel<PAIR><<<unsigned(stq_persistent_grid(p.tiles.max_items, 1)), kThreads, kSmem, s>>>(b, p);
-  return stq_launch_status();
+  return stq_launch(stq_gemm_kernel<PAIR>, dim3(unsigned(stq_persistent_grid(p.tiles.max_items, 1))), dim3(kThreads),
+                    kSmem, s, b, p);
 }
 
 }  // namespace
@@ -485,7 +486,7 @@ stq_status launch_stq_gemm(const CUtensorMap& b, const StqGemm& p, cudaStream_t 
 stq_status moe_stq_prefill_experts(const MoeArgs& a, int slots, cudaStream_t s) {
   const int P = a.P;
   // 1. activations -> MXFP8 g32 in sorted (expert-grouped) order
-  stq_status st = stq_mxfp8_quantize_gather_launch(a.x, P, a.H, a.perm, a.k, a.T, a.err, a.xq, a.xs, s);
+  stq_status st = stq_mxfp8_quantize_scatter_launch(a.x, a.T, a.H, a.inv, a.k, P, a.err, a.xq, a.xs, s);
   if (st != STQ_OK) return st;
   // 2. N tiles of 112 tokens of the touched experts
   if ((st = stq_tile_plan_launch(a.counts, a.E, kNT, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;

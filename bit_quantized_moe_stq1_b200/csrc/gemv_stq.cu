@@ -12,6 +12,7 @@ __global__ void __launch_bounds__(128) stq1_gemv_kernel(const uint8_t* __restric
                                                          const uint16_t* __restrict__ x, int64_t n,
                                                          float* __restrict__ y) {
   __shared__ float red[4][4][32];
+  stq_pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int nb = int(K / 256);
   const int64_t tile = blockIdx.x;
@@ -53,7 +54,7 @@ extern "C" stq_status stq1_gemv(const uint8_t* W, int64_t rows, int64_t K, const
                          : STQ_ERR_CUDA;
   {
     StqTimed tm(STQ_K_GEMV, stq_cuda_stream(stream));
-    stq1_gemv_kernel<<<unsigned(rows / 16), 128, 0, stq_cuda_stream(stream)>>>(W, rows, K, x, n, y);
+    return stq_launch(stq1_gemv_kernel, dim3(unsigned(rows / 16)), dim3(128), 0, stq_cuda_stream(stream), W, rows, K, x,
+                      n, y);
   }
-  return stq_launch_status();
 }

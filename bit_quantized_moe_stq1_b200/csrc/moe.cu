@@ -74,8 +74,11 @@ __global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __rest
   __shared__ int wsum[32];
   __shared__ int total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  stq_pdl_begin();
   for (int e = tid; e < E; e += 1024) cnt[e] = 0;
-  if (ws.sched != nullptr && tid < 4) ws.sched[tid] = 0;
+  // counters 0-2 (the STQ1_0 decode kernels); counter 3 belongs to the shared expert, which
+  // may run on another stream and is zeroed there (shared_gateup_wide_kernel)
+  if (ws.sched != nullptr && tid < 3) ws.sched[tid] = 0;
   __syncthreads();
   bool bad = false;
   for (int p = tid; p < P; p += 1024) {
@@ -133,6 +136,96 @@ __global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __rest
   }
 }
 
+// The same grouping over many CTAs (large P): chunks of 1024 pairs.
+//   hist   CTA c: histogram of chunk c's expert ids -> chist[c][e];
+//   scan   one CTA: counts, offsets, touched list, and chist[c][e] turned into the sorted
+//          position of chunk c's first pair of expert e (offsets[e] + the counts of e in
+//          chunks before c);
+//   place  CTA c: stable ranks inside the chunk (as above) from those positions.
+// The result equals the one-CTA kernel's exactly.
+__global__ void __launch_bounds__(1024) moe_permute_hist_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                                int32_t* __restrict__ chist, int32_t* err) {
+  extern __shared__ int32_t sm[];  // [E]
+  const int tid = threadIdx.x, c = blockIdx.x;
+  stq_pdl_begin();
+  for (int e = tid; e < E; e += 1024) sm[e] = 0;
+  __syncthreads();
+  const int p = c * 1024 + tid;
+  bool bad = false;
+  if (p < P) {
+    const int e = ids[p];
+    if (e >= 0 && e < E) atomicAdd(&sm[e], 1); else bad = true;
+  }
+  if (__syncthreads_or(bad) && tid == 0) stq_set_error(err, STQ_ERR_DEVICE);
+  for (int e = tid; e < E; e += 1024) chist[size_t(c) * E + e] = sm[e];
+}
+
+__global__ void __launch_bounds__(1024) moe_permute_scan_kernel(int E, int C, int32_t* __restrict__ chist, MoeWs ws) {
+  __shared__ int wsum[32];
+  __shared__ int total;
+  const int tid = threadIdx.x;
+  stq_pdl_begin();
+  if (ws.sched != nullptr && tid < 3) ws.sched[tid] = 0;   // as the one-CTA kernel
+  int v = 0;
+  if (tid < E) {
+    for (int c = 0; c < C; ++c) {
+      const int h = chist[size_t(c) * E + tid];
+      chist[size_t(c) * E + tid] = v;
+      v += h;
+    }
+  }
+  const int ex = block_excl_scan_1024(v, wsum, &total);
+  if (tid < E) {
+    ws.offsets[tid] = ex;
+    ws.counts[tid] = v;
+    for (int c = 0; c < C; ++c) chist[size_t(c) * E + tid] += ex;
+  }
+  if (tid == 0) ws.offsets[E] = total;
+  const int flag = (tid < E && v > 0) ? 1 : 0;
+  const int fx = block_excl_scan_1024(flag, wsum, &total);
+  if (flag) ws.tlist[fx] = tid;
+  if (tid == 0) *ws.ntouched = total;
+}
+
+__global__ void __launch_bounds__(1024) moe_permute_place_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                                 const int32_t* __restrict__ chist, MoeWs ws) {
+  extern __shared__ int32_t sm[];
+  int32_t* cursor = sm;          // [E]
+  int32_t* whist = sm + E;       // [32][E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, c = blockIdx.x;
+  stq_pdl_begin();
+  for (int e = tid; e < E; e += 1024) cursor[e] = chist[size_t(c) * E + e];
+  for (int i = tid; i < 32 * E; i += 1024) whist[i] = 0;
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  const int p = c * 1024 + tid;
+  const bool valid = p < P;
+  const int e = valid ? ids[p] : -1;
+  const bool ok = valid && e >= 0 && e < E;
+  const int key = ok ? e : -1 - lane;
+  const unsigned peers = __match_any_sync(kFull, key);
+  const int rank = __popc(peers & lt);
+  if (ok && rank == 0) whist[warp * E + e] = __popc(peers);
+  __syncthreads();
+  for (int e2 = tid; e2 < E; e2 += 1024) {
+    int run = cursor[e2];
+#pragma unroll 4
+    for (int w = 0; w < 32; ++w) {
+      const int cw = whist[w * E + e2];
+      whist[w * E + e2] = run;
+      run += cw;
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    const int pos = whist[warp * E + e] + rank;
+    ws.perm[pos] = p;
+    ws.inv[p] = pos;
+  } else if (valid) {
+    ws.inv[p] = -1;
+  }
+}
+
 // ----------------------------------------------------------------------------- router
 
 // Router logits, split over K: part[ks][t][e] = sum over the ks-th slice of H of
@@ -142,6 +235,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
                                                             const uint16_t* __restrict__ wr, int T, int H, int E,
                                                             int KS, float* __restrict__ part) {
   __shared__ float red[8][4][4][32];
+  stq_pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int e0 = (blockIdx.x / KS) * 16, ks = blockIdx.x % KS;
   const int slice = H / KS, kq = slice / 8;
@@ -202,6 +296,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 // ties to the lower id, weights renormalised over the chosen k.
 __global__ void router_topk_kernel(float* __restrict__ logits, int T, int E, int KS, int k,
                                    int32_t* __restrict__ ids, float* __restrict__ w) {
+  stq_pdl_begin();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -360,6 +455,9 @@ template <int NCH>
 __global__ void __launch_bounds__(kWideWarps * 32) shared_gateup_wide_kernel(MoeArgs a) {
   extern __shared__ float red[];  // [warp][2][NCH][4][32]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+  stq_pdl_begin();
+  // the work counter of the shared down launch that follows on this stream
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.sched[3] = 0;
   const int f0 = blockIdx.x * 16;
   const int nch = a.H / 32;
   const int k0 = 32 * (warp * nch / kWideWarps), k1 = 32 * ((warp + 1) * nch / kWideWarps);
@@ -410,6 +508,7 @@ __device__ __forceinline__ int next_item(int32_t* counter, int* slot) {
 __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
   __shared__ float red[4][2][4][4][32];
   __shared__ int s_item;
+  stq_pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int per_expert = a.I / 128;
   const int n_items = a.n_shared_cta + (a.routed ? *a.ntouched * per_expert : 0);
@@ -456,9 +555,10 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
 
 // Routed STQ1_0 down, persistent.  Items: the shared expert's 16-row tiles, then per
 // touched expert 256-row tiles of H (warp = 4 tiles).
-__global__ void __launch_bounds__(128, 3) moe_down_stq_kernel(MoeArgs a) {
+__global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
   __shared__ float red[4][2][4][4][32];
   __shared__ int s_item;
+  stq_pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int per_expert = a.H / 256;
   const int n_items = a.n_shared_cta + (a.routed ? *a.ntouched * per_expert : 0);
@@ -506,6 +606,7 @@ __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __re
                                    const int32_t* __restrict__ inv, const float* __restrict__ topk_w, int has_shared,
                                    const uint16_t* __restrict__ resid, void* __restrict__ y, int out_fp32,
                                    int32_t* err) {
+  stq_pdl_begin();
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int h4 = H / 4;
   if (idx >= int64_t(T) * h4) return;
@@ -581,6 +682,7 @@ MoeWsLayout moe_ws_layout(const moe_desc& d) {
   L.ntiles = take((P / 16 + E + 1) * 8);
   L.n_ntiles = take(4);
   L.sched = take(16);
+  L.chist = take(size_t((P + 1023) / 1024) * E * 4);
   L.total = o;
   return L;
 }
@@ -604,6 +706,7 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
   w.ntiles = reinterpret_cast<int2*>(b + L.ntiles);
   w.n_ntiles = reinterpret_cast<int32_t*>(b + L.n_ntiles);
   w.sched = reinterpret_cast<int32_t*>(b + L.sched);
+  w.chist = reinterpret_cast<int32_t*>(b + L.chist);
   return w;
 }
 
@@ -628,8 +731,7 @@ stq_status launch_shared_gateup_wide(const MoeArgs& a, cudaStream_t s) {
   const stq_status st = optin.ensure(shared_gateup_wide_kernel<NCH>, smem);
   if (st != STQ_OK) return st;
   StqTimed tm(STQ_K_SHARED_GATE_UP, s);
-  shared_gateup_wide_kernel<NCH><<<unsigned(a.I / 16), kWideWarps * 32, smem, s>>>(a);
-  return stq_launch_status();
+  return stq_launch(shared_gateup_wide_kernel<NCH>, dim3(unsigned(a.I / 16)), dim3(kWideWarps * 32), smem, s, a);
 }
 
 stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
@@ -641,11 +743,8 @@ stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
   a.routed = 0;
   a.n_shared_cta = a.H / 16;
   a.sched = a0.sched + 3;
-  {
-    StqTimed tm(STQ_K_SHARED_DOWN, s);
-    moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta, 3)), 128, 0, s>>>(a);
-  }
-  return stq_launch_status();
+  StqTimed tm(STQ_K_SHARED_DOWN, s);
+  return stq_launch(moe_down_stq_kernel, dim3(unsigned(stq_persistent_grid(a.n_shared_cta, 4))), dim3(128), 0, s, a);
 }
 
 extern "C" size_t moe_workspace_offset(const moe_desc* d, int32_t region) {
@@ -668,14 +767,38 @@ extern "C" size_t moe_workspace_offset(const moe_desc* d, int32_t region) {
   }
 }
 
+// From this many pairs (and with the workspace's chunk histograms) the grouping runs over
+// many CTAs.
+constexpr int kPermuteMultiCta = 8192;
+
 stq_status moe_launch_permute(const int32_t* ids, int P, int E, const MoeWs& ws, cudaStream_t s) {
+  if (P >= kPermuteMultiCta && ws.chist != nullptr) {
+    const int C = (P + 1023) / 1024;
+    const size_t smem = size_t(33) * E * sizeof(int32_t);
+    static StqSmemOptIn optin;
+    stq_status st = optin.ensure(moe_permute_place_kernel, int(smem));
+    if (st != STQ_OK) return st;
+    {
+      StqTimed tm(STQ_K_PERMUTE, s);
+      st = stq_launch(moe_permute_hist_kernel, dim3(unsigned(C)), dim3(1024), size_t(E) * sizeof(int32_t), s, ids, P, E,
+                      ws.chist, ws.err);
+    }
+    if (st != STQ_OK) return st;
+    {
+      StqTimed tm(STQ_K_PERMUTE, s);
+      st = stq_launch(moe_permute_scan_kernel, dim3(1), dim3(1024), 0, s, E, C, ws.chist, ws);
+    }
+    if (st != STQ_OK) return st;
+    StqTimed tm(STQ_K_PERMUTE, s);
+    return stq_launch(moe_permute_place_kernel, dim3(unsigned(C)), dim3(1024), smem, s, ids, P, E,
+                      static_cast<const int32_t*>(ws.chist), ws);
+  }
   const size_t smem = size_t(34) * E * sizeof(int32_t);
   static StqSmemOptIn optin;
   const stq_status st = optin.ensure(moe_permute_kernel, int(smem));
   if (st != STQ_OK) return st;
   StqTimed tm(STQ_K_PERMUTE, s);
-  moe_permute_kernel<<<1, 1024, smem, s>>>(ids, P, E, ws);
-  return stq_launch_status();
+  return stq_launch(moe_permute_kernel, dim3(1), dim3(1024), smem, s, ids, P, E, ws);
 }
 
 stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const float* topk_w, bool has_shared,
@@ -683,10 +806,9 @@ stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const f
   const int64_t n = int64_t(d.T) * (d.H / 4);
   if (n == 0) return STQ_OK;
   StqTimed tm(STQ_K_COMBINE, s);
-  moe_combine_kernel<<<unsigned(ceil_div<int64_t>(n, 256)), 256, 0, s>>>(
-      d.T, d.H, d.k, P, ws.Y, ws.inv, topk_w, has_shared ? 1 : 0, d.add_residual ? x : nullptr, y, d.out_fp32,
-      ws.err);
-  return stq_launch_status();
+  return stq_launch(moe_combine_kernel, dim3(unsigned(ceil_div<int64_t>(n, 256))), dim3(256), 0, s, d.T, d.H, d.k, P,
+                    static_cast<const float*>(ws.Y), static_cast<const int32_t*>(ws.inv), topk_w, has_shared ? 1 : 0,
+                    d.add_residual ? x : nullptr, y, d.out_fp32, ws.err);
 }
 
 // A library-owned stream per device, created on first use: the MXFP8 shared expert
@@ -784,7 +906,8 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     a.sdq = static_cast<const uint8_t*>(w->sh_down);
     a.sgs = w->sh_gate_sc; a.sus = w->sh_up_sc; a.sds = w->sh_down_sc;
   }
-  a.counts = ws.counts; a.offsets = ws.offsets; a.perm = ws.perm; a.tlist = ws.tlist; a.ntouched = ws.ntouched;
+  a.counts = ws.counts; a.offsets = ws.offsets; a.perm = ws.perm; a.inv = ws.inv; a.tlist = ws.tlist;
+  a.ntouched = ws.ntouched;
   a.h = ws.h; a.Y = ws.Y;
   a.xq = ws.xq; a.xs = ws.xs; a.hq = ws.hq; a.hs = ws.hs;
   a.ntiles = ws.ntiles; a.n_ntiles = ws.n_ntiles;
@@ -792,25 +915,30 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   a.err = ws.err;
   const int slots = d->E < P ? d->E : P;
 
-  // The MXFP8 shared expert on the side stream (its workspace rows P.. and the sticky error
-  // word are all it writes; nothing on the routed path reads them), joined before the combine.
+  const bool prefill = d->regime == STQ_REGIME_PREFILL ||
+                       (d->regime == STQ_REGIME_AUTO && P >= kStqPrefillTokensPerExpert * slots);
+  const bool stq_decode = w->fmt == STQ_FMT_STQ1_0 && !prefill;
+  // The shared expert depends on x alone.  Except in the STQ1_0 decode regime (whose
+  // persistent GEMV kernels take its BF16 tiles as extra work items) it runs on the side
+  // stream, beside the grouping, quantisation and routed experts: its workspace rows P..,
+  // its work counter (sched[3], zeroed on that stream) and the sticky error word are all it
+  // writes, and nothing on the routed path reads them.  Joined before the combine.
   SideStream* side = nullptr;
   ForkJoin* fj = nullptr;
-  if (shared_mx8) {
+  const bool on_side = shared_mx8 || (shared_bf16 && !stq_decode);
+  if (on_side) {
     if ((st = side_stream(&side, &fj)) != STQ_OK) return st;
     std::lock_guard<std::mutex> lock(side->mu);
     if (cudaEventRecord(fj->fork, s) != cudaSuccess || cudaStreamWaitEvent(side->stream, fj->fork, 0) != cudaSuccess)
       return STQ_ERR_CUDA;
-    if ((st = moe_shared_expert_mx8(a, side->stream)) != STQ_OK) return st;
+    st = shared_mx8 ? moe_shared_expert_mx8(a, side->stream) : moe_shared_expert_bf16(a, side->stream);
+    if (st != STQ_OK) return st;
     if (cudaEventRecord(fj->join, side->stream) != cudaSuccess) return STQ_ERR_CUDA;
   }
   if ((st = moe_launch_permute(topk_ids, P, d->E, ws, s)) != STQ_OK) return st;
 
-  const bool prefill = d->regime == STQ_REGIME_PREFILL ||
-                       (d->regime == STQ_REGIME_AUTO && P >= kStqPrefillTokensPerExpert * slots);
   if (w->fmt == STQ_FMT_STQ1_0 && prefill) {
     if ((st = moe_stq_prefill_experts(a, slots, s)) != STQ_OK) return st;
-    if (shared_bf16 && (st = moe_shared_expert_bf16(a, s)) != STQ_OK) return st;
   } else if (w->fmt == STQ_FMT_STQ1_0) {
     // the BF16 shared expert's tiles are the first work items of the two GEMV kernels
     a.routed = 1;
@@ -818,21 +946,23 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     a.sched = ws.sched;
     {
       StqTimed tm(STQ_K_GATE_UP, s);
-      moe_gateup_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->I / 128))), 128, 0, s>>>(a);
+      st = stq_launch(moe_gateup_stq_kernel, dim3(unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->I / 128)))),
+                      dim3(128), 0, s, a);
     }
-    if ((st = stq_launch_status()) != STQ_OK) return st;
+    if (st != STQ_OK) return st;
     a.n_shared_cta = shared_bf16 ? d->H / 16 : 0;
     a.sched = ws.sched + 1;
     {
       StqTimed tm(STQ_K_DOWN, s);
-      moe_down_stq_kernel<<<unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->H / 256), 3)), 128, 0, s>>>(a);
+      st = stq_launch(moe_down_stq_kernel, dim3(unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->H / 256), 4))),
+                      dim3(128), 0, s, a);
     }
-    if ((st = stq_launch_status()) != STQ_OK) return st;
+    if (st != STQ_OK) return st;
   } else {
-    st = moe_mx_experts(a, slots, shared_bf16, s);
+    st = moe_mx_experts(a, slots, s);
     if (st != STQ_OK) return st;
   }
-  if (shared_mx8 && cudaStreamWaitEvent(s, fj->join, 0) != cudaSuccess) return STQ_ERR_CUDA;
+  if (on_side && cudaStreamWaitEvent(s, fj->join, 0) != cudaSuccess) return STQ_ERR_CUDA;
   return moe_launch_combine(*d, P, ws, topk_w, has_shared, x, y, s);
 }
 
@@ -845,24 +975,23 @@ extern "C" int32_t stq_router_ksplit(int32_t H) {
 extern "C" stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T, int32_t H, int32_t E,
                                       int32_t k, float* logits, int32_t* topk_ids, float* topk_w,
                                       stq_stream_t stream) {
-  STQ_HOST_CHECK(x && w_router && logits && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(H % 256 == 0, STQ_ERR_SHAPE);
+  if (T == 0) return STQ_OK;  // nothing to do; the pointers may then be NULL
+  STQ_HOST_CHECK(x && w_router && logits && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
-  if (T == 0) return STQ_OK;
   cudaStream_t s = stq_cuda_stream(stream);
   const int KS = stq_router_ksplit(H);
+  stq_status st;
   {
     StqTimed tm(STQ_K_ROUTER_LOGITS, s);
-    router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 256, 0, s>>>(x, w_router, T, H, E, KS, logits);
+    st = stq_launch(router_logits_kernel, dim3(unsigned(ceil_div(E, 16) * KS)), dim3(256), 0, s, x, w_router, T, H, E,
+                    KS, logits);
   }
-  stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
-  {
-    StqTimed tm(STQ_K_ROUTER_TOPK, s);
-    router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(logits, T, E, KS, k, topk_ids, topk_w);
-  }
-  return stq_launch_status();
+  StqTimed tm(STQ_K_ROUTER_TOPK, s);
+  return stq_launch(router_topk_kernel, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, logits, T, E, KS, k, topk_ids,
+                    topk_w);
 }
 
 extern "C" stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E, int32_t* counts,
@@ -897,28 +1026,27 @@ static __device__ __align__(256) float g_router_scratch[kRouterStaticFloats];
 extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router, int32_t T, int32_t H,
                                              int32_t E, int32_t k, int32_t* topk_ids, float* topk_w,
                                              stq_stream_t stream) {
-  STQ_HOST_CHECK(x && w_router && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(T >= 0 && H > 0 && E > 0 && E <= 1024 && k > 0 && k <= 32 && k <= E, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(H % 256 == 0, STQ_ERR_SHAPE);
-  STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
   const int KS = stq_router_ksplit(H);
   STQ_HOST_CHECK(size_t(KS) * size_t(T) * size_t(E) <= kRouterStaticFloats, STQ_ERR_WORKSPACE);
+  if (T == 0) return STQ_OK;  // nothing to do; the pointers may then be NULL
+  STQ_HOST_CHECK(x && w_router && topk_ids && topk_w, STQ_ERR_INVALID_ARG);
+  STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(w_router), STQ_ERR_ALIGN);
   void* addr = nullptr;
   if (cudaGetSymbolAddress(&addr, g_router_scratch) != cudaSuccess || addr == nullptr) return STQ_ERR_CUDA;
   float* scratch = static_cast<float*>(addr);
-  if (T == 0) return STQ_OK;
   cudaStream_t s = stq_cuda_stream(stream);
   // Every entry the top-k step reads is written first by the logits step, so the
   // array needs no clearing between calls.
+  stq_status st;
   {
     StqTimed tm(STQ_K_ROUTER_LOGITS, s);
-    router_logits_kernel<<<unsigned(ceil_div(E, 16) * KS), 256, 0, s>>>(x, w_router, T, H, E, KS, scratch);
+    st = stq_launch(router_logits_kernel, dim3(unsigned(ceil_div(E, 16) * KS)), dim3(256), 0, s, x, w_router, T, H, E,
+                    KS, scratch);
   }
-  stq_status st = stq_launch_status();
   if (st != STQ_OK) return st;
-  {
-    StqTimed tm(STQ_K_ROUTER_TOPK, s);
-    router_topk_kernel<<<unsigned(ceil_div(T, 4)), 128, 0, s>>>(scratch, T, E, KS, k, topk_ids, topk_w);
-  }
-  return stq_launch_status();
+  StqTimed tm(STQ_K_ROUTER_TOPK, s);
+  return stq_launch(router_topk_kernel, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, scratch, T, E, KS, k, topk_ids,
+                    topk_w);
 }

@@ -4,7 +4,7 @@
 #include "common.cuh"
 
 struct MoeWsLayout {
-  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, ntiles, n_ntiles, sched, total;
+  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, ntiles, n_ntiles, sched, chist, total;
 };
 
 // Device pointers into the caller's workspace.
@@ -24,7 +24,9 @@ struct MoeWs {
   uint8_t* hs;   // [(P+T), I/32]
   int2* ntiles;  // [P/16 + E] (expert, first token) of each GEMM N tile
   int32_t* n_ntiles;
-  int32_t* sched;  // [4] work counters of the persistent GEMV kernels (zeroed by the permute kernel)
+  int32_t* sched;  // [4] work counters of the persistent GEMV kernels: 0-2 zeroed by the permute
+                   // kernel, 3 (the shared expert's down launch) by the shared gate/up kernel
+  int32_t* chist;  // [ceil(P/1024)][E] per-chunk expert counts of the many-CTA grouping (nullptr: one CTA)
 };
 
 // Kernel arguments (by value).
@@ -36,7 +38,7 @@ struct MoeArgs {
   const uint16_t *sg, *su, *sd;    // shared expert, bf16
   const uint8_t *sgq, *suq, *sdq;  // shared expert, MXFP8 codes
   const uint8_t *sgs, *sus, *sds;  // and scales
-  const int32_t *counts, *offsets, *perm, *tlist, *ntouched;
+  const int32_t *counts, *offsets, *perm, *inv, *tlist, *ntouched;
   uint16_t* h;
   float* Y;
   uint8_t *xq, *xs, *hq, *hs;
@@ -69,14 +71,18 @@ stq_status moe_shared_expert_mx8(const MoeArgs& a, cudaStream_t s);
 stq_status moe_stq_prefill_experts(const MoeArgs& a, int slots, cudaStream_t s);
 MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L);
 
-// Routed MXFP4 experts (+ the shared BF16 expert): gate/up, SwiGLU, down.
-stq_status moe_mx_experts(const MoeArgs& a, int slots, bool has_shared, cudaStream_t s);
+// Routed MXFP4 experts: activations quantised to MXFP8 in sorted pair order, gate/up,
+// SwiGLU, down.
+stq_status moe_mx_experts(const MoeArgs& a, int slots, cudaStream_t s);
+// Their prefill regime on CTA pairs (gemm_mx2.cu), activations already quantised.
+stq_status moe_mx_experts_pair(const MoeArgs& a, int slots, cudaStream_t s);
 
 // BF16 -> MXFP8 quantisation launch (pack.cu).
 stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales,
                                      cudaStream_t s);
-// Same, with output row r taken from input row rowmap[r] / k (gather into sorted pair order)
-// of src_rows input rows; err: the error word of the checked build's source-row check.
-stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int64_t K, const int32_t* rowmap, int k,
-                                            int64_t src_rows, int32_t* err, uint8_t* codes, uint8_t* scales,
-                                            cudaStream_t s);
+// Same into sorted pair order: each of the T token rows is quantised once and written to
+// the k output rows inv[t*k + s] (-1 = none; positions below out_rows); err: the error word
+// of the checked build's position check.
+stq_status stq_mxfp8_quantize_scatter_launch(const uint16_t* x, int64_t T, int64_t K, const int32_t* inv, int k,
+                                             int64_t out_rows, int32_t* err, uint8_t* codes, uint8_t* scales,
+                                             cudaStream_t s);

@@ -19,6 +19,7 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_bf16_kernel(const uint16_t* 
   __shared__ double part[kThreads / 32];
   __shared__ double s_scale;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  stq_pdl_begin();
   const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(row) * H);
   uint4* yr = reinterpret_cast<uint4*>(y + size_t(row) * H);
   const int n8 = H / 8;
@@ -71,9 +72,6 @@ extern "C" stq_status stq_rmsnorm_bf16(const uint16_t* x, int64_t T, int64_t H, 
   STQ_HOST_CHECK(x != nullptr && y != nullptr, STQ_ERR_INVALID_ARG);
   STQ_HOST_CHECK(stq_aligned16(x) && stq_aligned16(y), STQ_ERR_ALIGN);
   const cudaStream_t s = stq_cuda_stream(stream);
-  {
-    StqTimed tm(STQ_K_RMSNORM, s);
-    rmsnorm_bf16_kernel<<<unsigned(T), kThreads, 0, s>>>(x, int(H), eps, y);
-  }
-  return stq_launch_status();
+  StqTimed tm(STQ_K_RMSNORM, s);
+  return stq_launch(rmsnorm_bf16_kernel, dim3(unsigned(T)), dim3(kThreads), 0, s, x, int(H), eps, y);
 }

@@ -302,14 +302,19 @@ __global__ void mxfp4_unpack_kernel(const uint8_t* __restrict__ codes, const uin
 // Grid (column chunks of 2048 elements, rows; rows beyond 65535 loop): thread = 8
 // consecutive elements, 4 threads = one 32-element group, no 64-bit division per thread.
 // RPB rows per CTA (rows RPB*blockIdx.y .. +RPB, then strided by the grid): every row's
-// source index and activation load are issued before the first row is quantised, so the
-// two dependent load latencies are paid once per RPB rows.
+// activation load is issued before the first row is quantised, so the load latency is paid
+// once per RPB rows.
+// Scatter (dst != nullptr): source row r (a token) is quantised once and its codes and
+// scales are written to the k output rows dst[r*k + s], s = 0..k-1 (the sorted position of
+// each of its (token, slot) pairs; -1 = none); out_rows bounds those positions.  Otherwise
+// output row r is source row r.
 template <int RPB>
 __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                int64_t K, uint8_t* __restrict__ codes,
                                                                uint8_t* __restrict__ scales,
-                                                               const int32_t* __restrict__ rowmap, int k,
-                                                               int64_t src_rows, int32_t* err) {
+                                                               const int32_t* __restrict__ dst, int k,
+                                                               int64_t out_rows, int32_t* err) {
+  stq_pdl_begin();
   const int part = int(threadIdx.x & 3);
   const int64_t col8 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // 8-element chunk of the row
   const bool active = col8 < K / 8;                                     // whole 4-thread groups
@@ -319,16 +324,12 @@ __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* _
     for (int j = 0; j < RPB; ++j) {
       raw[j] = make_uint4(0u, 0u, 0u, 0u);
       const int64_t row = r0 + j;
-      if (active && row < rows) {
-        const int64_t src = rowmap != nullptr ? int64_t(rowmap[row] / k) : row;
-        if (STQ_DCHECK(src >= 0 && src < src_rows, err)) raw[j] = *reinterpret_cast<const uint4*>(x + src * K + col8 * 8);
-      }
+      if (active && row < rows) raw[j] = *reinterpret_cast<const uint4*>(x + row * K + col8 * 8);
     }
 #pragma unroll
     for (int j = 0; j < RPB; ++j) {
       const int64_t row = r0 + j;
       if (row >= rows) break;  // the same for every thread of the CTA
-      const int64_t gi = row * (K / 32) + (col8 >> 2);
       float v[8];
       float amax = 0.f;
       bool bad = false;
@@ -369,8 +370,18 @@ __global__ void __launch_bounds__(256) mxfp8_quant_bf16_kernel(const uint16_t* _
           if (i < 4) lo |= pair << (8 * i); else hi |= pair << (8 * (i - 4));
         }
       }
-      *reinterpret_cast<uint2*>(codes + gi * 32 + part * 8) = make_uint2(lo, hi);
-      if (part == 0) scales[gi] = uint8_t(e);
+      const int64_t g32 = col8 >> 2;  // 32-element group of the row
+      if (dst == nullptr) {
+        *reinterpret_cast<uint2*>(codes + row * K + col8 * 8) = make_uint2(lo, hi);
+        if (part == 0) scales[row * (K / 32) + g32] = uint8_t(e);
+      } else {
+        for (int s = 0; s < k; ++s) {
+          const int64_t pos = dst[row * k + s];
+          if (pos < 0 || !STQ_DCHECK(pos < out_rows, err)) continue;
+          *reinterpret_cast<uint2*>(codes + pos * K + col8 * 8) = make_uint2(lo, hi);
+          if (part == 0) scales[pos * (K / 32) + g32] = uint8_t(e);
+        }
+      }
     }
   }
 }
@@ -459,28 +470,26 @@ stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K,
   const int64_t threads = rows * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
+  const int32_t* no_map = nullptr;
+  int32_t* no_err = nullptr;
   if (rows >= kQuantMultiRow)
-    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1, rows,
-                                                                   nullptr);
-  else
-    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, nullptr, 1, rows,
-                                                                   nullptr);
-  return stq_launch_status();
+    return stq_launch(mxfp8_quant_bf16_kernel<8>, quant_grid(rows, K), dim3(256), 0, s, x, rows, K, codes, scales, no_map,
+                      1, rows, no_err);
+  return stq_launch(mxfp8_quant_bf16_kernel<1>, quant_grid(rows, K), dim3(256), 0, s, x, rows, K, codes, scales, no_map,
+                    1, rows, no_err);
 }
 
-stq_status stq_mxfp8_quantize_gather_launch(const uint16_t* x, int64_t rows, int64_t K, const int32_t* rowmap, int k,
-                                            int64_t src_rows, int32_t* err, uint8_t* codes, uint8_t* scales,
-                                            cudaStream_t s) {
-  const int64_t threads = rows * (K / 32) * 4;
+stq_status stq_mxfp8_quantize_scatter_launch(const uint16_t* x, int64_t T, int64_t K, const int32_t* inv, int k,
+                                             int64_t out_rows, int32_t* err, uint8_t* codes, uint8_t* scales,
+                                             cudaStream_t s) {
+  const int64_t threads = T * (K / 32) * 4;
   if (threads == 0) return STQ_OK;
   StqTimed tm(STQ_K_QUANT_X, s);
-  if (rows >= kQuantMultiRow)
-    mxfp8_quant_bf16_kernel<8><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k, src_rows,
-                                                                   err);
-  else
-    mxfp8_quant_bf16_kernel<1><<<quant_grid(rows, K), 256, 0, s>>>(x, rows, K, codes, scales, rowmap, k, src_rows,
-                                                                   err);
-  return stq_launch_status();
+  if (T >= kQuantMultiRow)
+    return stq_launch(mxfp8_quant_bf16_kernel<8>, quant_grid(T, K), dim3(256), 0, s, x, T, K, codes, scales, inv, k,
+                      out_rows, err);
+  return stq_launch(mxfp8_quant_bf16_kernel<1>, quant_grid(T, K), dim3(256), 0, s, x, T, K, codes, scales, inv, k,
+                    out_rows, err);
 }
 
 extern "C" stq_status mxfp8_quantize_bf16(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes,

@@ -173,7 +173,7 @@ enum { STQ_FMT_STQ1_0 = 0, STQ_FMT_MXFP4 = 1 };
  * logits are summed over that many slices of H); on return its first T*E floats
  * hold the logits [T, E].  A non-finite logit counts as probability 0 (a token whose
  * chosen probabilities are all 0 gets weights 1/k).  E <= 1024, k <= 32, k <= E,
- * H % 256 == 0. */
+ * H % 256 == 0.  T == 0 is a no-op (pointers may then be NULL). */
 int32_t stq_router_ksplit(int32_t H);
 stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_router, int32_t T,
                            int32_t H, int32_t E, int32_t k, float* logits,
@@ -206,19 +206,23 @@ stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
  * Every call shares the array and leaves its last contents there (each call
  * writes every entry it reads, so nothing needs clearing); calls whose kernels
  * overlap on the GPU (other streams, other host threads) race on it.  Allocates
- * nothing.  Outputs: topk_ids int32 [T, k], topk_w f32 [T, k]. */
+ * nothing.  Outputs: topk_ids int32 [T, k], topk_w f32 [T, k].  T == 0 is a no-op
+ * (pointers may then be NULL). */
 stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* w_router,
                                   int32_t T, int32_t H, int32_t E, int32_t k,
                                   int32_t* topk_ids, float* topk_w, stq_stream_t stream);
 
 /* Format of the shared expert (moe_weights.sh_fmt).
  *   STQ_SHARED_BF16   sh_gate / sh_up / sh_down are bf16 matrices; h is rounded to bf16.
+ *                     In the STQ1_0 decode regime its tiles are extra work items of the
+ *                     routed GEMV kernels; otherwise (MXFP4 experts, STQ1_0 prefill regime)
+ *                     it runs on the library-owned side stream described below.
  *   STQ_SHARED_MXFP8  "Hy4-preview-SF-WFP4AFP8", "Quant Diff": the shared experts'
  *                     gate/up/down are MXFP8 W8A8 g32.  sh_* are E4M3 codes (one byte
  *                     per weight, row-major) and sh_*_sc their UE8M0 scales [rows][K/32]
  *                     (as written by mxfp8_quantize_bf16); x and h are quantised to
  *                     MXFP8 g32 (the activation rule of mxfp8_quantize_bf16) and the
- *                     products accumulate in FP32.  It depends on x alone, so
+ *                     products accumulate in FP32.  The shared expert depends on x alone, so
  *                     moe_expert_forward runs it on a library-owned stream of the
  *                     current device (created with two events on first use, then
  *                     reused; not device memory), forked from `stream` after the
