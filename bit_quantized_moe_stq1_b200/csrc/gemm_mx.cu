@@ -399,8 +399,11 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, cudaStream_t s) {
   // 128 tokens per expert on average, the gate/up pair (whose SwiGLU/MXFP8 epilogue and
   // item balance measured slower there) at most 128
   const int slots_ = a.E < P ? a.E : P;
-  // prefill (128 or more routed tokens per expert on average): the CTA-pair GEMM
-  if (int64_t(P) / slots_ >= 128) return moe_mx_experts_pair(a, slots_, s);
+  // the CTA-pair GEMM from this many routed tokens per expert on average (0: not used; it
+  // measured slower than the one-CTA kernels on the 4096-token prefill layer)
+  constexpr int64_t kPairFromTokensPerExpert = 0;
+  if (kPairFromTokensPerExpert > 0 && int64_t(P) / slots_ >= kPairFromTokensPerExpert)
+    return moe_mx_experts_pair(a, slots_, s);
   const int nt_dn = pick_nt(int64_t(P) / slots_);
   const int nt = nt_dn > 128 ? 128 : nt_dn;
   if ((st = stq_tile_plan_launch(a.counts, a.E, nt, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;

@@ -13,12 +13,13 @@
 // rows) x up to 240 tokens of one expert over all of K.  Per item both CTAs:
 //   warps 0, 6 (producers, alternate 128-k stages): TMA of the CTA's 128 weight rows and of
 //      its half of the N token rows (rows n0 + rank * N/2 ..), whose completion bytes count
-//      on the rank-0 CTA's barrier; the UE8M0 scales, re-laid into the scale-factor atoms:
-//      the CTA's own 128 weight rows, and the activations of all N tokens;
+//      on the rank-0 CTA's barrier; in rank 0 also the UE8M0 scales of both CTAs, re-laid
+//      into the scale-factor atoms (each CTA's own 128 weight rows, and the activations of
+//      all N tokens), the peer's written into its shared memory;
 //   warp 1: TMEM (both CTAs, cta_group::2); in the rank-0 CTA one thread issues the scale
 //      copies and four M = 256 MMAs per stage, and commits to both CTAs' barriers;
 //   warps 2-5: the CTA's epilogue from its own TMEM (its 128 rows x N tokens).
-// Barriers: full[s] (rank 0; the two CTAs' loads and producers), empty[s] (both; one
+// Barriers: full[s] (rank 0; rank 0's producer and both CTAs' loads), empty[s] (both; one
 // commit), tfull[b] (both; one commit), tempty[b] (rank 0; the eight epilogue warps).
 // Every wait is bounded; after a timeout each role records STQ_ERR_TIMEOUT, keeps going to
 // the end, and both CTAs meet at a final cluster barrier before TMEM is freed, so no CTA
@@ -132,7 +133,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 2);                 // both CTAs' producers (rank 0's with the bytes)
+      tc::mbar_init(&full[s], 1);                 // rank 0's producer, with both CTAs' bytes
       tc::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -166,23 +167,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int q = 0; q < kStages; ++q) last_round[q] = -1;
     int cg = pid, cit = -1, cncols = 0;   // look-ahead cursor
     Item CI{};
-    auto sf_load = [&](uint32_t (&va)[4], uint32_t (&vb0)[4], uint32_t (&vb1)[4]) {
+    // rank 0 lays out the scale factors of both CTAs (its own weight rows, the peer's rows,
+    // and the activations of all N tokens, which both need), so that everything the MMAs
+    // read is published by rank 0's producers to rank 0's barriers
+    auto sf_load = [&](uint32_t (&va0)[4], uint32_t (&va1)[4], uint32_t (&vb0)[4], uint32_t (&vb1)[4]) {
       const int it = cg / nk, kt = cg % nk;
       if (it != cit) {
         cit = it;
-        CI = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, rank);
+        CI = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, 0);
         cncols = CI.valid ? gemm::item_cols(CI, NT) : 0;
       }
       const int nkj = CI.valid ? nk : 0;   // past the last item: zeros, no loads
-      if (PAIR) load_sf_gu(va, p.sa, p.sa2, CI.arow, k32, kt, nkj, lane);
-      else load_sf(va, p.sa, CI.arow, 128, 0x7fffffff, k32, kt, nkj, lane);
+      if (PAIR) {
+        load_sf_gu(va0, p.sa, p.sa2, CI.arow, k32, kt, nkj, lane);
+        load_sf_gu(va1, p.sa, p.sa2, CI.arow + kRowsPerCta, k32, kt, nkj, lane);
+      } else {
+        load_sf(va0, p.sa, CI.arow, 128, 0x7fffffff, k32, kt, nkj, lane);
+        load_sf(va1, p.sa, CI.arow + kRowsPerCta, 128, 0x7fffffff, k32, kt, nkj, lane);
+      }
       load_sf(vb0, p.sb, CI.brow, cncols, p.Ptot, k32, kt, nkj, lane);
       if (C::kSfbAtoms > 1) load_sf(vb1, p.sb, CI.brow + 128, cncols - 128, p.Ptot, k32, kt, nkj, lane);
       cg += 2;
     };
-    uint32_t ra[kLook][4], rb0[kLook][4], rb1[kLook][4];
+    auto peer_sf = [&](uint8_t* dst, const uint32_t (&v)[4]) {
+      tc::st_shared_cluster_v4(tc::mapa_shared(tc::smem_u32(dst + lane * 16), 1), make_uint4(v[0], v[1], v[2], v[3]));
+    };
+    uint32_t ra0[kLook][4], ra1[kLook][4], rb0[kLook][4], rb1[kLook][4];
+    if (rank == 0) {
 #pragma unroll
-    for (int d = 0; d < kLook; ++d) sf_load(ra[d], rb0[d], rb1[d]);
+      for (int d = 0; d < kLook; ++d) sf_load(ra0[d], ra1[d], rb0[d], rb1[d]);
+    }
     int g = pid, cur_it = -1, ncols = 0;
     Item I{};
     bool more = true;
@@ -201,15 +215,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         const int j = g >> 1;
         const int s = 2 * (j % np) + pid, r = j / np;
-        if (r > 0 && !tc::mbar_wait_cluster(&empty[s], (r - 1) & 1, p.err)) {
+        if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
           more = false;
           break;
         }
         uint8_t* st = smem + s * kStage;
-        store_sf(st + kOffSfa, ra[d], lane);
-        store_sf(st + kOffSfb, rb0[d], lane);
-        if (C::kSfbAtoms > 1) store_sf(st + kOffSfb + kSf, rb1[d], lane);
-        tc::fence_proxy_async_smem();
+        if (rank == 0) {
+          store_sf(st + kOffSfa, ra0[d], lane);
+          store_sf(st + kOffSfb, rb0[d], lane);
+          if (C::kSfbAtoms > 1) store_sf(st + kOffSfb + kSf, rb1[d], lane);
+          peer_sf(st + kOffSfa, ra1[d]);
+          peer_sf(st + kOffSfb, rb0[d]);
+          if (C::kSfbAtoms > 1) peer_sf(st + kOffSfb + kSf, rb1[d]);
+          tc::fence_proxy_async_cluster();
+        }
         __syncwarp();
         if (lane == 0) {
           const uint32_t bar0 = tc::mapa_shared(tc::smem_u32(&full[s]), 0);
@@ -222,11 +241,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc::tma_load_2d_pair(st + kOffA, &tmA, kt * kKT, I.arow, bar0);
           }
           tc::tma_load_2d_pair(st + kOffB, &tmB, kt * kKT, bhalf, bar0);
-          // rank 1's scale-factor stores are released to rank 0's MMA thread by this arrival
-          if (rank != 0) tc::mbar_arrive_remote(bar0);
         }
         last_round[s] = r;
-        sf_load(ra[d], rb0[d], rb1[d]);   // the step kLook ahead
+        if (rank == 0) sf_load(ra0[d], ra1[d], rb0[d], rb1[d]);   // the step kLook ahead
         g += 2;
       }
     }
@@ -234,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // pair passes the final cluster barrier
     if (rank == 0)
       for (int q = 0; q < kStages; ++q)
-        if (last_round[q] >= 0) tc::mbar_wait_cluster(&full[q], last_round[q] & 1, p.err);
+        if (last_round[q] >= 0) tc::mbar_wait(&full[q], last_round[q] & 1, p.err);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issue (rank 0)
     if (rank == 0 && lane == 0) {
@@ -245,13 +262,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!I.valid) break;
         const int ncols = gemm::item_cols(I, NT);
         const int buf = it & 1;
-        if (it >= 2 && !tc::mbar_wait_cluster(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) ok = false;
+        if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) ok = false;
         tc::fence_after_sync();
         const uint32_t acc_col = tmem + uint32_t(buf * kAccStride);
         for (int kt = 0; kt < nk && ok; ++kt, ++g) {
           const int j = g >> 1;
           const int s = 2 * (j % (kStages / 2)) + (g & 1), r = j / (kStages / 2);
-          if (!tc::mbar_wait_cluster(&full[s], r & 1, p.err)) {
+          if (!tc::mbar_wait(&full[s], r & 1, p.err)) {
             ok = false;
             break;
           }
@@ -283,7 +300,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const Item I = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, rank);
       if (!I.valid) break;
       const int buf = it & 1;
-      bool ok = tc::mbar_wait_cluster(&tfull[buf], (it >> 1) & 1, p.err);
+      bool ok = tc::mbar_wait(&tfull[buf], (it >> 1) & 1, p.err);
       if constexpr (PAIR) ok = gemm::all_of_epilogue(ok);
       if (!ok) break;
       tc::fence_after_sync();
@@ -291,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                      lane);
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive_remote(tc::mapa_shared(tc::smem_u32(&tempty[buf]), 0));
+      if (lane == 0) tc::mbar_arrive_peer(tc::mapa_shared(tc::smem_u32(&tempty[buf]), 0));
     }
   }
   // both CTAs: every role is done (or gave up) before TMEM is freed and the CTAs exit

@@ -104,41 +104,31 @@ __device__ __forceinline__ void stq_step(const StqBlockRegs<NT>& r, uint32_t lut
   }
 }
 
-// Activations: thread t of a quad holds, per block, k = 64t .. 64t+63 of its token column as
-// eight 16-byte chunks (chunk q feeds steps 2q and 2q+1).  They stream through a ring of
-// kXRing chunks loaded kXRing chunks ahead, across block boundaries, so a chunk's load
-// latency hides behind the steps before it without holding a whole block in registers.
-constexpr int kXRing = 4;
-
-__device__ __forceinline__ uint4 x_chunk(const uint4* xq, int j) {
-  // chunk j = 8 * (block - b0) + q of this lane (xq: the lane's first chunk; nullptr = padding)
-  return xq != nullptr ? xq[(j >> 3) * 32 + (j & 7)] : make_uint4(0u, 0u, 0u, 0u);
-}
-
-// acc[i][*] += (d/2) * sum over one 256-k block, for NT tiles; jb = the block's index from
-// b0 (its chunks are 8 jb .. 8 jb + 7), nchunks = the chunks of the whole range.
+template <int I, int NT>
+struct StqSteps {
+  __device__ __forceinline__ static void run(const StqBlockRegs<NT>& r, const uint4 (&xv)[8], uint32_t lut,
+                                             float (&part)[NT][4]) {
+    const uint4 q = xv[I >> 1];
+    if constexpr (I & 1)
+      stq_step<I, NT>(r, lut, q.z, q.w, part);
+    else
+      stq_step<I, NT>(r, lut, q.x, q.y, part);
+    StqSteps<I + 1, NT>::run(r, xv, lut, part);
+  }
+};
 template <int NT>
-__device__ __forceinline__ void stq_block(const StqBlockRegs<NT>& r, uint4 (&xr)[kXRing], const uint4* xq, int jb,
-                                          int nchunks, uint32_t lut, float (&acc)[NT][4]) {
+struct StqSteps<16, NT> {
+  __device__ __forceinline__ static void run(const StqBlockRegs<NT>&, const uint4 (&)[8], uint32_t, float (&)[NT][4]) {}
+};
+
+// acc[i][*] += (d/2) * sum over one 256-k block, for NT tiles.
+template <int NT>
+__device__ __forceinline__ void stq_block(const StqBlockRegs<NT>& r, const uint4 (&xv)[8], uint32_t lut,
+                                          float (&acc)[NT][4]) {
   float part[NT][4];
 #pragma unroll
   for (int i = 0; i < NT; ++i) part[i][0] = part[i][1] = part[i][2] = part[i][3] = 0.f;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint4 c = xr[q % kXRing];
-    const int jn = 8 * jb + q + kXRing;  // the chunk that takes this ring slot next
-    if (jn < nchunks) xr[q % kXRing] = x_chunk(xq, jn);
-    switch (q) {  // compile-time after unrolling
-      case 0: stq_step<0, NT>(r, lut, c.x, c.y, part); stq_step<1, NT>(r, lut, c.z, c.w, part); break;
-      case 1: stq_step<2, NT>(r, lut, c.x, c.y, part); stq_step<3, NT>(r, lut, c.z, c.w, part); break;
-      case 2: stq_step<4, NT>(r, lut, c.x, c.y, part); stq_step<5, NT>(r, lut, c.z, c.w, part); break;
-      case 3: stq_step<6, NT>(r, lut, c.x, c.y, part); stq_step<7, NT>(r, lut, c.z, c.w, part); break;
-      case 4: stq_step<8, NT>(r, lut, c.x, c.y, part); stq_step<9, NT>(r, lut, c.z, c.w, part); break;
-      case 5: stq_step<10, NT>(r, lut, c.x, c.y, part); stq_step<11, NT>(r, lut, c.z, c.w, part); break;
-      case 6: stq_step<12, NT>(r, lut, c.x, c.y, part); stq_step<13, NT>(r, lut, c.z, c.w, part); break;
-      default: stq_step<14, NT>(r, lut, c.x, c.y, part); stq_step<15, NT>(r, lut, c.z, c.w, part); break;
-    }
-  }
+  StqSteps<0, NT>::run(r, xv, lut, part);
 #pragma unroll
   for (int i = 0; i < NT; ++i) {
     const float dg = __half2float(__ushort_as_half((unsigned short)(r.d[i] & 0xFFFFu))) * 0.5f;
@@ -150,24 +140,32 @@ __device__ __forceinline__ void stq_block(const StqBlockRegs<NT>& r, uint4 (&xr)
   }
 }
 
-// Whole-warp STQ1_0 GEMV over blocks [b0, b1) of NT tiles, token column g of this lane's
-// quad taken from xrow (nullptr = padding column).  Weight loads for block b+1 are in
-// flight while block b is multiplied; activations stream kXRing chunks ahead.
+__device__ __forceinline__ void load_x_block(uint4 (&xv)[8], const uint16_t* xrow, int b, int t) {
+  if (xrow != nullptr) {
+    const uint4* p = reinterpret_cast<const uint4*>(xrow + 256 * b + 64 * t);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) xv[q] = p[q];
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) xv[q] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Whole-warp STQ1_0 GEMV over blocks [b0, b1) of NT tiles, token column g of this
+// lane's quad taken from xrow (nullptr = padding column).  Weight loads for block
+// b+1 are in flight while block b is multiplied.
 template <int NT>
 __device__ __forceinline__ void stq_warp_gemv(const uint8_t* const (&tb)[NT], int b0, int b1, const uint16_t* xrow,
                                               uint32_t lut, float (&acc)[NT][4]) {
   const int lane = threadIdx.x & 31, t = lane & 3;
   if (b0 >= b1) return;
-  const uint4* xq = xrow != nullptr ? reinterpret_cast<const uint4*>(xrow + 256 * b0 + 64 * t) : nullptr;
-  const int nchunks = 8 * (b1 - b0);
-  uint4 xr[kXRing];
-#pragma unroll
-  for (int j = 0; j < kXRing; ++j) xr[j] = x_chunk(xq, j);
   StqBlockRegs<NT> cur, nxt;
   stq_load<NT>(cur, tb, b0, lane);
   for (int b = b0; b < b1; ++b) {
     if (b + 1 < b1) stq_load<NT>(nxt, tb, b + 1, lane);
-    stq_block<NT>(cur, xr, xq, b - b0, nchunks, lut, acc);
+    uint4 xv[8];
+    load_x_block(xv, xrow, b, t);
+    stq_block<NT>(cur, xv, lut, acc);
     cur = nxt;
   }
 }
