@@ -11,14 +11,14 @@
 //
 // A work item is 256 weight rows (gate/up: 128 features, each CTA 64 gate + the same 64 up
 // rows) x up to 240 tokens of one expert over all of K.  Per item both CTAs:
-//   warps 0, 6 (producers, alternate 128-k stages): TMA of the CTA's 128 weight rows and of
+//   warps 5-8 (producers, 128-k stages in turn): TMA of the CTA's 128 weight rows and of
 //      its half of the N token rows (rows n0 + rank * N/2 ..), whose completion bytes count
 //      on the rank-0 CTA's barrier; in rank 0 also the UE8M0 scales of both CTAs, re-laid
 //      into the scale-factor atoms (each CTA's own 128 weight rows, and the activations of
 //      all N tokens), the peer's written into its shared memory;
-//   warp 1: TMEM (both CTAs, cta_group::2); in the rank-0 CTA one thread issues the scale
+//   warp 0: TMEM (both CTAs, cta_group::2); in the rank-0 CTA one thread issues the scale
 //      copies and four M = 256 MMAs per stage, and commits to both CTAs' barriers;
-//   warps 2-5: the CTA's epilogue from its own TMEM (its 128 rows x N tokens).
+//   warps 1-4: the CTA's epilogue from its own TMEM (its 128 rows x N tokens).
 // Barriers: full[s] (rank 0; rank 0's producer and both CTAs' loads), empty[s] (both; one
 // commit), tfull[b] (both; one commit), tempty[b] (rank 0; the eight epilogue warps).
 // Every wait is bounded; after a timeout each role records STQ_ERR_TIMEOUT, keeps going to
@@ -42,8 +42,12 @@ constexpr int kATile = 128 * 128;             // one CTA's 128 x 128 E2M1 weight
 constexpr uint32_t kATx = 128 * 128 / 2;      // bytes the TMA delivers for it
 constexpr int kSf = 512;                      // scale-factor atom: 128 rows x 4 k-blocks
 constexpr int kUBuf = 4 * 32 * 9 * 4;         // gate/up exchange of the epilogue
-constexpr int kThreads = 224;
-constexpr int kProducer2 = 6;
+// Warps: 0 MMA (rank 0 issues; TMEM in both), 1-4 epilogue (TMEM lane quarters 1, 2, 3, 0),
+// 5-8 producers.  Rank 0's producers lay out both CTAs' scale factors (about 2,000 cycles per
+// stage, measured), so four of them take the stages in turn and keep ahead of the MMAs.
+constexpr int kProducers = 4;
+constexpr int kProducer0 = 5;
+constexpr int kThreads = 32 * (kProducer0 + kProducers);
 constexpr uint32_t kCols = 512;
 
 // NT tokens per item (both CTAs; each holds NT/2 token rows): shared-memory stages and the
@@ -59,7 +63,7 @@ struct PairCfg {
   static constexpr int kOffSfa = kOffB + kBTile;
   static constexpr int kOffSfb = kOffSfa + kSf;
   static constexpr int kStage = (kOffSfb + kSfbAtoms * kSf + 1023) / 1024 * 1024;
-  static constexpr int kStagesRaw = ((226 * 1024 - 2048 - kUBuf) / kStage) & ~1;
+  static constexpr int kStagesRaw = ((226 * 1024 - 2048 - kUBuf) / kStage) & ~(kProducers - 1);
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
   static constexpr int kSmem = kStages * kStage + kUBuf + 1024 /* barriers */ + 1024 /* alignment */;
   static constexpr uint32_t kTxPair = 2 * (kATx + uint32_t(kBTile));   // both CTAs' bytes per stage
@@ -67,7 +71,7 @@ struct PairCfg {
   static constexpr int kColSfa = NT > 128 ? NT : 2 * NT;
   static constexpr int kColSfb = kColSfa + 4;
   static_assert(NT % 16 == 0 && NT <= 240, "tile N");
-  static_assert(kStages >= 2, "stages");
+  static_assert(kStages >= kProducers, "stages");
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kBTile % 1024 == 0 && kStage % 1024 == 0, "128-byte swizzle atoms");
   static_assert(kColSfb + 4 * kSfbAtoms <= (NT > 128 ? 256 : 512), "TMEM columns");
@@ -145,22 +149,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (PAIR) tc::prefetch_tensormap(&tmA2);
     tc::prefetch_tensormap(&tmB);
   }
-  if (warp == 1) tc::tmem_alloc_pair(tmem_holder, kCols);
+  if (warp == 0) tc::tmem_alloc_pair(tmem_holder, kCols);
   tc::fence_before_sync();
   tc::cluster_sync();   // both CTAs' barriers are initialised before any peer signals them
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_holder;
   stq_pdl_begin();   // barriers and TMEM are set up; from here on global memory is read
 
-  if (warp == 0 || warp == kProducer2) {
+  if (warp >= kProducer0) {
     // ---------------------------------------------------------------- producers
     // Global k-step g = item * nk + kt; producer pid takes the steps of its parity, its j-th
-    // step (j = g / 2) at stage 2 (j % np) + pid, round j / np (np = kStages / 2).  The
+    // step (j = g / kProducers) at stage kProducers (j % np) + pid, round j / np
+    // (np = kStages / kProducers).  The
     // scale factors, which the warp re-lays through registers, are read kLook of its steps
     // ahead (a second cursor over the same steps), so their latency hides behind earlier
     // stages, across item boundaries too.
-    const int pid = warp == 0 ? 0 : 1;
-    constexpr int np = kStages / 2;
+    const int pid = warp - kProducer0;
+    constexpr int np = kStages / kProducers;
     constexpr int kLook = 4;
     int last_round[kStages];
 #pragma unroll
@@ -187,7 +192,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       load_sf(vb0, p.sb, CI.brow, cncols, p.Ptot, k32, kt, nkj, lane);
       if (C::kSfbAtoms > 1) load_sf(vb1, p.sb, CI.brow + 128, cncols - 128, p.Ptot, k32, kt, nkj, lane);
-      cg += 2;
+      cg += kProducers;
     };
     auto peer_sf = [&](uint8_t* dst, const uint32_t (&v)[4]) {
       tc::st_shared_cluster_v4(tc::mapa_shared(tc::smem_u32(dst + lane * 16), 1), make_uint4(v[0], v[1], v[2], v[3]));
@@ -199,22 +204,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     int g = pid, cur_it = -1, ncols = 0;
     Item I{};
+    // the next item's descriptor is read one item ahead (its loads are in flight meanwhile)
+    Item In = cta_item<NT>(p.tiles, cid + (g / nk) * NC, MT2, kRowsPerCta, rank);
     bool more = true;
     while (more) {
 #pragma unroll
       for (int d = 0; d < kLook; ++d) {
         const int it = g / nk, kt = g % nk;
         if (it != cur_it) {
+          I = (cur_it < 0 || it == cur_it + 1) ? In : cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, rank);
           cur_it = it;
-          I = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, rank);
+          In = cta_item<NT>(p.tiles, cid + (it + 1) * NC, MT2, kRowsPerCta, rank);
           ncols = I.valid ? gemm::item_cols(I, NT) : 0;
         }
         if (!I.valid) {
           more = false;
           break;
         }
-        const int j = g >> 1;
-        const int s = 2 * (j % np) + pid, r = j / np;
+        const int j = g / kProducers;
+        const int s = kProducers * (j % np) + pid, r = j / np;
         if (r > 0 && !tc::mbar_wait(&empty[s], (r - 1) & 1, p.err)) {
           more = false;
           break;
@@ -244,7 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         last_round[s] = r;
         if (rank == 0) sf_load(ra0[d], ra1[d], rb0[d], rb1[d]);   // the step kLook ahead
-        g += 2;
+        g += kProducers;
       }
     }
     // rank 0: every load of both CTAs has landed (they count on its barriers) before the
@@ -252,22 +260,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (rank == 0)
       for (int q = 0; q < kStages; ++q)
         if (last_round[q] >= 0) tc::mbar_wait(&full[q], last_round[q] & 1, p.err);
-  } else if (warp == 1) {
+  } else if (warp == 0) {
     // ---------------------------------------------------------------- MMA issue (rank 0)
     if (rank == 0 && lane == 0) {
       int g = 0;
       bool ok = true;
+      Item In = cta_item<NT>(p.tiles, cid, MT2, kRowsPerCta, 0);
       for (int it = 0; ok; ++it) {
-        const Item I = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, 0);
+        const Item I = In;
         if (!I.valid) break;
+        In = cta_item<NT>(p.tiles, cid + (it + 1) * NC, MT2, kRowsPerCta, 0);   // read one item ahead
         const int ncols = gemm::item_cols(I, NT);
         const int buf = it & 1;
         if (it >= 2 && !tc::mbar_wait(&tempty[buf], ((it >> 1) - 1) & 1, p.err)) ok = false;
         tc::fence_after_sync();
         const uint32_t acc_col = tmem + uint32_t(buf * kAccStride);
         for (int kt = 0; kt < nk && ok; ++kt, ++g) {
-          const int j = g >> 1;
-          const int s = 2 * (j % (kStages / 2)) + (g & 1), r = j / (kStages / 2);
+          const int j = g / kProducers, np = kStages / kProducers;
+          const int s = kProducers * (j % np) + g % kProducers, r = j / np;
           if (!tc::mbar_wait(&full[s], r & 1, p.err)) {
             ok = false;
             break;
@@ -315,7 +325,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc::fence_before_sync();
   __syncwarp();
   tc::cluster_sync();
-  if (warp == 1) {
+  if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc_pair(tmem, kCols);
   }

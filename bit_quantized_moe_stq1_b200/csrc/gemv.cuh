@@ -153,8 +153,9 @@ __device__ __forceinline__ void load_x_block(uint4 (&xv)[8], const uint16_t* xro
 
 // Whole-warp STQ1_0 GEMV over blocks [b0, b1) of NT tiles, token column g of this
 // lane's quad taken from xrow (nullptr = padding column).  Weight loads for block
-// b+1 are in flight while block b is multiplied.
-template <int NT>
+// b+1 are in flight while block b is multiplied; with L2_AHEAD the tile-blocks of block
+// b+2 are also prefetched into L2 (six lanes, one 128-byte line each).
+template <int NT, bool L2_AHEAD = false>
 __device__ __forceinline__ void stq_warp_gemv(const uint8_t* const (&tb)[NT], int b0, int b1, const uint16_t* xrow,
                                               uint32_t lut, float (&acc)[NT][4]) {
   const int lane = threadIdx.x & 31, t = lane & 3;
@@ -162,6 +163,11 @@ __device__ __forceinline__ void stq_warp_gemv(const uint8_t* const (&tb)[NT], in
   StqBlockRegs<NT> cur, nxt;
   stq_load<NT>(cur, tb, b0, lane);
   for (int b = b0; b < b1; ++b) {
+    if (L2_AHEAD && b + 2 < b1 && lane < 6) {
+#pragma unroll
+      for (int i = 0; i < NT; ++i)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(tb[i] + size_t(b + 2) * kTileBlockBytes + 128 * lane));
+    }
     if (b + 1 < b1) stq_load<NT>(nxt, tb, b + 1, lane);
     uint4 xv[8];
     load_x_block(xv, xrow, b, t);

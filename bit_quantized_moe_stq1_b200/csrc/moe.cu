@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
       const int j = c0 + g;
       const uint16_t* xrow = j < cnt ? a.h + size_t(pos0 + j) * a.I : nullptr;
       float acc[4][4] = {};
-      stq_warp_gemv<4>(tb, 0, nb, xrow, lut, acc);
+      stq_warp_gemv<4, true>(tb, 0, nb, xrow, lut, acc);   // the L2 prefetch measured faster here
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
