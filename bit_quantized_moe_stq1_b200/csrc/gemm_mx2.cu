@@ -13,14 +13,14 @@
 // rows) x up to 240 tokens of one expert over all of K.  Per item both CTAs:
 //   warps 5-8 (producers, 128-k stages in turn): TMA of the CTA's 128 weight rows and of
 //      its half of the N token rows (rows n0 + rank * N/2 ..), whose completion bytes count
-//      on the rank-0 CTA's barrier; in rank 0 also the UE8M0 scales of both CTAs, re-laid
-//      into the scale-factor atoms (each CTA's own 128 weight rows, and the activations of
-//      all N tokens), the peer's written into its shared memory;
+//      on the rank-0 CTA's barrier; the UE8M0 scales re-laid into the scale-factor atoms
+//      (the CTA's own 128 weight rows, and the activations of all N tokens), which rank 1's
+//      producer releases to rank 0 with an arrival on rank 0's barrier;
 //   warp 0: TMEM (both CTAs, cta_group::2); in the rank-0 CTA one thread issues the scale
 //      copies and four M = 256 MMAs per stage, and commits to both CTAs' barriers;
 //   warps 1-4: the CTA's epilogue from its own TMEM (its 128 rows x N tokens).
-// Barriers: full[s] (rank 0; rank 0's producer and both CTAs' loads), empty[s] (both; one
-// commit), tfull[b] (both; one commit), tempty[b] (rank 0; the eight epilogue warps).
+// Barriers: full[s] (rank 0; both CTAs' producers and loads), empty[s] (both; one commit),
+// tfull[b] (both; one commit), tempty[b] (rank 0; the eight epilogue warps).
 // Every wait is bounded; after a timeout each role records STQ_ERR_TIMEOUT, keeps going to
 // the end, and both CTAs meet at a final cluster barrier before TMEM is freed, so no CTA
 // exits while the pair's copies or MMAs can still touch its memory.  No load multicasts.
@@ -137,7 +137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 1);                 // rank 0's producer, with both CTAs' bytes
+      tc::mbar_init(&full[s], 2);                 // both CTAs' producers (rank 0's with the bytes)
       tc::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -172,36 +172,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int q = 0; q < kStages; ++q) last_round[q] = -1;
     int cg = pid, cit = -1, cncols = 0;   // look-ahead cursor
     Item CI{};
-    // rank 0 lays out the scale factors of both CTAs (its own weight rows, the peer's rows,
-    // and the activations of all N tokens, which both need), so that everything the MMAs
-    // read is published by rank 0's producers to rank 0's barriers
-    auto sf_load = [&](uint32_t (&va0)[4], uint32_t (&va1)[4], uint32_t (&vb0)[4], uint32_t (&vb1)[4]) {
+    // each CTA lays out its own scale factors: its 128 weight rows, and the activations of
+    // all N tokens (both CTAs need those)
+    auto sf_load = [&](uint32_t (&va)[4], uint32_t (&vb0)[4], uint32_t (&vb1)[4]) {
       const int it = cg / nk, kt = cg % nk;
       if (it != cit) {
         cit = it;
-        CI = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, 0);
+        CI = cta_item<NT>(p.tiles, cid + it * NC, MT2, kRowsPerCta, rank);
         cncols = CI.valid ? gemm::item_cols(CI, NT) : 0;
       }
       const int nkj = CI.valid ? nk : 0;   // past the last item: zeros, no loads
-      if (PAIR) {
-        load_sf_gu(va0, p.sa, p.sa2, CI.arow, k32, kt, nkj, lane);
-        load_sf_gu(va1, p.sa, p.sa2, CI.arow + kRowsPerCta, k32, kt, nkj, lane);
-      } else {
-        load_sf(va0, p.sa, CI.arow, 128, 0x7fffffff, k32, kt, nkj, lane);
-        load_sf(va1, p.sa, CI.arow + kRowsPerCta, 128, 0x7fffffff, k32, kt, nkj, lane);
-      }
+      if (PAIR) load_sf_gu(va, p.sa, p.sa2, CI.arow, k32, kt, nkj, lane);
+      else load_sf(va, p.sa, CI.arow, 128, 0x7fffffff, k32, kt, nkj, lane);
       load_sf(vb0, p.sb, CI.brow, cncols, p.Ptot, k32, kt, nkj, lane);
       if (C::kSfbAtoms > 1) load_sf(vb1, p.sb, CI.brow + 128, cncols - 128, p.Ptot, k32, kt, nkj, lane);
       cg += kProducers;
     };
-    auto peer_sf = [&](uint8_t* dst, const uint32_t (&v)[4]) {
-      tc::st_shared_cluster_v4(tc::mapa_shared(tc::smem_u32(dst + lane * 16), 1), make_uint4(v[0], v[1], v[2], v[3]));
-    };
-    uint32_t ra0[kLook][4], ra1[kLook][4], rb0[kLook][4], rb1[kLook][4];
-    if (rank == 0) {
+    uint32_t ra[kLook][4], rb0[kLook][4], rb1[kLook][4];
 #pragma unroll
-      for (int d = 0; d < kLook; ++d) sf_load(ra0[d], ra1[d], rb0[d], rb1[d]);
-    }
+    for (int d = 0; d < kLook; ++d) sf_load(ra[d], rb0[d], rb1[d]);
     int g = pid, cur_it = -1, ncols = 0;
     Item I{};
     // the next item's descriptor is read one item ahead (its loads are in flight meanwhile)
@@ -228,15 +217,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* st = smem + s * kStage;
-        if (rank == 0) {
-          store_sf(st + kOffSfa, ra0[d], lane);
-          store_sf(st + kOffSfb, rb0[d], lane);
-          if (C::kSfbAtoms > 1) store_sf(st + kOffSfb + kSf, rb1[d], lane);
-          peer_sf(st + kOffSfa, ra1[d]);
-          peer_sf(st + kOffSfb, rb0[d]);
-          if (C::kSfbAtoms > 1) peer_sf(st + kOffSfb + kSf, rb1[d]);
-          tc::fence_proxy_async_cluster();
-        }
+        store_sf(st + kOffSfa, ra[d], lane);
+        store_sf(st + kOffSfb, rb0[d], lane);
+        if (C::kSfbAtoms > 1) store_sf(st + kOffSfb + kSf, rb1[d], lane);
+        tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           const uint32_t bar0 = tc::mapa_shared(tc::smem_u32(&full[s]), 0);
@@ -249,9 +233,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc::tma_load_2d_pair(st + kOffA, &tmA, kt * kKT, I.arow, bar0);
           }
           tc::tma_load_2d_pair(st + kOffB, &tmB, kt * kKT, bhalf, bar0);
+          // rank 1's scale-factor stores are released to rank 0's MMA thread by this arrival
+          if (rank != 0) tc::mbar_arrive_remote(bar0);
         }
         last_round[s] = r;
-        if (rank == 0) sf_load(ra0[d], ra1[d], rb0[d], rb1[d]);   // the step kLook ahead
+        sf_load(ra[d], rb0[d], rb1[d]);   // the step kLook ahead
         g += kProducers;
       }
     }
@@ -278,7 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int kt = 0; kt < nk && ok; ++kt, ++g) {
           const int j = g / kProducers, np = kStages / kProducers;
           const int s = kProducers * (j % np) + g % kProducers, r = j / np;
-          if (!tc::mbar_wait(&full[s], r & 1, p.err)) {
+          if (!tc::mbar_wait_cluster(&full[s], r & 1, p.err)) {   // rank 1's arrival releases at cluster scope
             ok = false;
             break;
           }
