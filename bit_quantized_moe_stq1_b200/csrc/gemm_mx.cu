@@ -404,9 +404,22 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, cudaStream_t s) {
   constexpr int64_t kPairFromTokensPerExpert = 0;
   if (kPairFromTokensPerExpert > 0 && int64_t(P) / slots_ >= kPairFromTokensPerExpert)
     return moe_mx_experts_pair(a, slots_, s);
+  // The gate/up pair with the tokens on M (gemm_mx_tm.cu) from this many routed tokens per
+  // expert on average.  The down projection stays on this file's 240-token N tile unless
+  // kDownTokensOnM: its token-major launch (N = 192, two accumulators) measured 0.99 ms
+  // against 0.82 ms on the 4096-token prefill layer.
+  constexpr int64_t kTokensOnMFrom = 32;
+  constexpr bool kDownTokensOnM = false;
+  const bool down_tokens_on_m = kDownTokensOnM && moe_mx_down_tm_fits(a);
+  const bool tokens_on_m = int64_t(P) / slots_ >= kTokensOnMFrom;
   const int nt_dn = pick_nt(int64_t(P) / slots_);
   const int nt = nt_dn > 128 ? 128 : nt_dn;
-  if ((st = stq_tile_plan_launch(a.counts, a.E, nt, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
+  if (tokens_on_m) {
+    if ((st = moe_mx_gate_up_tm(a, slots_, s)) != STQ_OK) return st;
+    if (down_tokens_on_m) return moe_mx_down_tm(a, slots_, s);
+  } else if ((st = stq_tile_plan_launch(a.counts, a.E, nt, a.ntiles, a.n_ntiles, s)) != STQ_OK) {
+    return st;
+  }
   const int max_tiles = P / nt + slots_;
   // 3. gate/up pair with SwiGLU and MXFP8 h
   CUtensorMap mg, mu, mx, md, mh;
@@ -429,13 +442,14 @@ stq_status moe_mx_experts(const MoeArgs& a, int slots, cudaStream_t s) {
   gp.out.hq = a.hq;
   gp.out.hs = a.hs;
   gp.err = a.err;
-  {
+  if (!tokens_on_m) {
     StqTimed tm(STQ_K_GATE_UP_MX, s);
     st = launch_nt<true>(nt, mg, mu, mx, gp, s);
   }
   if (st != STQ_OK) return st;
   // 4. down (the N-tile plan is redone for its tile width once the gate/up launch is done with it)
-  if (nt_dn != nt && (st = stq_tile_plan_launch(a.counts, a.E, nt_dn, a.ntiles, a.n_ntiles, s)) != STQ_OK) return st;
+  if ((tokens_on_m || nt_dn != nt) && (st = stq_tile_plan_launch(a.counts, a.E, nt_dn, a.ntiles, a.n_ntiles, s)) != STQ_OK)
+    return st;
   GemmProblem dp = gp;
   dp.tiles.R = a.H;
   dp.tiles.max_items = (P / nt_dn + slots_) * (a.H / 128);

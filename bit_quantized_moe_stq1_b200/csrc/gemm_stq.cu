@@ -8,21 +8,25 @@
 // MXFP8 activations by tcgen05.mma kind::mxf8f6f4 with a unit weight scale (UE8M0 127);
 // the activations keep their UE8M0 scale per 32 k.  d, FP16 with 11 significant bits,
 // fits neither operand format, so each block's product lands in its own TMEM partial
-// buffer and is promoted in FP32: acc += d[row] * partial.
+// buffer and is promoted in FP32: acc += d[row] * partial, with acc in registers.
 //
 // Tile: 128 weight rows (M; for gate/up the 64 gate rows of 64 features and the same
 // up rows) x 112 tokens of one expert (N), over all of K, one 256-k block per stage.
-// TMEM (512 columns): partial buffers at 0 and 128, accumulators at 256 and 384 (112
-// columns each), the scale factors at 112..123.
+// TMEM (512 columns): partial buffers at 0 and 128, finished accumulators at 256 and 384
+// (112 columns each), the scale factors at 112..123.
 //
-// Warp roles (448 threads, one CTA per SM, persistent over work items):
+// Warp roles (576 threads, one CTA per SM, persistent over work items):
 //   warp 0       TMA of the activation tile (two 128-k boxes, 128-byte swizzle) and its
 //                scale factors (loaded four stages ahead into a register ring), re-laid
 //                into the scale-factor atoms the MMA reads;
 //   warp 1       TMEM allocation and, from one thread, tcgen05.cp of the scales and the
 //                eight K = 32 MMAs of a stage into the partial buffer of the block;
-//   warps 2-5    promotion: acc += d * partial, TMEM to TMEM through registers;
-//   warps 6-9    epilogue of a finished accumulator (FP32 outputs, or SwiGLU and the
+//   warps 2-9    promotion: two warps per TMEM lane quarter (weight row), each holding 56
+//                of the tile's token columns in registers; per block one TMEM load of the
+//                partial, which frees the buffer, and acc += d * partial; after the item's
+//                last block one TMEM store of the accumulator into a finished-accumulator
+//                buffer;
+//   warps 14-17  epilogue of a finished accumulator (FP32 outputs, or SwiGLU and the
 //                MXFP8 re-quantisation of h);
 //   warps 10-13  decode: each warp turns two 16-row STQ1_0 tile-blocks into E4M3 rows of
 //                the A tile (a shuffle of a 32-entry pattern table per 5-bit code gives
@@ -46,15 +50,19 @@ constexpr int kOffB = 2 * kSubA;
 constexpr int kOffSfb = kOffB + 2 * kSubB;
 constexpr int kStage = (kOffSfb + 2 * kSf + 1023) / 1024 * 1024;
 constexpr int kStages = 3;
+constexpr int kHalf = kNT / 2;           // token columns per promotion warp
 constexpr int kUBuf = 4 * 32 * 9 * 4;    // gate/up exchange of the epilogue
 constexpr int kSmem = kStages * kStage + kUBuf + kSf /* unit weight scales */ + 1024 /* barriers */ +
                       1024 /* alignment */;
 constexpr uint32_t kTxB = 2 * kSubB;     // bytes the TMA delivers per stage
-constexpr int kThreads = 448;
+constexpr int kThreads = 576;
 constexpr int kDecodeWarp0 = 10;
+constexpr int kEpiWarp0 = 14;
 constexpr int kDecodeWarps = 4;
 constexpr int kColP = 0;                 // partial buffers: kColP + 128 * i
-constexpr int kColAcc = 256;             // accumulators: kColAcc + 128 * i
+constexpr int kPBufs = 2;
+constexpr int kColAcc = 256;             // finished accumulators on their way out: kColAcc + 128 * i
+constexpr int kPromoWarps = 8;
 constexpr int kColSfa = 112;
 constexpr int kColSfb = 116;             // two atoms: 116, 120
 constexpr uint32_t kCols = 512;
@@ -186,7 +194,7 @@ namespace {
 
 // Persistent over work items b, b + gridDim.x, ...; all roles walk the same item list,
 // and a per-CTA block counter g (items x K blocks) drives every ring: stage g % 3, partial
-// buffer g % 2; accumulator buffer = item % 2.
+// buffer g % 2; finished-accumulator buffer item % 2.
 template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     stq_gemm_kernel(const __grid_constant__ CUtensorMap tmB, StqGemm p) {
@@ -196,9 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sfa_unit = smem + kStages * kStage + kUBuf;
   uint64_t* full = reinterpret_cast<uint64_t*>(sfa_unit + kSf);  // [kStages]: TMA bytes + 3 arrivals
   uint64_t* empty = full + kStages;                              // [kStages]: MMAs of the stage done
-  uint64_t* pfull = empty + kStages;                             // [2]: partial written
-  uint64_t* pempty = pfull + 2;                                  // [2]: partial promoted (4 warps)
-  uint64_t* afull = pempty + 2;                                  // [2]: accumulator complete (4 warps)
+  uint64_t* pfull = empty + kStages;                             // [kPBufs]: partial written
+  uint64_t* pempty = pfull + kPBufs;                             // [kPBufs]: partial read (8 warps)
+  uint64_t* afull = pempty + kPBufs;                             // [2]: accumulator staged (8 warps)
   uint64_t* aempty = afull + 2;                                  // [2]: accumulator drained (4 warps)
   uint64_t* mdone = aempty + 2;                                  // every MMA of this CTA completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
@@ -217,10 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&full[s], 1 + kDecodeWarps);
       tc::mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kPBufs; ++b) {
       tc::mbar_init(&pfull[b], 1);
-      tc::mbar_init(&pempty[b], 4);
-      tc::mbar_init(&afull[b], 4);
+      tc::mbar_init(&pempty[b], kPromoWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&afull[b], kPromoWarps);
       tc::mbar_init(&aempty[b], 4);
     }
     tc::mbar_init(mdone, 1);
@@ -305,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!I.valid) break;
         const uint32_t idesc_n = uint32_t(gemm::item_cols(I, kNT));
         for (int kb = 0; kb < nb; ++kb, ++g) {
-          const int s = g % kStages, r = g / kStages, pb = g & 1, pr = g >> 1;
+          const int s = g % kStages, r = g / kStages, pb = g % kPBufs, pr = g / kPBufs;
           if (pr > 0 && !tc::mbar_wait(&pempty[pb], (pr - 1) & 1, p.err)) {
             ok = false;
             break;
@@ -336,24 +346,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_wait(mdone, 0, p.err);
     }
     __syncwarp();
-  } else if (warp <= 5) {
+  } else if (warp <= 9) {
     // ---------------------------------------------------------------- promotion
-    const int q = warp & 3;
+    // Warp w: TMEM lane quarter q = w % 4 (A-tile rows 32q..32q+31), token columns
+    // 56c..56c+55 of the tile (c = 0 for warps 2-5, 1 for 6-9), accumulated in registers.
+    const int q = warp & 3, c = (warp - 2) >> 2;
     const int m = 32 * q + lane;  // A-tile row = TMEM lane
-    const uint32_t lane_base = tmem + (uint32_t(32 * q) << 16);
+    const uint32_t lane_base = tmem + (uint32_t(32 * q) << 16) + uint32_t(kHalf * c);
     int g = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const Item I = gemm::get_item(p.tiles, blockIdx.x + it * G, MT, kRows, kNT);
       if (!I.valid) break;
-      const int abuf = it & 1, ar = it >> 1;
-      if (ar > 0 && !tc::mbar_wait(&aempty[abuf], (ar - 1) & 1, p.err)) break;
-      const uint32_t tacc = lane_base + uint32_t(kColAcc + 128 * abuf);
-      const int ncols = gemm::item_cols(I, kNT);  // columns the MMAs wrote
+      float acc[kHalf];
+#pragma unroll
+      for (int j = 0; j < kHalf; ++j) acc[j] = 0.f;
       const uint16_t* dp = d_ptr<PAIR>(p, I, m, 0);
       uint16_t dnext = __ldg(dp);
       for (int kb = 0; kb < nb; ++kb, ++g) {
-        const int pb = g & 1, pr = g >> 1;
+        const int pb = g % kPBufs, pr = g / kPBufs;
         const float d = __half2float(__ushort_as_half(dnext));
         if (kb + 1 < nb) dnext = __ldg(dp + (kb + 1) * (stq::kTileBlockBytes / 2));
         if (!tc::mbar_wait(&pfull[pb], pr & 1, p.err)) {
@@ -362,50 +373,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::fence_after_sync();
         const uint32_t tp = lane_base + uint32_t(kColP + 128 * pb);
-        // 32 columns per TMEM round trip (a 16-column tail when ncols is an odd multiple of 16)
-#pragma unroll 1
-        for (int c0 = 0; c0 < ncols; c0 += 32) {
-          if (c0 + 32 <= ncols) {
-            uint32_t v[32], a[32];
-            tc::tmem_ld_x32(tp + c0, v);
-            if (kb > 0) {
-              tc::tmem_ld_x32(tacc + c0, a);
-              tc::tmem_ld_wait();
+        // 16 columns per TMEM round trip: 18 warps leave 96 registers per thread (five warps
+        // share a sub-partition's 16K registers), and the accumulator takes 56 of them
 #pragma unroll
-              for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(fmaf(d, __uint_as_float(v[j]), __uint_as_float(a[j])));
-            } else {
-              tc::tmem_ld_wait();
+        for (int c0 = 0; c0 < 48; c0 += 16) {
+          uint32_t v[16];
+          tc::tmem_ld_x16(tp + c0, v);
+          tc::tmem_ld_wait();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(d * __uint_as_float(v[j]));
-            }
-            tc::tmem_st_x32(tacc + c0, a);
-          } else {
-            uint32_t v[16], a[16];
-            tc::tmem_ld_x16(tp + c0, v);
-            if (kb > 0) {
-              tc::tmem_ld_x16(tacc + c0, a);
-              tc::tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(fmaf(d, __uint_as_float(v[j]), __uint_as_float(a[j])));
-            } else {
-              tc::tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 16; ++j) a[j] = __float_as_uint(d * __uint_as_float(v[j]));
-            }
-            tc::tmem_st_x16(tacc + c0, a);
-          }
+          for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(d, __uint_as_float(v[j]), acc[c0 + j]);
         }
-        // the partial is read and the accumulator written: release the partial buffer
-        tc::tmem_st_wait();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&pempty[pb]);
+        {
+          uint32_t x[8];
+          tc::tmem_ld_x8(tp + 48, x);
+          tc::tmem_ld_wait();
+          // the partial is in registers: hand the buffer back to the MMA warp
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&pempty[pb]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[48 + j] = fmaf(d, __uint_as_float(x[j]), acc[48 + j]);
+        }
       }
       if (!ok) break;
+      // hand the finished accumulator to the epilogue warps through TMEM buffer it % 2
+      const int abuf = it & 1, ar = it >> 1;
+      if (ar > 0 && !tc::mbar_wait(&aempty[abuf], (ar - 1) & 1, p.err)) break;
+      tc::fence_after_sync();
+      const uint32_t stg = lane_base + uint32_t(kColAcc + 128 * abuf);
+#pragma unroll
+      for (int c0 = 0; c0 < 48; c0 += 16) {
+        uint32_t a16[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) a16[j] = __float_as_uint(acc[c0 + j]);
+        tc::tmem_st_x16(stg + c0, a16);
+      }
+      {
+        uint32_t a8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a8[j] = __float_as_uint(acc[48 + j]);
+        tc::tmem_st_x8(stg + 48, a8);
+      }
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&afull[abuf]);
     }
-  } else if (warp <= 9) {
+  } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;
     for (int it = 0;; ++it) {

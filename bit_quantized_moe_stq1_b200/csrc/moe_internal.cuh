@@ -76,6 +76,12 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L);
 stq_status moe_mx_experts(const MoeArgs& a, int slots, cudaStream_t s);
 // Their prefill regime on CTA pairs (gemm_mx2.cu), activations already quantised.
 stq_status moe_mx_experts_pair(const MoeArgs& a, int slots, cudaStream_t s);
+// Their prefill regime with the tokens on M (gemm_mx_tm.cu), activations already quantised:
+// the gate/up launch (with its 128-token tile plan) and the down launch on the same plan.
+stq_status moe_mx_gate_up_tm(const MoeArgs& a, int slots, cudaStream_t s);
+stq_status moe_mx_down_tm(const MoeArgs& a, int slots, cudaStream_t s);
+// Whether the down launch's 192-row weight tiles divide H.
+bool moe_mx_down_tm_fits(const MoeArgs& a);
 
 // BF16 -> MXFP8 quantisation launch (pack.cu).
 stq_status stq_mxfp8_quantize_launch(const uint16_t* x, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales,
