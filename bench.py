@@ -52,14 +52,14 @@ MMA_MICROBENCH_TFLOPS = 2 * 8190 * 148 * 1.965e9 / 1e12
 # capture of the same kernel build on a smaller case (named profile under profiles/); a
 # launch's traffic grows with its touched experts, so the full launch's traffic is this
 # figure times its touched experts.  An entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (2.109465e9 + 6.812928e6) / 157}  # decode_mx, 157 touched
+MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (860.81e6 + 3.76e6) / 64}  # decode_mx, 64 experts, 64 touched
 # DRAM bytes (read + write) of one full-size launch, from an ncu capture of the same workload
 # and kernel build; an entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_LAUNCH = {("stq_matvec", "gemv"): 2.09e6, ("w4a8_gemm", "gemm"): 7.55e6,
-                               ("stq_pack_ls", "pack_ls"): 50.41e6,
-                               ("decode_stq", "gate_up"): 285.818880e6 + 8.129536e6,
-                               ("prefill_stq", "gate_up_stq_tc"): 1.608519e9 + 64.757248e6,
-                               ("prefill_w4a8", "gate_up_mx"): 3.751041e9 + 71.260672e6}
+MEASURED_TRAFFIC_PER_LAUNCH = {("stq_matvec", "gemv"): 2.09e6, ("w4a8_gemm", "gemm"): 7.54e6,
+                               ("stq_pack_ls", "pack_ls"): 50.40e6 + 9.47e3,
+                               ("decode_stq", "gate_up"): 285.817344e6 + 6.748672e6,
+                               ("prefill_w4a8", "gate_up_mx"): 3.74e9 + 69.87e6,
+                               ("prefill_stq", "gate_up_stq_tc"): 1.61e9 + 63.35e6}
 
 
 def peaks():
@@ -753,6 +753,16 @@ def run_ours(args):
     import bit_quantized_moe_stq1_b200 as S
 
     wl = make_workload(args.workload, S, dev, args.experts)
+    if args.probe_step is not None:
+        # one eager step for a profiler capture of its launches, then that batch's accounting
+        wl.step(args.probe_step)
+        torch.cuda.synchronize(dev)
+        acct = wl.accounting(args.probe_step)
+        print(json.dumps({"workload": args.workload, "experts": args.experts, "probe_step": args.probe_step,
+                          "batch": args.probe_step % N_BATCHES,
+                          "touched_experts_per_layer": getattr(wl, "_acct", {}).get(args.probe_step % N_BATCHES),
+                          "hbm_bytes": acct.get("bytes")}))
+        return
     if isinstance(wl, StreamLayer):
         return run_stream(args, wl, S, dev, dist, n, rank, local)
     out = measure(wl, S, dev, dist, n, local, args.steps, args.warmup)
@@ -1022,6 +1032,8 @@ def main():
                     help="skip the other configurations timed after the default workload")
     ap.add_argument("--experts", type=int, default=256,
                     help="routed experts per layer (256 = the workloads; fewer only for small profiler captures)")
+    ap.add_argument("--probe-step", type=int, default=None,
+                    help="run step i once, eagerly, print that batch's touched experts and exit (for counter captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
