@@ -13,14 +13,15 @@
 // Tile: 128 weight rows (M; for gate/up the 64 gate rows of 64 features and the same
 // up rows) x 112 tokens of one expert (N), over all of K, one 256-k block per stage.
 // TMEM (512 columns): partial buffers at 0 and 128, finished accumulators at 256 and 384
-// (112 columns each), the scale factors at 112..123.
+// (112 columns each); the weights' unit scale atom at 112 and the three stages' activation
+// scale factors at 116, 240 and 248 (columns the 112-wide partials leave free).
 //
 // Warp roles (576 threads, one CTA per SM, persistent over work items):
 //   warp 0       TMA of the activation tile (two 128-k boxes, 128-byte swizzle) and its
 //                scale factors (loaded four stages ahead into a register ring), re-laid
-//                into the scale-factor atoms the MMA reads;
-//   warp 1       TMEM allocation and, from one thread, tcgen05.cp of the scales and the
-//                eight K = 32 MMAs of a stage into the partial buffer of the block;
+//                into the scale-factor atoms and copied into the stage's TMEM slot;
+//   warp 1       TMEM allocation and, from one thread, the eight K = 32 MMAs of a stage
+//                into the partial buffer of the block;
 //   warps 2-9    promotion: two warps per TMEM lane quarter (weight row), each holding 56
 //                of the tile's token columns in registers; per block one TMEM load of the
 //                partial, which frees the buffer, and acc += d * partial; after the item's
@@ -64,10 +65,12 @@ constexpr int kPBufs = 2;
 constexpr int kColAcc = 256;             // finished accumulators on their way out: kColAcc + 128 * i
 constexpr int kPromoWarps = 8;
 constexpr int kColSfa = 112;
-constexpr int kColSfb = 116;             // two atoms: 116, 120
+// Stage s's two activation scale-factor atoms (8 columns), in columns the partials leave free.
+__host__ __device__ constexpr int col_sfb(int s) { return s == 0 ? 116 : s == 1 ? 240 : 248; }
 constexpr uint32_t kCols = 512;
 static_assert(kSubB % 1024 == 0 && kStage % 1024 == 0, "128-byte swizzle atoms");
 static_assert(kSmem <= 227 * 1024, "shared memory");
+static_assert(kStages == 3 && kNT <= 112, "scale-factor slots in the partial buffers' free columns");
 
 struct StqGemm {
   gemm::Tiling tiles;          // tiles.R = weight rows per expert
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&full[s], 1 + kDecodeWarps);
+      tc::mbar_init(&full[s], 2 + kDecodeWarps);   // TMA bytes, the scale copies, the decoders
       tc::mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < kPBufs; ++b) {
@@ -287,6 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+          // the scale factors go to this stage's TMEM slot from here, so the MMA thread only
+          // issues MMAs (the MMAs of the slot's previous round are done: empty[s] above)
+          tc::fence_after_sync();
+          tc::cp_sf_32x128b_x4(tmem + uint32_t(col_sfb(s)), tc::smem_desc_sf(tc::smem_u32(st + kOffSfb)));
+          tc::cp_sf_32x128b_x4(tmem + uint32_t(col_sfb(s) + 4), tc::smem_desc_sf(tc::smem_u32(st + kOffSfb + kSf)));
+          tc::commit(&full[s]);
           tc::mbar_arrive_expect_tx(&full[s], kTxB);
           tc::tma_load_2d(st + kOffB, &tmB, kb * 256, I.brow, &full[s]);
           tc::tma_load_2d(st + kOffB + kSubB, &tmB, kb * 256 + 128, I.brow, &full[s]);
@@ -326,8 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::fence_after_sync();
           uint8_t* st = smem + s * kStage;
-          tc::cp_sf_32x128b_x4(tmem + kColSfb, tc::smem_desc_sf(tc::smem_u32(st + kOffSfb)));
-          tc::cp_sf_32x128b_x4(tmem + kColSfb + 4, tc::smem_desc_sf(tc::smem_u32(st + kOffSfb + kSf)));
+          const uint32_t sfb = tmem + uint32_t(col_sfb(s));
           const uint32_t d_col = tmem + uint32_t(kColP + 128 * pb);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t da = tc::smem_desc_sw128(tc::smem_u32(st + kOffA + h * kSubA)) + 2 * j;
             const uint64_t db = tc::smem_desc_sw128(tc::smem_u32(st + kOffB + h * kSubB)) + 2 * j;
             const uint32_t idesc = tc::idesc_mxf8f6f4_ab(int(idesc_n), tc::kFmtE4M3, tc::kFmtE4M3, 0u, uint32_t(j));
-            tc::mma_mxf8f6f4(d_col, da, db, idesc, tmem + kColSfa, (tmem + uint32_t(kColSfb + 4 * h)) | (uint32_t(j) << 30),
+            tc::mma_mxf8f6f4(d_col, da, db, idesc, tmem + kColSfa, (sfb + uint32_t(4 * h)) | (uint32_t(j) << 30),
                              kk > 0 ? 1u : 0u);
           }
           tc::commit(&empty[s]);
