@@ -52,7 +52,7 @@ MMA_MICROBENCH_TFLOPS = 2 * 8190 * 148 * 1.965e9 / 1e12
 # capture of the same kernel build on a smaller case (named profile under profiles/); a
 # launch's traffic grows with its touched experts, so the full launch's traffic is this
 # figure times its touched experts.  An entry is removed when its kernel changes.
-MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (860.81e6 + 3.76e6) / 64}  # decode_mx, 64 experts, 64 touched
+MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (860.83e6 + 3.90e6) / 64}  # decode_mx, 64 experts, 64 touched
 # DRAM bytes (read + write) of one full-size launch, from an ncu capture of the same workload
 # and kernel build; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC_PER_LAUNCH = {("stq_matvec", "gemv"): 2.09e6, ("w4a8_gemm", "gemm"): 7.54e6,
