@@ -80,7 +80,7 @@ SIGNATURES = {
 
 KERNEL_KINDS = ["router_logits", "router_topk", "permute", "quant_x", "gate_up", "down", "combine", "gemv", "gemm",
                 "gate_up_mx", "down_mx", "plan", "shared_gate_up", "shared_down", "rmsnorm",
-                "pack_ls", "gate_up_stq_tc", "down_stq_tc"]
+                "pack_ls", "gate_up_stq_tc", "down_stq_tc", "act_limbs"]
 
 
 class StqTiming(ctypes.Structure):

@@ -53,7 +53,7 @@ static stq_timing* g_timing = nullptr;
 static const char* const kKindNames[] = {"router_logits", "router_topk", "permute", "quant_x", "gate_up", "down",
                                          "combine", "gemv", "gemm", "gate_up_mx", "down_mx", "plan",
                                          "shared_gate_up", "shared_down", "rmsnorm", "pack_ls", "gate_up_stq_tc",
-                                         "down_stq_tc"};
+                                         "down_stq_tc", "act_limbs"};
 static_assert(sizeof(kKindNames) / sizeof(kKindNames[0]) == STQ_K_COUNT, "one name per kernel kind");
 
 extern "C" const char* stq_kernel_kind_name(int32_t kind) {

@@ -21,6 +21,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace stq {
 
@@ -173,6 +174,152 @@ __device__ __forceinline__ void stq_warp_gemv(const uint8_t* const (&tb)[NT], in
     load_x_block(xv, xrow, b, t);
     stq_block<NT>(cur, xv, lut, acc);
     cur = nxt;
+  }
+}
+
+// ----------------------------------------------------------------------------- integer variant
+//
+// The same decode into int8 weights (+1 = 0x01, -1 = 0xFF, 0 = 0x00): the shuffled table
+// entry is then a finished A-fragment register of mma.sync m16n8k32 s8 (four consecutive k
+// of one row), so a 5-bit code costs one shift and one shuffle and no byte permutes.  The
+// activations enter as three signed 8-bit limbs of a fixed-point value per 256-k block
+// (written by stq_act_limbs_kernel): v = q * 2^(Eb - 148), q = hi*2^16 + mid*2^8 + lo, with
+// Eb the largest bf16 exponent field of the block.  Every element within 2^14 of the
+// block's largest magnitude is exact; smaller ones are rounded to the nearest multiple of
+// 2^(Eb - 148), an absolute error of at most 2^-22 of the block's largest magnitude.  The
+// s32 sums of one block are exact (|sum| <= 256 * 128).
+//
+// The eight B columns are (token, limb) pairs: column c = 3j + l is limb l of the item's
+// token j (j = 0, 1; columns 6 and 7 are zero), so one mma serves two tokens.  K order:
+// in mma m of a block, thread t's a0/a1 (rows g, g+8) hold the codes of k = 64t + 8m + 0..3
+// (stream codes 4m, 4m+1) and a2/a3 those of k = 64t + 8m + 4..7 (codes 4m+2, 4m+3); its
+// b0/b1 hold the activations of the same k: in the limb rows' block layout (k = 64t + 16q + i
+// at byte 16*(4q + t) + i) the 16-byte chunk 4*(m/2) + t, bytes 8*(m%2) .. 8*(m%2) + 7.
+
+// Table entry of code c for the integer decode.
+__device__ __forceinline__ uint32_t lut_entry_i8(uint32_t c) {
+  const uint32_t z = (c >> 3) & 3u, s = c & 7u;
+  uint32_t e = 0, n = 0;
+#pragma unroll
+  for (uint32_t l = 0; l < 4; ++l) {
+    if (l != z) {
+      e |= (((s >> n) & 1u) ? 0xFFu : 0x01u) << (8 * l);
+      ++n;
+    }
+  }
+  return e;
+}
+
+// D = A * B + D for one m16n8k32 s8 tile with s32 accumulators.
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int M, int NT>
+struct StqStepsI8 {
+  __device__ __forceinline__ static void run(const StqBlockRegs<NT>& r, const uint4 (&xv)[4], uint32_t lut,
+                                             int (&part)[NT][4]) {
+    const uint4 q = xv[M >> 1];
+    const uint32_t b0 = (M & 1) ? q.z : q.x, b1 = (M & 1) ? q.w : q.y;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const uint32_t a0 = __shfl_sync(kFull, lut, code_at<4 * M>(r.w[i]));
+      const uint32_t a1 = __shfl_sync(kFull, lut, code_at<4 * M + 1>(r.w[i]));
+      const uint32_t a2 = __shfl_sync(kFull, lut, code_at<4 * M + 2>(r.w[i]));
+      const uint32_t a3 = __shfl_sync(kFull, lut, code_at<4 * M + 3>(r.w[i]));
+      mma_s8_16832(part[i], a0, a1, a2, a3, b0, b1);
+    }
+    StqStepsI8<M + 1, NT>::run(r, xv, lut, part);
+  }
+};
+template <int NT>
+struct StqStepsI8<8, NT> {
+  __device__ __forceinline__ static void run(const StqBlockRegs<NT>&, const uint4 (&)[4], uint32_t, int (&)[NT][4]) {}
+};
+
+// Floats per row of the limb scales of K = 256 nb: three rows of nb (one per limb), padded
+// to a multiple of four so that a row copies as whole 16-byte units.
+__host__ __device__ constexpr int stq_limb_scale_pitch(int nb) { return (3 * nb + 3) & ~3; }
+
+// The operand rows of one lane for the integer GEMV of an item with one or two tokens, in
+// shared memory.
+struct StqI8Cols {
+  const int8_t* xl;  // this lane's B column: one limb row of one token (any row for an empty column)
+  const float* s0;   // per-block scales (limb weight included) of output column 2t (nullptr = zero)
+  const float* s1;   // ... of output column 2t+1
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   tc::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+               : "memory");
+}
+
+// Whole-warp STQ1_0 GEMV over the nb blocks of NT tiles on the integer path: the weights in
+// registers, the loads of block b+1 in flight while block b is multiplied (with L2_AHEAD,
+// block b+2 also prefetched into L2); the activation limbs and scales read from the item's
+// shared-memory stage once its barrier `xbar` completes phase `xphase`, so that no global
+// load sits between two blocks.  acc[i][q] accumulates, in FP32, d * scale * (s32 block
+// sum) of output column 2t + (q & 1) (rows g, g+8 for q < 2, q >= 2); stq_i8_tokens folds
+// the columns into tokens.  Returns false if the wait gave up (STQ_ERR_TIMEOUT recorded).
+template <int NT, bool L2_AHEAD = false>
+__device__ __forceinline__ bool stq_warp_gemv_i8(const uint8_t* const (&tb)[NT], int nb, const StqI8Cols& c,
+                                                 uint64_t* xbar, uint32_t xphase, uint32_t lut, float (&acc)[NT][4],
+                                                 int32_t* err) {
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  if (nb <= 0) return true;
+  StqBlockRegs<NT> cur, nxt;
+  stq_load<NT>(cur, tb, 0, lane);
+  if (!__all_sync(kFull, tc::mbar_wait(xbar, xphase, err))) return false;
+  for (int b = 0; b < nb; ++b) {
+    if (L2_AHEAD && b + 2 < nb && lane < 6) {
+#pragma unroll
+      for (int i = 0; i < NT; ++i)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(tb[i] + size_t(b + 2) * kTileBlockBytes + 128 * lane));
+    }
+    if (b + 1 < nb) stq_load<NT>(nxt, tb, b + 1, lane);
+    uint4 xv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const uint4*>(c.xl + 256 * b + 16 * (4 * q + t));
+    const float sc0 = c.s0 != nullptr ? c.s0[b] : 0.f;
+    const float sc1 = c.s1 != nullptr ? c.s1[b] : 0.f;
+    int part[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) part[i][0] = part[i][1] = part[i][2] = part[i][3] = 0;
+    StqStepsI8<0, NT>::run(cur, xv, lut, part);
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const float dg = __half2float(__ushort_as_half((unsigned short)(cur.d[i] & 0xFFFFu)));
+      const float dg8 = __half2float(__ushort_as_half((unsigned short)(cur.d[i] >> 16)));
+      acc[i][0] = fmaf(dg * sc0, __int2float_rn(part[i][0]), acc[i][0]);
+      acc[i][1] = fmaf(dg * sc1, __int2float_rn(part[i][1]), acc[i][1]);
+      acc[i][2] = fmaf(dg8 * sc0, __int2float_rn(part[i][2]), acc[i][2]);
+      acc[i][3] = fmaf(dg8 * sc1, __int2float_rn(part[i][3]), acc[i][3]);
+    }
+    cur = nxt;
+  }
+  return true;
+}
+
+// Sum the limb columns of the two tokens: y[j][r] = row g + 8r of token j, valid in lane
+// t = 0 (token 0) and t = 2 (token 1) of each quad.  Token 0 is (column 0 + column 1) +
+// column 2, token 1 is (column 4 + column 5) + column 3: a fixed order.  Whole warp.
+__device__ __forceinline__ void stq_i8_tokens(const float (&acc)[4], float (&y)[2]) {
+  const int t = threadIdx.x & 3;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const float ce = acc[2 * r], co = acc[2 * r + 1];  // columns 2t, 2t+1
+    const float v0 = t == 0 ? ce + co : (t == 1 ? ce : 0.f);
+    const float v1 = t == 2 ? ce + co : (t == 1 ? co : 0.f);
+    const float o0 = __shfl_xor_sync(kFull, v0, 1);  // t=0 <-> t=1
+    const float o1 = __shfl_xor_sync(kFull, v1, 3);  // t=1 <-> t=2
+    y[r] = t == 0 ? v0 + o0 : v1 + o1;
   }
 }
 

@@ -502,12 +502,153 @@ __device__ __forceinline__ int next_item(int32_t* counter, int* slot) {
   return item;
 }
 
+// Activation rows src [rows, K] (bf16, K a multiple of 256) -> the integer decode GEMV's
+// operand: three signed 8-bit limbs per element, limbs[row][l][K] (l = 0: hi, 1: mid,
+// 2: lo), and per 256-k block b the scale of each limb, scales[row * pitch + l * nb + b] =
+// 2^(Eb - 148 + 8*(2 - l)) (pitch = stq_limb_scale_pitch(nb)), Eb = the largest exponent
+// field of the block's elements (1 for subnormals and zeros).  Inside each 256-byte block
+// the limb of k = 64t + 16q + i sits at byte 16*(4q + t) + i, so that the four lanes of a
+// GEMV quad read consecutive 16-byte chunks (conflict-free shared-memory loads).  An element
+// with significand m (implicit bit included) and exponent field e' = max(e, 1) is
+// q = m * 2^(e' - Eb + 14), rounded to nearest, ties to even, when e' < Eb - 14; |q| < 2^22,
+// and q = hi*2^16 + mid*2^8 + lo with every limb in [-128, 127].  A block holding an Inf or
+// NaN gets a NaN scale.  One warp per block; lane l takes elements 8l..8l+7.
+__global__ void __launch_bounds__(256) stq_act_limbs_kernel(const uint16_t* __restrict__ src, int64_t rows, int K,
+                                                           int8_t* __restrict__ limbs, float* __restrict__ scales) {
+  stq_pdl_begin();
+  const int nb = K / 256, lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (wid >= rows * nb) return;  // whole warps
+  const int64_t row = wid / nb;
+  const int b = int(wid - row * nb);
+  const uint4 v = *reinterpret_cast<const uint4*>(src + row * K + 256 * b + 8 * lane);
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  uint32_t emax = 1;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t e = (u[i >> 1] >> (16 * (i & 1) + 7)) & 0xFFu;
+    emax = e > emax ? e : emax;
+  }
+  const uint32_t eb = __reduce_max_sync(kFull, emax);
+  const int pitch = stq_limb_scale_pitch(nb);
+  uint32_t lb[3][2] = {};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t x = (u[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+    const uint32_t e = (x >> 7) & 0xFFu, ep = e > 1u ? e : 1u;
+    const uint32_t m = (x & 0x7Fu) | (e != 0u ? 0x80u : 0u);
+    uint32_t q;
+    if (ep + 14u >= eb) {
+      q = m << (ep + 14u - eb);
+    } else {
+      const uint32_t r = eb - ep - 14u < 9u ? eb - ep - 14u : 9u;
+      q = (m + (1u << (r - 1u)) - 1u + ((m >> r) & 1u)) >> r;
+    }
+    const int32_t vq = (x & 0x8000u) ? -int32_t(q) : int32_t(q);
+    const int32_t lo = int32_t(int8_t(vq & 0xFF));
+    const int32_t v1 = (vq - lo) >> 8;
+    const int32_t mid = int32_t(int8_t(v1 & 0xFF));
+    const int32_t hi = (v1 - mid) >> 8;
+    const int sh = 8 * (i & 3);
+    lb[0][i >> 2] |= (uint32_t(hi) & 0xFFu) << sh;
+    lb[1][i >> 2] |= (uint32_t(mid) & 0xFFu) << sh;
+    lb[2][i >> 2] |= (uint32_t(lo) & 0xFFu) << sh;
+  }
+  // this lane's elements k = 8*lane .. 8*lane + 7: t = lane / 8, q = (lane % 8) / 2, i from 8 * (lane % 2)
+  const int off = 16 * (4 * ((lane & 7) >> 1) + (lane >> 3)) + 8 * (lane & 1);
+#pragma unroll
+  for (int l = 0; l < 3; ++l)
+    *reinterpret_cast<uint2*>(limbs + (row * 3 + l) * K + 256 * b + off) = make_uint2(lb[l][0], lb[l][1]);
+  if (lane < 3)
+    scales[row * pitch + lane * nb + b] = eb == 255u ? __int_as_float(0x7FC00000) : ldexpf(1.f, int(eb) - 132 - 8 * lane);
+}
+
+// Items with at most this many tokens take the integer GEMV (two tokens per mma).
+constexpr int kI8MaxTokens = 2;
+
+// Resident CTAs per SM of the two persistent GEMV kernels: with the integer path three
+// (168 registers a thread: its weights, operands and sums without spills; measured faster
+// than four CTAs at 128 registers), without it four (128 registers, the BF16 path's best).
+template <bool I8>
+constexpr int gemv_ctas_per_sm() { return I8 ? 3 : 4; }
+
+// The shared expert's partial sums (float[4][2][4][4][32]): all the shared memory a launch
+// without the integer path takes.
+constexpr int kGemvRedBytes = int(sizeof(float)) * 4 * 2 * 4 * 4 * 32;
+
+// Shared memory of the two persistent GEMV kernels for K = H (gate/up) or I (down), when
+// the integer path is on (otherwise a launch takes kGemvRedBytes): the item's activation
+// stage (limb rows of its <= 2 tokens, pitch K + 64 so that the two token-limb rows a
+// quarter-warp reads fall in different banks, then their scale rows) and the stage's
+// barrier.  The shared expert's partial sums alias the stage (a CTA takes all its
+// shared-expert items before its first routed one).  Kept below 48 KB (no opt-in): in the
+// stacked decode step, launches that opted in to more measured about 30 us each slower to
+// overlap with the kernel before them.
+struct GemvSmem {
+  int xst, sst, xbar, total, pitch_x, pitch_s;
+};
+__host__ __device__ inline GemvSmem gemv_smem_layout(int K) {
+  GemvSmem L;
+  L.pitch_x = K + 64;
+  L.pitch_s = stq_limb_scale_pitch(K / 256);
+  L.xst = 0;
+  L.sst = L.xst + 2 * 3 * L.pitch_x;
+  const int end = L.sst + 2 * L.pitch_s * 4;
+  L.xbar = (end > kGemvRedBytes ? end : kGemvRedBytes);
+  L.total = L.xbar + 8;
+  return L;
+}
+constexpr int kGemvSmemLimit = 47 * 1024;  // below the 48 KB default with the static shared memory
+
+// The integer-path operand rows of a lane in the activation stage (row c = limb c % 3 of
+// token c / 3; v0, v1: tokens 0 and 1 present).  Absent columns read row 0 with a zero scale.
+__device__ __forceinline__ StqI8Cols i8_cols(const uint8_t* smem, const GemvSmem& L, int nb, bool v0, bool v1) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  auto present = [&](int c) { return c < 6 && (c < 3 ? v0 : v1); };
+  const int8_t* xst = reinterpret_cast<const int8_t*>(smem + L.xst);
+  const float* sst = reinterpret_cast<const float*>(smem + L.sst);
+  auto scale_row = [&](int c) { return present(c) ? sst + (c / 3) * L.pitch_s + (c % 3) * nb : nullptr; };
+  StqI8Cols cols;
+  cols.xl = xst + (present(g) ? g : 0) * L.pitch_x;
+  cols.s0 = scale_row(2 * t);
+  cols.s1 = scale_row(2 * t + 1);
+  return cols;
+}
+
+// Thread 0: bulk copies of the limb rows (3 x K bytes) and scale row of each present token
+// (source rows r0, r1; -1 = absent) into the activation stage, completing on its barrier.
+__device__ __forceinline__ void i8_stage_fill(uint8_t* smem, const GemvSmem& L, const int8_t* limbs,
+                                              const float* scales, int K, int r0, int r1) {
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L.xbar);
+  const uint32_t per_token = uint32_t(3 * K + 4 * L.pitch_s);
+  tc::fence_proxy_async_smem();  // earlier generic accesses of the stage before the copies
+  tc::mbar_arrive_expect_tx(bar, (r0 >= 0 ? per_token : 0u) + (r1 >= 0 ? per_token : 0u));
+  const int rows[2] = {r0, r1};
+  for (int j = 0; j < 2; ++j) {
+    if (rows[j] < 0) continue;
+    for (int l = 0; l < 3; ++l)
+      bulk_load(smem + L.xst + (3 * j + l) * L.pitch_x, limbs + (size_t(rows[j]) * 3 + l) * K, uint32_t(K), bar);
+    bulk_load(smem + L.sst + j * L.pitch_s * 4, scales + size_t(rows[j]) * L.pitch_s, uint32_t(4 * L.pitch_s), bar);
+  }
+}
+
 // Routed STQ1_0 gate/up + SwiGLU, persistent.  Items: first the shared expert's
 // 16-feature tiles (BF16, K split over the four warps), then, per touched expert,
 // 128-feature tiles (warp = 32 features = 2 gate tiles + 2 up tiles over all of H).
-__global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
-  __shared__ float red[4][2][4][4][32];
+template <bool I8>
+__global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_gateup_stq_kernel(MoeArgs a) {
+  extern __shared__ __align__(128) uint8_t gemv_smem[];
   __shared__ int s_item;
+  auto red = reinterpret_cast<float (*)[2][4][4][32]>(gemv_smem);
+  // the stage and its barrier exist only on the integer path (the launch's shared memory)
+  const GemvSmem L = gemv_smem_layout(a.H);
+  if (I8 && threadIdx.x == 0 && a.xl != nullptr) {
+    tc::mbar_init(reinterpret_cast<uint64_t*>(gemv_smem + L.xbar), 1);
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  bool live = true;    // false after a wait of this warp gave up
+  uint32_t xphase = 0; // phase of the activation stage's barrier
   stq_pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int per_expert = a.I / 128;
@@ -515,7 +656,7 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
   const int nb = a.H / 256;
   const size_t mat = size_t(a.I) * nb * 42;
   const size_t tstride = size_t(nb) * kTileBlockBytes;
-  const uint32_t lut = lut_entry(lane);
+  const uint32_t lut = lut_entry(lane), lut8 = lut_entry_i8(lane);
   for (;;) {
     const int item = next_item(a.sched, &s_item);
     if (item >= n_items) break;
@@ -534,6 +675,32 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
     const uint8_t* ub = a.wu + size_t(e) * mat;
     const uint8_t* tb[4] = {gb + size_t(f0 / 16) * tstride, gb + size_t(f0 / 16 + 1) * tstride,
                             ub + size_t(f0 / 16) * tstride, ub + size_t(f0 / 16 + 1) * tstride};
+    if (I8 && cnt <= kI8MaxTokens && a.xl != nullptr) {
+      int tk[2] = {-1, -1};
+      for (int j = 0; j < cnt; ++j) {
+        const int tok = a.perm[pos0 + j] / a.k;
+        tk[j] = STQ_DCHECK(tok >= 0 && tok < a.T, a.err) ? tok : -1;
+      }
+      if (threadIdx.x == 0 && live) i8_stage_fill(gemv_smem, L, a.xl, a.xls, a.H, tk[0], tk[1]);
+      float acc[4][4] = {};
+      if (!live) continue;
+      live = stq_warp_gemv_i8<4>(tb, nb, i8_cols(gemv_smem, L, nb, tk[0] >= 0, tk[1] >= 0),
+                                 reinterpret_cast<uint64_t*>(gemv_smem + L.xbar), xphase, lut8, acc, a.err);
+      xphase ^= 1u;
+      if (!live) continue;
+      float y[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) stq_i8_tokens(acc[i], y[i]);
+      const int j = t == 0 ? 0 : (t == 2 ? 1 : kI8MaxTokens);
+      if (j < cnt) {
+#pragma unroll
+        for (int tp = 0; tp < 2; ++tp)
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+            a.h[size_t(pos0 + j) * a.I + f0 + 16 * tp + g + 8 * r] = float_to_bf16_bits(silu_f32(y[tp][r]) * y[tp + 2][r]);
+      }
+      continue;
+    }
     for (int c0 = 0; c0 < cnt; c0 += 8) {
       const int j = c0 + g;
       const int tok = j < cnt ? a.perm[pos0 + j] / a.k : -1;
@@ -555,9 +722,20 @@ __global__ void __launch_bounds__(128, 4) moe_gateup_stq_kernel(MoeArgs a) {
 
 // Routed STQ1_0 down, persistent.  Items: the shared expert's 16-row tiles, then per
 // touched expert 256-row tiles of H (warp = 4 tiles).
-__global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
-  __shared__ float red[4][2][4][4][32];
+template <bool I8>
+__global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_down_stq_kernel(MoeArgs a) {
+  extern __shared__ __align__(128) uint8_t gemv_smem[];
   __shared__ int s_item;
+  auto red = reinterpret_cast<float (*)[2][4][4][32]>(gemv_smem);
+  // the stage and its barrier exist only on the integer path (the launch's shared memory)
+  const GemvSmem L = gemv_smem_layout(a.I);
+  if (I8 && threadIdx.x == 0 && a.hl != nullptr) {
+    tc::mbar_init(reinterpret_cast<uint64_t*>(gemv_smem + L.xbar), 1);
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  bool live = true;    // false after a wait of this warp gave up
+  uint32_t xphase = 0; // phase of the activation stage's barrier
   stq_pdl_begin();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
   const int per_expert = a.H / 256;
@@ -565,7 +743,7 @@ __global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
   const int nb = a.I / 256;
   const size_t mat = size_t(a.H) * nb * 42;
   const size_t tstride = size_t(nb) * kTileBlockBytes;
-  const uint32_t lut = lut_entry(lane);
+  const uint32_t lut = lut_entry(lane), lut8 = lut_entry_i8(lane);
   for (;;) {
     const int item = next_item(a.sched, &s_item);
     if (item >= n_items) break;
@@ -583,6 +761,26 @@ __global__ void __launch_bounds__(128, 4) moe_down_stq_kernel(MoeArgs a) {
     const uint8_t* db = a.wd + size_t(e) * mat;
     const uint8_t* tb[4] = {db + size_t(r0 / 16) * tstride, db + size_t(r0 / 16 + 1) * tstride,
                             db + size_t(r0 / 16 + 2) * tstride, db + size_t(r0 / 16 + 3) * tstride};
+    if (I8 && cnt <= kI8MaxTokens && a.hl != nullptr) {
+      if (threadIdx.x == 0 && live) i8_stage_fill(gemv_smem, L, a.hl, a.hls, a.I, pos0, cnt > 1 ? pos0 + 1 : -1);
+      float acc[4][4] = {};
+      if (!live) continue;
+      live = stq_warp_gemv_i8<4, true>(tb, nb, i8_cols(gemv_smem, L, nb, true, cnt > 1),
+                                       reinterpret_cast<uint64_t*>(gemv_smem + L.xbar), xphase, lut8, acc, a.err);
+      xphase ^= 1u;
+      if (!live) continue;
+      float y[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) stq_i8_tokens(acc[i], y[i]);
+      const int j = t == 0 ? 0 : (t == 2 ? 1 : kI8MaxTokens);
+      if (j < cnt) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) a.Y[size_t(pos0 + j) * a.H + r0 + 16 * i + g + 8 * r] = y[i][r];
+      }
+      continue;
+    }
     for (int c0 = 0; c0 < cnt; c0 += 8) {
       const int j = c0 + g;
       const uint16_t* xrow = j < cnt ? a.h + size_t(pos0 + j) * a.I : nullptr;
@@ -679,6 +877,10 @@ MoeWsLayout moe_ws_layout(const moe_desc& d) {
   L.xs = take((P + T) * (H / 32));
   L.hq = take((P + T) * I);
   L.hs = take((P + T) * (I / 32));
+  L.xl = take(T * 3 * H);
+  L.xls = take(T * size_t(stq_limb_scale_pitch(int(H / 256))) * 4);
+  L.hl = take(P * 3 * I);
+  L.hls = take(P * size_t(stq_limb_scale_pitch(int(I / 256))) * 4);
   L.ntiles = take((P / 16 + E + 1) * 8);
   L.n_ntiles = take(4);
   L.sched = take(16);
@@ -703,6 +905,10 @@ MoeWs moe_ws_pointers(void* workspace, const MoeWsLayout& L) {
   w.xs = b + L.xs;
   w.hq = b + L.hq;
   w.hs = b + L.hs;
+  w.xl = reinterpret_cast<int8_t*>(b + L.xl);
+  w.xls = reinterpret_cast<float*>(b + L.xls);
+  w.hl = reinterpret_cast<int8_t*>(b + L.hl);
+  w.hls = reinterpret_cast<float*>(b + L.hls);
   w.ntiles = reinterpret_cast<int2*>(b + L.ntiles);
   w.n_ntiles = reinterpret_cast<int32_t*>(b + L.n_ntiles);
   w.sched = reinterpret_cast<int32_t*>(b + L.sched);
@@ -744,7 +950,8 @@ stq_status moe_shared_expert_bf16(const MoeArgs& a0, cudaStream_t s) {
   a.n_shared_cta = a.H / 16;
   a.sched = a0.sched + 3;
   StqTimed tm(STQ_K_SHARED_DOWN, s);
-  return stq_launch(moe_down_stq_kernel, dim3(unsigned(stq_persistent_grid(a.n_shared_cta, 4))), dim3(128), 0, s, a);
+  return stq_launch(moe_down_stq_kernel<false>, dim3(unsigned(stq_persistent_grid(a.n_shared_cta, gemv_ctas_per_sm<false>()))),
+                    dim3(128), kGemvRedBytes, s, a);
 }
 
 extern "C" size_t moe_workspace_offset(const moe_desc* d, int32_t region) {
@@ -854,6 +1061,56 @@ static stq_status side_stream(SideStream** out, ForkJoin** fj) {
   return STQ_OK;
 }
 
+// Largest average of routed tokens per expert for which the STQ1_0 decode regime makes
+// the activation limbs of the integer GEMV.
+constexpr int kI8LimbsAvgTokens = 2;
+
+stq_status moe_launch_act_limbs(const uint16_t* src, int64_t rows, int K, int8_t* limbs, float* scales,
+                                cudaStream_t s) {
+  const int64_t warps = rows * (K / 256);
+  if (warps == 0) return STQ_OK;
+  StqTimed tm(STQ_K_ACT_LIMBS, s);
+  return stq_launch(stq_act_limbs_kernel, dim3(unsigned(ceil_div<int64_t>(warps, 8))), dim3(256), 0, s, src, rows, K,
+                    limbs, scales);
+}
+
+// The routed STQ1_0 experts in the decode regime: the two persistent GEMV kernels (the BF16
+// shared expert's tiles as their first items), with the integer path (I8: the activation
+// limbs of x made before gate/up, those of h between gate/up and down) or without it.
+template <bool I8>
+stq_status launch_stq_decode(MoeArgs a, const moe_desc& d, const MoeWs& ws, const uint16_t* x, int P, int slots,
+                             bool shared_bf16, cudaStream_t s) {
+  stq_status st;
+  const int smem_gu = I8 ? gemv_smem_layout(d.H).total : kGemvRedBytes;
+  const int smem_dn = I8 ? gemv_smem_layout(d.I).total : kGemvRedBytes;
+  if (I8) {
+    if ((st = moe_launch_act_limbs(x, d.T, d.H, ws.xl, ws.xls, s)) != STQ_OK) return st;
+    a.xl = ws.xl;
+    a.xls = ws.xls;
+  }
+  a.routed = 1;
+  a.n_shared_cta = shared_bf16 ? d.I / 16 : 0;
+  a.sched = ws.sched;
+  {
+    StqTimed tm(STQ_K_GATE_UP, s);
+    st = stq_launch(moe_gateup_stq_kernel<I8>,
+                    dim3(unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d.I / 128), gemv_ctas_per_sm<I8>()))),
+                    dim3(128), smem_gu, s, a);
+  }
+  if (st != STQ_OK) return st;
+  if (I8) {
+    if ((st = moe_launch_act_limbs(ws.h, P, d.I, ws.hl, ws.hls, s)) != STQ_OK) return st;
+    a.hl = ws.hl;
+    a.hls = ws.hls;
+  }
+  a.n_shared_cta = shared_bf16 ? d.H / 16 : 0;
+  a.sched = ws.sched + 1;
+  StqTimed tm(STQ_K_DOWN, s);
+  return stq_launch(moe_down_stq_kernel<I8>,
+                    dim3(unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d.H / 256), gemv_ctas_per_sm<I8>()))),
+                    dim3(128), smem_dn, s, a);
+}
+
 // Average routed tokens per expert from which STQ_REGIME_AUTO runs the STQ1_0 experts
 // on the tensor-core GEMM instead of the decode GEMV.
 constexpr int kStqPrefillTokensPerExpert = 32;
@@ -940,23 +1197,12 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
   if (w->fmt == STQ_FMT_STQ1_0 && prefill) {
     if ((st = moe_stq_prefill_experts(a, slots, s)) != STQ_OK) return st;
   } else if (w->fmt == STQ_FMT_STQ1_0) {
-    // the BF16 shared expert's tiles are the first work items of the two GEMV kernels
-    a.routed = 1;
-    a.n_shared_cta = shared_bf16 ? d->I / 16 : 0;
-    a.sched = ws.sched;
-    {
-      StqTimed tm(STQ_K_GATE_UP, s);
-      st = stq_launch(moe_gateup_stq_kernel, dim3(unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->I / 128)))),
-                      dim3(128), 0, s, a);
-    }
-    if (st != STQ_OK) return st;
-    a.n_shared_cta = shared_bf16 ? d->H / 16 : 0;
-    a.sched = ws.sched + 1;
-    {
-      StqTimed tm(STQ_K_DOWN, s);
-      st = stq_launch(moe_down_stq_kernel, dim3(unsigned(stq_persistent_grid(a.n_shared_cta + slots * (d->H / 256), 4))),
-                      dim3(128), 0, s, a);
-    }
+    // The integer GEMV serves items of at most two tokens; its limbs are made when the
+    // average expert has at most four and the activation stages fit in kGemvSmemLimit.
+    const bool i8 = int64_t(P) <= kI8LimbsAvgTokens * int64_t(slots) &&
+                    gemv_smem_layout(d->H).total <= kGemvSmemLimit && gemv_smem_layout(d->I).total <= kGemvSmemLimit;
+    st = i8 ? launch_stq_decode<true>(a, *d, ws, x, P, slots, shared_bf16, s)
+            : launch_stq_decode<false>(a, *d, ws, x, P, slots, shared_bf16, s);
     if (st != STQ_OK) return st;
   } else {
     st = moe_mx_experts(a, slots, s);

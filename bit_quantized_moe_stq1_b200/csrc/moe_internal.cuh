@@ -4,7 +4,8 @@
 #include "common.cuh"
 
 struct MoeWsLayout {
-  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, ntiles, n_ntiles, sched, chist, total;
+  size_t err, counts, offsets, tlist, ntouched, perm, inv, h, Y, xq, xs, hq, hs, xl, xls, hl, hls, ntiles, n_ntiles,
+      sched, chist, total;
 };
 
 // Device pointers into the caller's workspace.
@@ -22,6 +23,10 @@ struct MoeWs {
   uint8_t* xs;   // [(P+T), H/32]
   uint8_t* hq;   // [(P+T), I] MXFP8 codes of h, same rows
   uint8_t* hs;   // [(P+T), I/32]
+  int8_t* xl;    // [T][3][H] activation limbs of x (integer decode GEMV)
+  float* xls;    // [T][stq_limb_scale_pitch(H/256)] their block scales, one row per limb
+  int8_t* hl;    // [P][3][I] limbs of the routed rows of h
+  float* hls;    // [P][stq_limb_scale_pitch(I/256)]
   int2* ntiles;  // [P/16 + E] (expert, first token) of each GEMM N tile
   int32_t* n_ntiles;
   int32_t* sched;  // [4] work counters of the persistent GEMV kernels: 0-2 zeroed by the permute
@@ -42,6 +47,10 @@ struct MoeArgs {
   uint16_t* h;
   float* Y;
   uint8_t *xq, *xs, *hq, *hs;
+  const int8_t* xl;  // limbs of x / of the routed h rows for the integer decode GEMV
+  const float* xls;  // (nullptr: every item takes the BF16 path)
+  const int8_t* hl;
+  const float* hls;
   int2* ntiles;
   int32_t* n_ntiles;
   int32_t* err;

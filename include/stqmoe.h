@@ -281,7 +281,12 @@ size_t moe_workspace_bytes(const moe_desc* d);
  * with FFN_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x)).  The intermediate h is
  * rounded to bf16 (STQ1_0 decode regime and the BF16 shared expert) or re-quantised
  * to MXFP8 (MXFP4 experts, the STQ1_0 prefill regime and the MXFP8 shared expert,
- * whose input x is quantised to MXFP8 first).  Slots are summed in order
+ * whose input x is quantised to MXFP8 first).  In the STQ1_0 decode regime an expert
+ * with at most two routed tokens (when the layer averages at most two per expert)
+ * multiplies its activations (x, then h) as a fixed-point value per 256-k block, 22 bits
+ * below the block's largest bf16 exponent: exact for every element within 2^14 of the
+ * block's largest magnitude, an error of at most 2^-22 of it otherwise; its sums are
+ * exact integers per block, scaled in FP32.  Slots are summed in order
  * s = 0..k-1, without atomics.  Duplicate ids in a token are separate slots; an
  * id outside [0, E) sets STQ_ERR_DEVICE in the workspace error word and its slot
  * contributes 0.  workspace: >= moe_workspace_bytes(d) bytes, 256-B aligned. */
@@ -380,7 +385,7 @@ stq_status stq_wait_selftest(int32_t* err, stq_stream_t stream);
 enum { STQ_K_ROUTER_LOGITS = 0, STQ_K_ROUTER_TOPK, STQ_K_PERMUTE, STQ_K_QUANT_X,
        STQ_K_GATE_UP, STQ_K_DOWN, STQ_K_COMBINE, STQ_K_GEMV, STQ_K_GEMM,
        STQ_K_GATE_UP_MX, STQ_K_DOWN_MX, STQ_K_PLAN, STQ_K_SHARED_GATE_UP, STQ_K_SHARED_DOWN,
-       STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_GATE_UP_STQ_TC, STQ_K_DOWN_STQ_TC, STQ_K_COUNT };
+       STQ_K_RMSNORM, STQ_K_PACK_LS, STQ_K_GATE_UP_STQ_TC, STQ_K_DOWN_STQ_TC, STQ_K_ACT_LIMBS, STQ_K_COUNT };
 
 /* Caller-owned host struct.  While installed, every kernel launched by
  * moe_router_topk, moe_router_topk_static, moe_expert_forward, stq1_gemv, w4a8_gemm,

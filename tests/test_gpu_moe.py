@@ -362,6 +362,42 @@ def test_moe_stq_wide_range_activations(S):
     _check_layer(r, T, H, I, E, k)
 
 
+@pytest.mark.parametrize("T,H,I,E,k", [(8, 512, 256, 16, 2), (6, 1024, 512, 8, 2)])
+def test_moe_stq_decode_integer_path_exactness(S, T, H, I, E, k):
+    """Experts with one or two routed tokens (a layer averaging at most two per expert)
+    run the integer GEMV: activations as a 22-bit fixed point per 256-k block, exact
+    integer sums per block.  With every block's elements within 2^14 of its largest
+    magnitude the down projection of the GPU's own h then matches the float64 product to a
+    few FP32 roundings, far inside the layer tolerance (1e-3 S); experts with more tokens
+    keep that tolerance.  An activation row spanning 2^-20 .. 2^0 inside each block checks
+    the rounded elements against their bound, 2^-22 of the block's largest magnitude per
+    element."""
+    r = _run_layer(S, T, H, I, E, k, True, ("exact", T, H, I, E, k))
+    counts, offsets, perm, _ = M.permute(r["ids"], E)
+    gw = r["gw"]
+    small = [e for e in np.flatnonzero(counts) if counts[e] <= 2]
+    assert small, "no expert with one or two tokens"
+    for e in small:
+        pos = np.arange(offsets[e], offsets[e + 1])
+        Wd = gw[2][e * H:(e + 1) * H].double().cpu().numpy()
+        h = r["h"][pos]
+        # every 256-block of h within 2^14 of its largest magnitude: the fixed point is exact
+        hb = np.abs(h).reshape(len(pos), -1, 256)
+        nz = np.where(hb > 0, hb, np.inf).min(axis=2)
+        if np.all(hb.max(axis=2) <= nz * 2.0 ** 14):
+            y, sy = M.matvec_with_scale(Wd, h)
+            err = np.abs(r["Y"][pos] - y)
+            assert np.all(err <= 1e-6 * sy + 1e-12), float(np.max(err / (1e-6 * sy + 1e-12)))
+    _check_layer(r, T, H, I, E, k)
+
+    # wide range inside each block: rounded elements stay within their bound
+    g = W.generator(DEV, 0, "exact-wide", "mag")
+    mag = torch.exp2(-torch.randint(0, 21, (T, H), generator=g, device=DEV).float())
+    x = (W.bf16_normal((T, H), 1.0, DEV, 0, "exact-wide", "x").float() * mag).to(torch.bfloat16)
+    r = _run_layer(S, T, H, I, E, k, True, ("exact", T, H, I, E, k), x=x)
+    _check_layer(r, T, H, I, E, k)
+
+
 def test_moe_bad_expert_id_reports_and_skips(S):
     T, H, I, E, k = 2, 256, 256, 4, 2
     gw, packs, sh, wr, x = _make_layer(S, T, H, I, E, k, False, "bad")
