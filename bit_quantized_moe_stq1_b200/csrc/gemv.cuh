@@ -268,41 +268,77 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // load sits between two blocks.  acc[i][q] accumulates, in FP32, d * scale * (s32 block
 // sum) of output column 2t + (q & 1) (rows g, g+8 for q < 2, q >= 2); stq_i8_tokens folds
 // the columns into tokens.  Returns false if the wait gave up (STQ_ERR_TIMEOUT recorded).
-template <int NT, bool L2_AHEAD = false>
+// One 256-k block of the integer path: activations and scales of block b from the stage,
+// weights from r.
+template <int NT>
+__device__ __forceinline__ void stq_block_i8(const StqBlockRegs<NT>& r, int b, const StqI8Cols& c, uint32_t lut,
+                                             float (&acc)[NT][4]) {
+  const int t = threadIdx.x & 3;
+  uint4 xv[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const uint4*>(c.xl + 256 * b + 16 * (4 * q + t));
+  const float sc0 = c.s0 != nullptr ? c.s0[b] : 0.f;
+  const float sc1 = c.s1 != nullptr ? c.s1[b] : 0.f;
+  int part[NT][4];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) part[i][0] = part[i][1] = part[i][2] = part[i][3] = 0;
+  StqStepsI8<0, NT>::run(r, xv, lut, part);
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const float dg = __half2float(__ushort_as_half((unsigned short)(r.d[i] & 0xFFFFu)));
+    const float dg8 = __half2float(__ushort_as_half((unsigned short)(r.d[i] >> 16)));
+    acc[i][0] = fmaf(dg * sc0, __int2float_rn(part[i][0]), acc[i][0]);
+    acc[i][1] = fmaf(dg * sc1, __int2float_rn(part[i][1]), acc[i][1]);
+    acc[i][2] = fmaf(dg8 * sc0, __int2float_rn(part[i][2]), acc[i][2]);
+    acc[i][3] = fmaf(dg8 * sc1, __int2float_rn(part[i][3]), acc[i][3]);
+  }
+}
+
+template <int NT, bool L2_AHEAD>
+__device__ __forceinline__ void stq_prefetch_l2(const uint8_t* const (&tb)[NT], int b, int nb) {
+  const int lane = threadIdx.x & 31;
+  if (L2_AHEAD && b < nb && lane < 6) {
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(tb[i] + size_t(b) * kTileBlockBytes + 128 * lane));
+  }
+}
+
+// Whole-warp STQ1_0 GEMV over the nb blocks of NT tiles on the integer path: the weights in
+// registers, the loads of block b+1 in flight while block b is multiplied (with L2_AHEAD
+// block b+2 also prefetched into L2; with PINGPONG two buffers used in turn instead of a
+// copy per block, measured faster for the down projection's short items and slower for
+// gate/up); the activation limbs and scales read from the item's shared-memory stage once
+// its barrier `xbar` completes phase `xphase`, so that no global load sits between two
+// blocks.  acc[i][q] accumulates, in FP32, d * scale * (s32 block sum) of output column
+// 2t + (q & 1) (rows g, g+8 for q < 2, q >= 2); stq_i8_tokens folds the columns into
+// tokens.  Returns false if the wait gave up (STQ_ERR_TIMEOUT recorded).
+template <int NT, bool L2_AHEAD = false, bool PINGPONG = false>
 __device__ __forceinline__ bool stq_warp_gemv_i8(const uint8_t* const (&tb)[NT], int nb, const StqI8Cols& c,
                                                  uint64_t* xbar, uint32_t xphase, uint32_t lut, float (&acc)[NT][4],
                                                  int32_t* err) {
-  const int lane = threadIdx.x & 31, t = lane & 3;
+  const int lane = threadIdx.x & 31;
   if (nb <= 0) return true;
-  StqBlockRegs<NT> cur, nxt;
-  stq_load<NT>(cur, tb, 0, lane);
+  StqBlockRegs<NT> r0, r1;
+  stq_load<NT>(r0, tb, 0, lane);
   if (!__all_sync(kFull, tc::mbar_wait(xbar, xphase, err))) return false;
-  for (int b = 0; b < nb; ++b) {
-    if (L2_AHEAD && b + 2 < nb && lane < 6) {
-#pragma unroll
-      for (int i = 0; i < NT; ++i)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(tb[i] + size_t(b + 2) * kTileBlockBytes + 128 * lane));
+  if (!PINGPONG) {
+    for (int b = 0; b < nb; ++b) {
+      stq_prefetch_l2<NT, L2_AHEAD>(tb, b + 2, nb);
+      if (b + 1 < nb) stq_load<NT>(r1, tb, b + 1, lane);
+      stq_block_i8<NT>(r0, b, c, lut, acc);
+      r0 = r1;
     }
-    if (b + 1 < nb) stq_load<NT>(nxt, tb, b + 1, lane);
-    uint4 xv[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const uint4*>(c.xl + 256 * b + 16 * (4 * q + t));
-    const float sc0 = c.s0 != nullptr ? c.s0[b] : 0.f;
-    const float sc1 = c.s1 != nullptr ? c.s1[b] : 0.f;
-    int part[NT][4];
-#pragma unroll
-    for (int i = 0; i < NT; ++i) part[i][0] = part[i][1] = part[i][2] = part[i][3] = 0;
-    StqStepsI8<0, NT>::run(cur, xv, lut, part);
-#pragma unroll
-    for (int i = 0; i < NT; ++i) {
-      const float dg = __half2float(__ushort_as_half((unsigned short)(cur.d[i] & 0xFFFFu)));
-      const float dg8 = __half2float(__ushort_as_half((unsigned short)(cur.d[i] >> 16)));
-      acc[i][0] = fmaf(dg * sc0, __int2float_rn(part[i][0]), acc[i][0]);
-      acc[i][1] = fmaf(dg * sc1, __int2float_rn(part[i][1]), acc[i][1]);
-      acc[i][2] = fmaf(dg8 * sc0, __int2float_rn(part[i][2]), acc[i][2]);
-      acc[i][3] = fmaf(dg8 * sc1, __int2float_rn(part[i][3]), acc[i][3]);
-    }
-    cur = nxt;
+    return true;
+  }
+  for (int b = 0; b < nb; b += 2) {
+    stq_prefetch_l2<NT, L2_AHEAD>(tb, b + 2, nb);
+    if (b + 1 < nb) stq_load<NT>(r1, tb, b + 1, lane);
+    stq_block_i8<NT>(r0, b, c, lut, acc);
+    if (b + 1 >= nb) break;
+    stq_prefetch_l2<NT, L2_AHEAD>(tb, b + 3, nb);
+    if (b + 2 < nb) stq_load<NT>(r0, tb, b + 2, lane);
+    stq_block_i8<NT>(r1, b + 1, c, lut, acc);
   }
   return true;
 }

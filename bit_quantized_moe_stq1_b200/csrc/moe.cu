@@ -580,8 +580,9 @@ constexpr int kGemvRedBytes = int(sizeof(float)) * 4 * 2 * 4 * 4 * 32;
 // the integer path is on (otherwise a launch takes kGemvRedBytes): the item's activation
 // stage (limb rows of its <= 2 tokens, pitch K + 64 so that the two token-limb rows a
 // quarter-warp reads fall in different banks, then their scale rows) and the stage's
-// barrier.  The shared expert's partial sums alias the stage (a CTA takes all its
-// shared-expert items before its first routed one).  Kept below 48 KB (no opt-in): in the
+// barrier.  The shared expert's partial sums alias the stage: every copy into the stage has
+// been waited on by the whole CTA before its item ends, and the copies of a routed item are
+// issued after the barrier that ends the previous item.  Kept below 48 KB (no opt-in): in the
 // stacked decode step, launches that opted in to more measured about 30 us each slower to
 // overlap with the kernel before them.
 struct GemvSmem {
@@ -632,9 +633,10 @@ __device__ __forceinline__ void i8_stage_fill(uint8_t* smem, const GemvSmem& L, 
   }
 }
 
-// Routed STQ1_0 gate/up + SwiGLU, persistent.  Items: first the shared expert's
-// 16-feature tiles (BF16, K split over the four warps), then, per touched expert,
-// 128-feature tiles (warp = 32 features = 2 gate tiles + 2 up tiles over all of H).
+// Routed STQ1_0 gate/up + SwiGLU, persistent.  Items: the shared expert's 16-feature tiles
+// (BF16, K split over the four warps) and, per touched expert, 128-feature tiles (warp = 32
+// features = 2 gate tiles + 2 up tiles over all of H); the shared ones first on the BF16
+// path, last on the integer path.
 template <bool I8>
 __global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_gateup_stq_kernel(MoeArgs a) {
   extern __shared__ __align__(128) uint8_t gemv_smem[];
@@ -660,11 +662,15 @@ __global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_gateup_stq_ke
   for (;;) {
     const int item = next_item(a.sched, &s_item);
     if (item >= n_items) break;
-    if (item < a.n_shared_cta) {
-      shared_gateup(a, item, red);
+    // the integer path takes the routed items first and the shared expert's smaller ones
+    // last, where they fill the tail of the launch; the BF16 path the other way round
+    const int n_shared = a.n_shared_cta, n_routed = n_items - n_shared;
+    const bool shared_item = I8 ? item >= n_routed : item < n_shared;
+    if (shared_item) {
+      shared_gateup(a, I8 ? item - n_routed : item, red);
       continue;
     }
-    const int bid = item - a.n_shared_cta;
+    const int bid = I8 ? item : item - n_shared;
     const int slot = bid / per_expert, ct = bid % per_expert;
     const int e = a.tlist[slot];
     if (!STQ_DCHECK(e >= 0 && e < a.E, a.err)) continue;
@@ -720,8 +726,9 @@ __global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_gateup_stq_ke
   }
 }
 
-// Routed STQ1_0 down, persistent.  Items: the shared expert's 16-row tiles, then per
-// touched expert 256-row tiles of H (warp = 4 tiles).
+// Routed STQ1_0 down, persistent.  Items: the shared expert's 16-row tiles and, per touched
+// expert, 256-row tiles of H (warp = 4 tiles); the shared ones first on the BF16 path, last
+// on the integer path.
 template <bool I8>
 __global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_down_stq_kernel(MoeArgs a) {
   extern __shared__ __align__(128) uint8_t gemv_smem[];
@@ -747,11 +754,15 @@ __global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_down_stq_kern
   for (;;) {
     const int item = next_item(a.sched, &s_item);
     if (item >= n_items) break;
-    if (item < a.n_shared_cta) {
-      shared_down(a, item, red);
+    // the integer path takes the routed items first and the shared expert's smaller ones
+    // last, where they fill the tail of the launch; the BF16 path the other way round
+    const int n_shared = a.n_shared_cta, n_routed = n_items - n_shared;
+    const bool shared_item = I8 ? item >= n_routed : item < n_shared;
+    if (shared_item) {
+      shared_down(a, I8 ? item - n_routed : item, red);
       continue;
     }
-    const int bid = item - a.n_shared_cta;
+    const int bid = I8 ? item : item - n_shared;
     const int slot = bid / per_expert, ct = bid % per_expert;
     const int e = a.tlist[slot];
     if (!STQ_DCHECK(e >= 0 && e < a.E, a.err)) continue;
@@ -765,7 +776,7 @@ __global__ void __launch_bounds__(128, gemv_ctas_per_sm<I8>()) moe_down_stq_kern
       if (threadIdx.x == 0 && live) i8_stage_fill(gemv_smem, L, a.hl, a.hls, a.I, pos0, cnt > 1 ? pos0 + 1 : -1);
       float acc[4][4] = {};
       if (!live) continue;
-      live = stq_warp_gemv_i8<4, true>(tb, nb, i8_cols(gemv_smem, L, nb, true, cnt > 1),
+      live = stq_warp_gemv_i8<4, true, true>(tb, nb, i8_cols(gemv_smem, L, nb, true, cnt > 1),
                                        reinterpret_cast<uint64_t*>(gemv_smem + L.xbar), xphase, lut8, acc, a.err);
       xphase ^= 1u;
       if (!live) continue;
