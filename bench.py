@@ -57,7 +57,7 @@ MEASURED_TRAFFIC_PER_EXPERT = {"gate_up_mx": (860.83e6 + 3.90e6) / 64}  # decode
 # and kernel build; an entry is removed when its kernel changes.
 MEASURED_TRAFFIC_PER_LAUNCH = {("stq_matvec", "gemv"): 2.09e6, ("w4a8_gemm", "gemm"): 7.54e6,
                                ("stq_pack_ls", "pack_ls"): 50.40e6 + 9.47e3,
-                               ("decode_stq", "gate_up"): 286.010880e6 + 1.244416e6,
+                               ("decode_stq", "gate_up"): 286.006528e6 + 1.105152e6,
                                ("prefill_w4a8", "gate_up_mx"): 3.74e9 + 69.87e6,
                                ("prefill_stq", "gate_up_stq_tc"): 1.60e9 + 63.20e6}
 
