@@ -362,7 +362,7 @@ def test_moe_stq_wide_range_activations(S):
     _check_layer(r, T, H, I, E, k)
 
 
-@pytest.mark.parametrize("T,H,I,E,k", [(8, 512, 256, 16, 2), (6, 1024, 512, 8, 2)])
+@pytest.mark.parametrize("T,H,I,E,k", [(8, 512, 256, 16, 2), (6, 1024, 512, 8, 2), (6, 768, 512, 8, 2)])
 def test_moe_stq_decode_integer_path_exactness(S, T, H, I, E, k):
     """Experts with one or two routed tokens (a layer averaging at most two per expert)
     run the integer GEMV: activations as a 22-bit fixed point per 256-k block, exact
@@ -395,6 +395,15 @@ def test_moe_stq_decode_integer_path_exactness(S, T, H, I, E, k):
     mag = torch.exp2(-torch.randint(0, 21, (T, H), generator=g, device=DEV).float())
     x = (W.bf16_normal((T, H), 1.0, DEV, 0, "exact-wide", "x").float() * mag).to(torch.bfloat16)
     r = _run_layer(S, T, H, I, E, k, True, ("exact", T, H, I, E, k), x=x)
+    _check_layer(r, T, H, I, E, k)
+
+
+def test_moe_stq_decode_large_h_takes_the_bf16_path(S):
+    """H = 8192: the integer path's activation stage (six limb rows of H + 64 bytes) would pass
+    the 47 KB shared-memory limit, so the layer runs the BF16 GEMV for every expert; results stay
+    within the layer tolerance."""
+    T, H, I, E, k = 4, 8192, 256, 8, 2
+    r = _run_layer(S, T, H, I, E, k, True, ("largeh", T, H, I, E, k))
     _check_layer(r, T, H, I, E, k)
 
 
