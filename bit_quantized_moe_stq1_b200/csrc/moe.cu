@@ -293,14 +293,15 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 }
 
 // One warp per token: softmax over E (max-shifted exp), top-k by probability with
-// ties to the lower id, weights renormalised over the chosen k.
+// ties to the lower id, weights renormalised over the chosen k.  Each lane holds
+// kMaxPer candidates (E <= 32 * kMaxPer): 8 for up to 256 experts, else 32.
+template <int kMaxPer>
 __global__ void router_topk_kernel(float* __restrict__ logits, int T, int E, int KS, int k,
                                    int32_t* __restrict__ ids, float* __restrict__ w) {
   stq_pdl_begin();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  constexpr int kMaxPer = 32;  // E <= 1024
   constexpr int kMaxKs = 8;
   float p[kMaxPer];
   const int per = (E + 31) / 32;
@@ -1247,8 +1248,10 @@ extern "C" stq_status moe_router_topk(const uint16_t* x, const uint16_t* w_route
   }
   if (st != STQ_OK) return st;
   StqTimed tm(STQ_K_ROUTER_TOPK, s);
-  return stq_launch(router_topk_kernel, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, logits, T, E, KS, k, topk_ids,
-                    topk_w);
+  return E <= 256 ? stq_launch(router_topk_kernel<8>, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, logits, T, E, KS, k,
+                               topk_ids, topk_w)
+                  : stq_launch(router_topk_kernel<32>, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, logits, T, E, KS,
+                               k, topk_ids, topk_w);
 }
 
 extern "C" stq_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E, int32_t* counts,
@@ -1304,6 +1307,8 @@ extern "C" stq_status moe_router_topk_static(const uint16_t* x, const uint16_t* 
   }
   if (st != STQ_OK) return st;
   StqTimed tm(STQ_K_ROUTER_TOPK, s);
-  return stq_launch(router_topk_kernel, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, scratch, T, E, KS, k, topk_ids,
-                    topk_w);
+  return E <= 256 ? stq_launch(router_topk_kernel<8>, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, scratch, T, E, KS, k,
+                               topk_ids, topk_w)
+                  : stq_launch(router_topk_kernel<32>, dim3(unsigned(ceil_div(T, 4))), dim3(128), 0, s, scratch, T, E, KS,
+                               k, topk_ids, topk_w);
 }
