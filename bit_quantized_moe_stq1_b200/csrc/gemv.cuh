@@ -254,6 +254,8 @@ struct StqI8Cols {
   const float* s1;   // ... of output column 2t+1
 };
 
+// One 1-D bulk copy global -> this CTA's shared memory (no multicast); `bytes` and both
+// addresses multiples of 16; completes on `bar`'s transaction count.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    tc::smem_u32(dst)),
