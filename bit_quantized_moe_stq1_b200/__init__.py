@@ -34,7 +34,8 @@ _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c
 
 class MoeDesc(ctypes.Structure):
     _fields_ = [("T", _i32), ("H", _i32), ("I", _i32), ("E", _i32), ("k", _i32),
-                ("out_fp32", _i32), ("add_residual", _i32), ("regime", _i32)]
+                ("out_fp32", _i32), ("add_residual", _i32), ("regime", _i32), ("norm_out", _i32),
+                ("norm_eps", ctypes.c_float)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -334,8 +335,10 @@ def moe_permute(topk_ids, E, err=None, stream=None):
 REGIME_AUTO, REGIME_DECODE, REGIME_PREFILL = 0, 1, 2
 
 
-def make_desc(T, H, I, E, k, out_fp32=False, add_residual=False, regime=REGIME_AUTO):
-    return MoeDesc(T, H, I, E, k, int(bool(out_fp32)), int(bool(add_residual)), int(regime))
+def make_desc(T, H, I, E, k, out_fp32=False, add_residual=False, regime=REGIME_AUTO, norm_eps=None):
+    """norm_eps: None, or the eps of an RMS normalisation of the output rows (bf16 output)."""
+    return MoeDesc(T, H, I, E, k, int(bool(out_fp32)), int(bool(add_residual)), int(regime),
+                   int(norm_eps is not None), float(norm_eps if norm_eps is not None else 0.0))
 
 
 def moe_workspace_bytes(desc):

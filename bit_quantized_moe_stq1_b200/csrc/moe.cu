@@ -852,6 +852,109 @@ __global__ void moe_combine_kernel(int T, int H, int k, int P, const float* __re
   }
 }
 
+// The combine and the stacked layers' RMS normalisation in one launch: one CTA of 1024
+// threads per token row.  Phase 1 forms every element exactly as moe_combine_kernel does
+// (slot-ordered FMAs, then the shared expert, then the residual, rounded to bf16) into
+// shared memory; phase 2 sums the squares of the bf16 row in rmsnorm_bf16_kernel's FP64
+// order (threads 0..255, uint4 chunks tid, tid + 256, ... ascending, an xor tree per warp,
+// the eight warp partials in warp order); phase 3 writes x * (1 / sqrt(ms + eps)) rounded
+// through FP32 to bf16.  The result has the bits of the two kernels run in sequence.  The
+// residual may alias y: a row's reads all come before its writes.
+__global__ void __launch_bounds__(1024) moe_combine_norm_kernel(int T, int H, int k, int P, const float* __restrict__ Y,
+                                                                const int32_t* __restrict__ inv,
+                                                                const float* __restrict__ topk_w, int has_shared,
+                                                                const uint16_t* resid, uint16_t* y, float eps,
+                                                                int32_t* err) {
+  extern __shared__ uint4 srow[];  // the bf16 row, H / 8 chunks
+  __shared__ double part[8];
+  __shared__ double s_scale;
+  __shared__ int s_pos[32];        // the row's k slots (k <= 32): sorted position, -1 = none
+  __shared__ float s_w[32];
+  stq_pdl_begin();
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h4 = H / 4, n8 = H / 8;
+  if (tid < k) {
+    const int pos = inv[size_t(t) * k + tid];
+    s_pos[tid] = (pos < 0 || !STQ_DCHECK(pos < P, err)) ? -1 : pos;
+    s_w[tid] = topk_w[size_t(t) * k + tid];
+  }
+  __syncthreads();
+  uint2* row2 = reinterpret_cast<uint2*>(srow);
+  for (int c = tid; c < h4; c += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // eight slots' loads at a time, then their FMAs in slot order
+    for (int s0 = 0; s0 < k; s0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int pos = s0 + j < k ? s_pos[s0 + j] : -1;
+        v[j] = pos >= 0 ? reinterpret_cast<const float4*>(Y + size_t(pos) * H)[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (s0 + j >= k || s_pos[s0 + j] < 0) continue;
+        const float w = s_w[s0 + j];
+        acc.x = fmaf(w, v[j].x, acc.x);
+        acc.y = fmaf(w, v[j].y, acc.y);
+        acc.z = fmaf(w, v[j].z, acc.z);
+        acc.w = fmaf(w, v[j].w, acc.w);
+      }
+    }
+    if (has_shared) {
+      const float4 v = reinterpret_cast<const float4*>(Y + size_t(P + t) * H)[c];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if (resid != nullptr) {
+      const uint2 r = reinterpret_cast<const uint2*>(resid + size_t(t) * H)[c];
+      acc.x += bf16_bits_to_float(r.x & 0xFFFFu);
+      acc.y += bf16_bits_to_float(r.x >> 16);
+      acc.z += bf16_bits_to_float(r.y & 0xFFFFu);
+      acc.w += bf16_bits_to_float(r.y >> 16);
+    }
+    row2[c] = make_uint2(uint32_t(float_to_bf16_bits(acc.x)) | (uint32_t(float_to_bf16_bits(acc.y)) << 16),
+                         uint32_t(float_to_bf16_bits(acc.z)) | (uint32_t(float_to_bf16_bits(acc.w)) << 16));
+  }
+  __syncthreads();
+  if (tid < 256) {
+    double ss = 0.0;
+    for (int i = tid; i < n8; i += 256) {
+      const uint4 v = srow[i];
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const double a = bf16_bits_to_float(w4[j] & 0xFFFFu), b = bf16_bits_to_float(w4[j] >> 16);
+        ss = fma(a, a, ss);
+        ss = fma(b, b, ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(kFull, ss, o);
+    if (lane == 0) part[warp] = ss;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double tot = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += part[w];
+    s_scale = 1.0 / sqrt(tot / double(H) + double(eps));
+  }
+  __syncthreads();
+  const double r = s_scale;
+  uint4* yr = reinterpret_cast<uint4*>(y + size_t(t) * H);
+  for (int i = tid; i < n8; i += blockDim.x) {
+    const uint4 v = srow[i];
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = __double2float_rn(double(bf16_bits_to_float(w4[j] & 0xFFFFu)) * r);
+      const float b = __double2float_rn(double(bf16_bits_to_float(w4[j] >> 16)) * r);
+      o[j] = uint32_t(float_to_bf16_bits(a)) | (uint32_t(float_to_bf16_bits(b)) << 16);
+    }
+    yr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 }  // namespace
 
 // ----------------------------------------------------------------------------- host side
@@ -932,7 +1035,8 @@ static bool desc_ok(const moe_desc* d) {
   // P = T*k below 2^30 (as moe_permute): pair and row indices, P + T included, stay in int32
   return d && d->T >= 0 && d->H > 0 && d->I > 0 && d->E > 0 && d->E <= 1024 && d->k > 0 && d->k <= 32 &&
          d->k <= d->E && int64_t(d->T) * d->k < (int64_t(1) << 30) && d->regime >= STQ_REGIME_AUTO &&
-         d->regime <= STQ_REGIME_PREFILL;
+         d->regime <= STQ_REGIME_PREFILL &&
+         (d->norm_out == 0 || (d->norm_out == 1 && d->out_fp32 == 0 && d->norm_eps >= 0.f && d->norm_eps < 3.0e38f));
 }
 
 extern "C" size_t moe_workspace_bytes(const moe_desc* d) {
@@ -1020,14 +1124,32 @@ stq_status moe_launch_permute(const int32_t* ids, int P, int E, const MoeWs& ws,
   return stq_launch(moe_permute_kernel, dim3(1), dim3(1024), smem, s, ids, P, E, ws);
 }
 
+// Rows up to this many elements take the fused combine + RMS normalisation (the row's
+// bf16 values in shared memory, below the 48 KB default).
+constexpr int kCombineNormMaxH = 23 * 1024;
+
 stq_status moe_launch_combine(const moe_desc& d, int P, const MoeWs& ws, const float* topk_w, bool has_shared,
                               const uint16_t* x, void* y, cudaStream_t s) {
   const int64_t n = int64_t(d.T) * (d.H / 4);
   if (n == 0) return STQ_OK;
-  StqTimed tm(STQ_K_COMBINE, s);
-  return stq_launch(moe_combine_kernel, dim3(unsigned(ceil_div<int64_t>(n, 256))), dim3(256), 0, s, d.T, d.H, d.k, P,
+  if (d.norm_out && d.H <= kCombineNormMaxH) {
+    StqTimed tm(STQ_K_COMBINE, s);
+    return stq_launch(moe_combine_norm_kernel, dim3(unsigned(d.T)), dim3(1024), size_t(d.H) * 2, s, d.T, d.H, d.k, P,
+                      static_cast<const float*>(ws.Y), static_cast<const int32_t*>(ws.inv), topk_w,
+                      has_shared ? 1 : 0, d.add_residual ? x : nullptr, static_cast<uint16_t*>(y), d.norm_eps,
+                      ws.err);
+  }
+  stq_status st;
+  {
+    StqTimed tm(STQ_K_COMBINE, s);
+    st = stq_launch(moe_combine_kernel, dim3(unsigned(ceil_div<int64_t>(n, 256))), dim3(256), 0, s, d.T, d.H, d.k, P,
                     static_cast<const float*>(ws.Y), static_cast<const int32_t*>(ws.inv), topk_w, has_shared ? 1 : 0,
                     d.add_residual ? x : nullptr, y, d.out_fp32, ws.err);
+  }
+  if (st != STQ_OK || !d.norm_out) return st;
+  // rows too wide for the fused kernel: the normalisation as its own launch
+  return stq_rmsnorm_bf16(static_cast<const uint16_t*>(y), d.T, d.H, d.norm_eps, static_cast<uint16_t*>(y),
+                          reinterpret_cast<stq_stream_t>(s));
 }
 
 // A library-owned stream per device, created on first use: the MXFP8 shared expert

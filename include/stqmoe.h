@@ -271,6 +271,11 @@ typedef struct {
   int32_t out_fp32;         /* 1: y is float32 [T, H]; 0: y is bf16 [T, H]      */
   int32_t add_residual;     /* 1: y += x                                         */
   int32_t regime;           /* STQ_REGIME_* (STQ1_0 experts)                     */
+  int32_t norm_out;         /* 1: y = RMSNorm(y) after the residual: unit gain,
+                               y / sqrt(mean(y^2) + norm_eps) per token row over the
+                               bf16-rounded y, the same bits as stq_rmsnorm_bf16 on
+                               the unnormalised output; requires out_fp32 = 0      */
+  float norm_eps;           /* eps of norm_out, finite and >= 0                  */
 } moe_desc;
 
 /* Bytes of device workspace moe_expert_forward needs for `d` (256-byte aligned

@@ -58,6 +58,11 @@ def test_binding_loads_and_host_side_calls(built):
     # routed h (bf16) + Y (f32) dominate: (P+T)*I*2 + (P+T)*H*4
     assert ws >= (64 + 8) * 2048 * 2 + (64 + 8) * 6144 * 4
     assert S.moe_workspace_bytes(S.make_desc(8, 6144, 2048, 256, 300)) == 0       # k > E
+    # the fused RMS normalisation wants a bf16 output and a finite eps >= 0
+    assert S.moe_workspace_bytes(S.make_desc(8, 512, 256, 8, 2, norm_eps=1e-6)) > 0
+    assert S.moe_workspace_bytes(S.make_desc(8, 512, 256, 8, 2, out_fp32=True, norm_eps=1e-6)) == 0
+    assert S.moe_workspace_bytes(S.make_desc(8, 512, 256, 8, 2, norm_eps=-1.0)) == 0
+    assert S.moe_workspace_bytes(S.make_desc(8, 512, 256, 8, 2, norm_eps=float("nan"))) == 0
     # T*k < 2^30 keeps pair and row indices (P + T) in int32
     assert S.moe_workspace_bytes(S.make_desc((1 << 27) - 1, 256, 256, 256, 8)) > 0
     assert S.moe_workspace_bytes(S.make_desc(1 << 27, 256, 256, 256, 8)) == 0
@@ -77,7 +82,8 @@ C_LAYOUT = r"""
 int main(void) {
   printf("moe_desc %zu\nmoe_weights %zu\n", sizeof(moe_desc), sizeof(moe_weights));
   F(moe_desc, T); F(moe_desc, H); F(moe_desc, I); F(moe_desc, E); F(moe_desc, k);
-  F(moe_desc, out_fp32); F(moe_desc, add_residual); F(moe_desc, regime);
+  F(moe_desc, out_fp32); F(moe_desc, add_residual); F(moe_desc, regime); F(moe_desc, norm_out);
+  F(moe_desc, norm_eps);
   F(moe_weights, fmt); F(moe_weights, gate); F(moe_weights, up); F(moe_weights, down);
   F(moe_weights, gate_sc); F(moe_weights, up_sc); F(moe_weights, down_sc);
   F(moe_weights, sh_gate); F(moe_weights, sh_up); F(moe_weights, sh_down); F(moe_weights, sh_fmt);

@@ -59,3 +59,37 @@ def test_rmsnorm_empty_and_bad_args(S):
     assert S.rmsnorm_bf16(x).shape == (0, 64)
     with pytest.raises(RuntimeError):
         S.rmsnorm_bf16(torch.zeros((2, 12), dtype=torch.bfloat16, device=DEV))
+
+
+def _bits16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy()
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [(32, 6144, 256, 16, 4), (5, 768, 256, 8, 2), (3, 24576, 256, 4, 2)])
+def test_norm_out_matches_the_separate_normalisation(S, T, H, I, E, k):
+    """moe_desc.norm_out: the combine with the RMS normalisation fused (or, past the fused
+    kernel's row width, the two launches) gives the bits of the unnormalised layer output
+    followed by stq_rmsnorm_bf16, with the residual read from x and with y aliasing x."""
+    tag = ("normout", T, H, I, E, k)
+    gw = [W.stq_grid_weights(E * I, H, DEV, 0, *tag, "g"), W.stq_grid_weights(E * I, H, DEV, 0, *tag, "u"),
+          W.stq_grid_weights(E * H, I, DEV, 0, *tag, "d")]
+    packs = [S.stq1_pack(m) for m in gw]
+    sh = [W.bf16_normal((I, H), 0.02, DEV, 0, *tag, "sg"), W.bf16_normal((I, H), 0.02, DEV, 0, *tag, "su"),
+          W.bf16_normal((H, I), 0.02, DEV, 0, *tag, "sd")]
+    ew = S.ExpertWeights(S.FMT_STQ1_0, *packs, None, None, None, *sh)
+    x = W.bf16_normal((T, H), 1.0, DEV, 0, *tag, "x")
+    ids, tw = W.uniform_routing(T, E, k, DEV, 0, *tag, "ids")
+    plain = S.make_desc(T, H, I, E, k, add_residual=True)
+    fused = S.make_desc(T, H, I, E, k, add_residual=True, norm_eps=W.STACK_RMS_EPS)
+    ws = torch.zeros(S.moe_workspace_bytes(plain), dtype=torch.uint8, device=DEV)
+    assert S.moe_workspace_bytes(fused) == S.moe_workspace_bytes(plain)
+    ref = torch.empty((T, H), dtype=torch.bfloat16, device=DEV)
+    S.moe_expert_forward(plain, x, ids, tw, ew, ref, ws)
+    S.rmsnorm_bf16(ref, W.STACK_RMS_EPS, y=ref)
+    got = torch.empty_like(ref)
+    S.moe_expert_forward(fused, x, ids, tw, ew, got, ws)
+    assert S.moe_get_device_error(ws) == 0
+    assert np.array_equal(_bits16(got), _bits16(ref))
+    inplace = x.clone()
+    S.moe_expert_forward(fused, inplace, ids, tw, ew, inplace, ws)
+    assert np.array_equal(_bits16(inplace), _bits16(ref))
