@@ -65,16 +65,15 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int* wsum, int* total
 
 // ----------------------------------------------------------------------------- permute
 
-__global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __restrict__ ids, int P, int E,
-                                                           MoeWs ws) {
-  extern __shared__ int32_t sm[];
+// The grouping by one CTA of 1024 threads; sm: 34 E ints of shared memory.
+__device__ __forceinline__ void permute_cta(const int32_t* __restrict__ ids, int P, int E, const MoeWs& ws,
+                                            int32_t* sm) {
   int32_t* cnt = sm;             // [E]
   int32_t* cursor = sm + E;      // [E]
   int32_t* whist = sm + 2 * E;   // [32][E]
   __shared__ int wsum[32];
   __shared__ int total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  stq_pdl_begin();
   for (int e = tid; e < E; e += 1024) cnt[e] = 0;
   // counters 0-2 (the STQ1_0 decode kernels); counter 3 belongs to the shared expert, which
   // may run on another stream and is zeroed there (shared_gateup_wide_kernel)
@@ -134,6 +133,13 @@ __global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __rest
     }
     __syncthreads();
   }
+}
+
+__global__ void __launch_bounds__(1024) moe_permute_kernel(const int32_t* __restrict__ ids, int P, int E,
+                                                           MoeWs ws) {
+  extern __shared__ int32_t sm[];
+  stq_pdl_begin();
+  permute_cta(ids, P, E, ws, sm);
 }
 
 // The same grouping over many CTAs (large P): chunks of 1024 pairs.
@@ -514,12 +520,9 @@ __device__ __forceinline__ int next_item(int32_t* counter, int* slot) {
 // q = m * 2^(e' - Eb + 14), rounded to nearest, ties to even, when e' < Eb - 14; |q| < 2^22,
 // and q = hi*2^16 + mid*2^8 + lo with every limb in [-128, 127].  A block holding an Inf or
 // NaN gets a NaN scale.  One warp per block; lane l takes elements 8l..8l+7.
-__global__ void __launch_bounds__(256) stq_act_limbs_kernel(const uint16_t* __restrict__ src, int64_t rows, int K,
-                                                           int8_t* __restrict__ limbs, float* __restrict__ scales) {
-  stq_pdl_begin();
+__device__ __forceinline__ void act_limbs_warp(const uint16_t* __restrict__ src, int K, int8_t* __restrict__ limbs,
+                                               float* __restrict__ scales, int64_t wid) {
   const int nb = K / 256, lane = threadIdx.x & 31;
-  const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (wid >= rows * nb) return;  // whole warps
   const int64_t row = wid / nb;
   const int b = int(wid - row * nb);
   const uint4 v = *reinterpret_cast<const uint4*>(src + row * K + 256 * b + 8 * lane);
@@ -562,6 +565,29 @@ __global__ void __launch_bounds__(256) stq_act_limbs_kernel(const uint16_t* __re
     *reinterpret_cast<uint2*>(limbs + (row * 3 + l) * K + 256 * b + off) = make_uint2(lb[l][0], lb[l][1]);
   if (lane < 3)
     scales[row * pitch + lane * nb + b] = eb == 255u ? __int_as_float(0x7FC00000) : ldexpf(1.f, int(eb) - 132 - 8 * lane);
+}
+
+__global__ void __launch_bounds__(256) stq_act_limbs_kernel(const uint16_t* __restrict__ src, int64_t rows, int K,
+                                                           int8_t* __restrict__ limbs, float* __restrict__ scales) {
+  stq_pdl_begin();
+  const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (wid < rows * (K / 256)) act_limbs_warp(src, K, limbs, scales, wid);  // whole warps
+}
+
+// The grouping (CTA 0, as moe_permute_kernel) and the limbs of x (the other CTAs, one warp
+// per 256-k block, as stq_act_limbs_kernel) in one launch: the two depend on separate
+// inputs.
+__global__ void __launch_bounds__(1024) moe_permute_limbs_kernel(const int32_t* __restrict__ ids, int P, int E, MoeWs ws,
+                                                                 const uint16_t* __restrict__ x, int T, int H,
+                                                                 int8_t* __restrict__ xl, float* __restrict__ xls) {
+  extern __shared__ int32_t sm[];
+  stq_pdl_begin();
+  if (blockIdx.x == 0) {
+    permute_cta(ids, P, E, ws, sm);
+    return;
+  }
+  const int64_t wid = int64_t(blockIdx.x - 1) * 32 + (threadIdx.x >> 5);
+  if (wid < int64_t(T) * (H / 256)) act_limbs_warp(x, H, xl, xls, wid);
 }
 
 // Items with at most this many tokens take the integer GEMV (two tokens per mma).
@@ -1213,12 +1239,12 @@ stq_status moe_launch_act_limbs(const uint16_t* src, int64_t rows, int K, int8_t
 // limbs of x made before gate/up, those of h between gate/up and down) or without it.
 template <bool I8>
 stq_status launch_stq_decode(MoeArgs a, const moe_desc& d, const MoeWs& ws, const uint16_t* x, int P, int slots,
-                             bool shared_bf16, cudaStream_t s) {
+                             bool shared_bf16, bool x_limbs_done, cudaStream_t s) {
   stq_status st;
   const int smem_gu = I8 ? gemv_smem_layout(d.H).total : kGemvRedBytes;
   const int smem_dn = I8 ? gemv_smem_layout(d.I).total : kGemvRedBytes;
   if (I8) {
-    if ((st = moe_launch_act_limbs(x, d.T, d.H, ws.xl, ws.xls, s)) != STQ_OK) return st;
+    if (!x_limbs_done && (st = moe_launch_act_limbs(x, d.T, d.H, ws.xl, ws.xls, s)) != STQ_OK) return st;
     a.xl = ws.xl;
     a.xls = ws.xls;
   }
@@ -1326,17 +1352,30 @@ extern "C" stq_status moe_expert_forward(const moe_desc* d, const uint16_t* x, c
     if (st != STQ_OK) return st;
     if (cudaEventRecord(fj->join, side->stream) != cudaSuccess) return STQ_ERR_CUDA;
   }
-  if ((st = moe_launch_permute(topk_ids, P, d->E, ws, s)) != STQ_OK) return st;
+  // The STQ1_0 decode regime's integer GEMV serves items of at most two tokens; its limbs
+  // are made when the average expert has at most two and the activation stages fit in
+  // kGemvSmemLimit.  With the one-CTA grouping, x's limbs come from the same launch.
+  const bool i8 = stq_decode && int64_t(P) <= kI8LimbsAvgTokens * int64_t(slots) &&
+                  gemv_smem_layout(d->H).total <= kGemvSmemLimit && gemv_smem_layout(d->I).total <= kGemvSmemLimit;
+  const bool fused_limbs = i8 && !(P >= kPermuteMultiCta && ws.chist != nullptr);
+  if (fused_limbs) {
+    const size_t smem = size_t(34) * d->E * sizeof(int32_t);
+    static StqSmemOptIn optin;
+    if ((st = optin.ensure(moe_permute_limbs_kernel, int(smem))) != STQ_OK) return st;
+    const int64_t warps = int64_t(d->T) * (d->H / 256);
+    StqTimed tm(STQ_K_PERMUTE, s);
+    st = stq_launch(moe_permute_limbs_kernel, dim3(unsigned(1 + ceil_div<int64_t>(warps, 32))), dim3(1024), smem, s,
+                    topk_ids, P, d->E, ws, x, d->T, d->H, ws.xl, ws.xls);
+  } else {
+    st = moe_launch_permute(topk_ids, P, d->E, ws, s);
+  }
+  if (st != STQ_OK) return st;
 
   if (w->fmt == STQ_FMT_STQ1_0 && prefill) {
     if ((st = moe_stq_prefill_experts(a, slots, s)) != STQ_OK) return st;
   } else if (w->fmt == STQ_FMT_STQ1_0) {
-    // The integer GEMV serves items of at most two tokens; its limbs are made when the
-    // average expert has at most four and the activation stages fit in kGemvSmemLimit.
-    const bool i8 = int64_t(P) <= kI8LimbsAvgTokens * int64_t(slots) &&
-                    gemv_smem_layout(d->H).total <= kGemvSmemLimit && gemv_smem_layout(d->I).total <= kGemvSmemLimit;
-    st = i8 ? launch_stq_decode<true>(a, *d, ws, x, P, slots, shared_bf16, s)
-            : launch_stq_decode<false>(a, *d, ws, x, P, slots, shared_bf16, s);
+    st = i8 ? launch_stq_decode<true>(a, *d, ws, x, P, slots, shared_bf16, fused_limbs, s)
+            : launch_stq_decode<false>(a, *d, ws, x, P, slots, shared_bf16, false, s);
     if (st != STQ_OK) return st;
   } else {
     st = moe_mx_experts(a, slots, s);
