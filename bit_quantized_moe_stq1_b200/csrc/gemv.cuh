@@ -183,7 +183,8 @@ __device__ __forceinline__ void stq_warp_gemv(const uint8_t* const (&tb)[NT], in
 // entry is then a finished A-fragment register of mma.sync m16n8k32 s8 (four consecutive k
 // of one row), so a 5-bit code costs one shift and one shuffle and no byte permutes.  The
 // activations enter as three signed 8-bit limbs of a fixed-point value per 256-k block
-// (written by stq_act_limbs_kernel): v = q * 2^(Eb - 148), q = hi*2^16 + mid*2^8 + lo, with
+// (written by stq_act_limbs_kernel, x's by the grouping's launch when it can take them):
+// v = q * 2^(Eb - 148), q = hi*2^16 + mid*2^8 + lo, with
 // Eb the largest bf16 exponent field of the block.  Every element within 2^14 of the
 // block's largest magnitude is exact; smaller ones are rounded to the nearest multiple of
 // 2^(Eb - 148), an absolute error of at most 2^-22 of the block's largest magnitude.  The
